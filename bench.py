@@ -1,0 +1,442 @@
+"""Throughput benchmark of the MoE FFN forward layer on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path (route -> dispatch -> expert up/down -> combine)
+over one batch of the workload, enqueued through the C ABI with CUDA events between the
+kernels (the same kernels moe_forward launches). Inputs are resident in HBM; L2 is flushed
+(a 512 MiB write) between timed steps, outside the per-step events. Rank 0 prints one JSON
+line. With N>1 (torchrun) every rank runs an independent replica on its own GPU (the layer
+has no data-path collective); value = tokens of all ranks / max-over-ranks time.
+
+--impl reference times the CPU oracle on the host cores (a bounded token sample of the same
+workload) and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE fwd tokens/s; grouped-GEMM TFLOP/s & %bf16 peak; route/combine % HBM BW"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ small host helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(cfg) -> str:
+    act = {0: "SiLU", 1: "GELU(erf)", 2: "GELU(tanh)"}[cfg.activation]
+    s = (f"{cfg.name}: N={cfg.N} D={cfg.D} F={cfg.F} E={cfg.E} k={cfg.k} {act} "
+         f"{'renormalised' if cfg.renormalize else 'no-renorm'} top-k")
+    if cfg.capacity_factor > 0:
+        s += f", CF={cfg.capacity_factor}"
+    return s
+
+
+def dtype_name(cfg) -> str:
+    from top_routing_expert_fp32_b200 import configs
+    return "bf16" if cfg.dtype == configs.DTYPE_BF16 else "f32"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device) -> float:
+    """Max over ranks (all ranks call it, same order)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and getattr(device, "type", "cpu") == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(tokens_per_rank: int, world: int, max_ms_total: float, steps: int) -> dict:
+    """Whole-job throughput from the slowest rank's time."""
+    ms_per_step = max_ms_total / steps
+    return dict(value=tokens_per_rank * world * steps / (max_ms_total / 1e3),
+                ms_per_step=ms_per_step)
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a background thread."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.05):
+        self.samples = []  # (t, sm_mhz, reasons_mask)
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                if not uuid.startswith("GPU-"):
+                    uuid = "GPU-" + uuid
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.time(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if len(win) < 3:
+            win = self.samples
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = sorted({name for _, _, m in win for name, bit in self.REASONS.items() if m & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win)}
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e["source_sha"] != source_hash(e["sources"]):
+            return None
+        return e["bytes_per_launch"]
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_tokens_per_s(cfg, budget_s: float = 12.0):
+    """The oracle (as it stands) on a bounded token sample of the workload. Without capacity the
+    tokens are independent, so a prefix of the batch is the same computation per token; with
+    capacity the sample is its own batch of n tokens (capacity recomputed for n)."""
+    import numpy as np
+    import torch
+    import oracle
+    from top_routing_expert_fp32_b200 import configs, inputs
+
+    inp = inputs.make_inputs(cfg, "cpu")
+    od = oracle.BF16 if cfg.dtype == configs.DTYPE_BF16 else oracle.F32
+    X = oracle.torch_to_numpy(inp.X)
+    Wr = inp.W_r.numpy()
+    b = None if inp.bias is None else inp.bias.numpy()
+    W1, W2, W3 = (oracle.torch_to_numpy(w) for w in (inp.W1, inp.W2, inp.W3))
+
+    def run(n):
+        t = time.perf_counter()
+        oracle.forward(X[:n], Wr, b, W1, W2, W3, k=cfg.k, cf=cfg.capacity_factor,
+                       renorm=cfg.renormalize, act=cfg.activation, dtype=od)
+        return time.perf_counter() - t
+
+    n = min(cfg.N, max(1, oracle.num_threads()))
+    dt = run(n)
+    while dt < budget_s / 8 and n < cfg.N:
+        n = min(cfg.N, n * 2)
+        dt = run(n)
+    if dt < budget_s / 2 and n < cfg.N:
+        n = min(cfg.N, max(n + 1, int(n * (budget_s / 2) / max(dt, 1e-3))))
+        dt = run(n)
+    return dict(value=n / dt, unit="tokens/s", cores=oracle.num_threads(), kind="oracle",
+                sample=f"first {n} of {cfg.N} tokens of the workload, full forward in fp64, "
+                       f"{dt:.1f} s wall")
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, cfg, world, rank, device):
+    import torch
+    from top_routing_expert_fp32_b200 import abi, configs, inputs
+
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+    inp = inputs.make_inputs(cfg, device, seed=cfg.seed + rank * 0)
+    N, E, k, D, F = cfg.N, cfg.E, cfg.k, cfg.D, cfg.F
+    p = abi.problem(cfg)
+    ws = abi.workspace(p, device)
+    tdt = inp.X.dtype
+    R = N * k
+    logits = None
+    idx = torch.empty((N, k), dtype=torch.int32, device=device)
+    gate = torch.empty((N, k), dtype=torch.float32, device=device)
+    load = torch.empty((E,), dtype=torch.int32, device=device)
+    offsets = torch.empty((E + 1,), dtype=torch.int32, device=device)
+    pos = torch.empty((N, k), dtype=torch.int32, device=device)
+    dropped = torch.empty((N, k), dtype=torch.uint8, device=device)
+    row_token = torch.empty((R,), dtype=torch.int32, device=device)
+    X_perm = torch.empty((R, D), dtype=tdt, device=device)
+    H = torch.empty((R, F), dtype=tdt, device=device)
+    Y = torch.empty((R, D), dtype=tdt, device=device)
+    out = torch.empty((N, D), dtype=tdt, device=device)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    names = ["route", "dispatch", "up", "down", "combine"]
+    launches = {"route": 1, "dispatch": 3, "up": 1, "down": 1, "combine": 1}
+
+    def step(ev):
+        ev[0].record(stream)
+        abi.route(p, inp.X, inp.W_r, inp.bias, logits, idx, gate, None, ws)
+        ev[1].record(stream)
+        abi.dispatch(p, inp.X, idx, load, offsets, pos, dropped, row_token, X_perm, ws)
+        ev[2].record(stream)
+        abi.expert_up(p, X_perm, offsets, inp.W1, inp.W2, H, ws)
+        ev[3].record(stream)
+        abi.expert_down(p, H, offsets, inp.W3, Y, ws)
+        ev[4].record(stream)
+        abi.combine(p, Y, idx, gate, offsets, pos, dropped, out)
+        ev[5].record(stream)
+
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    for _ in range(args.warmup):
+        step(new_events())
+        flush.fill_(1)
+    torch.cuda.synchronize(device)
+    if abi.device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    sampler = ClockSampler(device.index).start()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    t_wall0 = time.time()
+    evs = []
+    for _ in range(args.steps):
+        ev = new_events()
+        step(ev)
+        evs.append(ev)
+        flush.fill_(1)   # outside the step's events: evicts X, H, Y from L2
+    torch.cuda.synchronize(device)
+    barrier(device)
+    t_wall1 = time.time()
+    sampler.stop()
+    if abi.device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    per = {n: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, n in enumerate(names)}
+    total_ms = sum(ev[0].elapsed_time(ev[5]) for ev in evs)
+    max_total = reduce_max(total_ms, device)
+    agg = aggregate(N, world, max_total, args.steps)
+    mean = {n: sum(v) / len(v) for n, v in per.items()}
+
+    kept = int(offsets[E].item())
+    tokens_with_kept = int((dropped == 0).any(1).sum().item())
+    es = 2 if cfg.dtype == configs.DTYPE_BF16 else 4
+    flops_up = 4.0 * kept * D * F
+    flops_down = 2.0 * kept * D * F
+    bytes_route = N * D * es + D * E * 4 + N * k * 8
+    bytes_gather = (tokens_with_kept + kept) * D * es
+    bytes_combine = kept * D * es + N * D * es + N * k * 13
+    hbm = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops"]
+    kern = {
+        "route": {"ms": mean["route"], "GB/s": bytes_route / mean["route"] / 1e6},
+        "dispatch": {"ms": mean["dispatch"], "gather_GB/s_lower_bound":
+                     bytes_gather / mean["dispatch"] / 1e6},
+        "up": {"ms": mean["up"], "TFLOP/s": flops_up / mean["up"] / 1e9},
+        "down": {"ms": mean["down"], "TFLOP/s": flops_down / mean["down"] / 1e9},
+        "combine": {"ms": mean["combine"], "GB/s": bytes_combine / mean["combine"] / 1e6},
+    }
+    for n in ("route", "combine"):
+        kern[n]["frac_hbm"] = kern[n]["GB/s"] / hbm
+        kern[n]["frac_8TBs"] = kern[n]["GB/s"] / 8000.0
+    for n in ("up", "down"):
+        kern[n]["frac_bf16_peak"] = kern[n]["TFLOP/s"] / tc
+    ffn_ms = mean["up"] + mean["down"]
+    gemm_tflops = 6.0 * kept * D * F / ffn_ms / 1e9
+
+    if cfg.dtype == configs.DTYPE_BF16 and kept >= 4 * 128:
+        dom = "up"
+        roof = {"kernel": "grouped_gemm_sm100<dual> (expert up-projection + gating)",
+                "bound": "tensor", "achieved": kern["up"]["TFLOP/s"], "peak": tc,
+                "unit": "TFLOP/s", "frac": kern["up"]["TFLOP/s"] / tc,
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
+                if peak_src == "measured" else "fallback",
+                "flops_per_launch": flops_up}
+    else:
+        # decode-sized / fp32: bound by streaming the expert weights through HBM
+        dom = "up"
+        wbytes = 2.0 * E * D * F * es
+        gbs = wbytes / mean["up"] / 1e6
+        roof = {"kernel": "expert up-projection (weight streaming)", "bound": "hbm",
+                "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "peak_source": peak_src, "bytes_per_launch": wbytes}
+    roof["traffic"] = traffic_from_profile("up", cfg.name)
+
+    # end-to-end through the public host-buffer entry point
+    ws_h = abi.workspace(p, device, host=True)
+    xh = inp.X.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
+    barrier(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e_total = 0.0
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0.record(stream)
+        abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
+        e1.record(stream)
+        e1.synchronize()
+        e_total += e0.elapsed_time(e1)
+    e_max = reduce_max(e_total, device)
+    e2e_value = N * world * args.steps / (e_max / 1e3)
+    h2d = N * D * es
+    d2h = N * D * es
+    barrier(device)
+
+    line = {
+        "metric": METRIC, "value": agg["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": agg["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_name(cfg),
+        "data": "synthetic, seeded: X~N(0,1), W_r/W1/W2~N(0,1/D), W3~N(0,1/F)"
+                + (", bias~N(0,2)" if cfg.router_bias_var > 0 else ""),
+        "config": {"workload": workload_desc(cfg), "tokens_per_gpu": N,
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "flushed between steps (512 MiB write outside the step events)",
+                   "kept_records": kept,
+                   "grouped_gemm_TFLOP/s": gemm_tflops,
+                   "grouped_gemm_frac_bf16_peak": gemm_tflops / tc,
+                   "kernels": kern},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "api": "moe_forward_host (pinned host X in, host out; copies in the timed region)"},
+        "gpu_launches": sum(launches.values()) * args.steps,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    return line
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.CONFIGS[args.workload or configs.BENCH_WORKLOAD]
+    world, rank, local = dist_env()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = oracle_tokens_per_s(cfg, budget_s=min(20.0, 6.0 * args.steps))
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * cfg.N / cb["value"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic, seeded (same inputs as the GPU arm)",
+                "config": {"workload": workload_desc(cfg)},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    line = run_gpu(args, cfg, world, rank, device)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = oracle_tokens_per_s(cfg)
+        else:
+            line["cpu_baseline"] = None
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

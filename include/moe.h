@@ -1,0 +1,218 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts FFN forward library.
+ *
+ * The layer (one data-parallel hot path, single GPU):
+ *   logits = X W_r (+bias) in fp32 -> softmax over E -> top-k -> gates (optionally
+ *   renormalised over the selected set) -> per-expert load -> capacity ceil(CF*N*k/E) with a
+ *   slot-major drop mask -> expert-contiguous permutation of the N*k records -> per-expert
+ *   gated FFN [act(x W1_e) (.) (x W2_e)] W3_e -> gate-weighted sum back to the N tokens.
+ *
+ * Sources, cited by page title and section:
+ *   - Grok-1 book ch.5 "MoE routing & experts": 5.2 (fp32 router x.W_r, softmax, TopK),
+ *     5.2.3 (softmax then top-k, no renormalisation), 5.3.2 (expert weights stacked with a
+ *     leading expert dimension), 5.3.5 (GeGLU expert, gate-weighted sum over k).
+ *   - LLMs-from-scratch ch.12 "MoE": 12.1 (X:[B,T,D], W_r:[D,E], top-k softmax over the
+ *     selected set, f_e(x) = [SiLU(x W1_e) (.) (x W2_e)] W3_e, W1,W2:[D,F], W3:[F,D]),
+ *     12.2 (flatten to [N,D], N*k dispatch records, accumulate the k contributions).
+ *   - MoE formula-to-code walkthrough: 1.1 (stable softmax), 1.2 (top-k ordered by
+ *     descending score, renormalisation), 1.3 (expert load), 2.1 (balance loss), 3.1
+ *     (capacity), 3.2 (dispatch with a dropped mask), 3.3 (drop rate).
+ *   - MoE series (GShard/Mixtral/Switch): 2.2 (an overflowed slot contributes nothing).
+ *
+ * Conventions shared by every entry point:
+ *   - Array pointers are DEVICE pointers unless the entry point says otherwise. The caller
+ *     allocates and owns every buffer, including the workspace; the library never
+ *     allocates device memory.
+ *   - Layouts are dense row-major. X [N,D]; W_r [D,E] fp32; bias [E] fp32; W1, W2 [E,D,F]
+ *     (W1 = activated branch, Grok "linear"; W2 = linear branch, Grok "linear_v");
+ *     W3 [E,F,D] (Grok "linear_1"); logits [N,E] fp32; topk_idx [N,k] int32 (rank 0 = the
+ *     largest logit); topk_gate [N,k] fp32; load [E] int32; offsets [E+1] int32;
+ *     pos [N,k] int32; dropped [N,k] uint8; row_token [N*k] int32; X_perm [N*k,D];
+ *     H [N*k,F]; Y [N*k,D]; out [N,D].
+ *   - X, W1..W3, X_perm, H, Y and out all have the problem's dtype (fp32 or bf16).
+ *   - Every device pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is enqueued
+ *     asynchronously; nothing synchronises the host except where stated.
+ *   - Errors: arguments are checked on the host before anything is enqueued; a bad
+ *     argument returns MOE_ERR_INVALID_ARG and a shape outside the kernels' support returns
+ *     MOE_ERR_UNSUPPORTED, in both cases with nothing enqueued. A failed CUDA call returns
+ *     MOE_ERR_CUDA (work enqueued before it by the same call stays enqueued).
+ *     moe_last_error() gives a message for the calling thread.
+ *   - Workspace: a device buffer of moe_workspace_size() bytes, 256-byte aligned, owned by
+ *     the caller. Its first 256 bytes hold the device error word: zero them once with
+ *     moe_workspace_init() before the first use. Calls that share a workspace must be
+ *     ordered on one stream (they reuse its scratch regions).
+ *   - Determinism: identical inputs give bitwise identical outputs; no floating-point
+ *     atomics are used anywhere.
+ *   - Kernels that wait on an on-chip barrier give up after a bounded time and record a
+ *     code in the workspace's device error word (see moe_get_device_error).
+ *   - Requires an sm_100a GPU (B200).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_CUDA = 3,
+  MOE_ERR_DEVICE = 4 /* a kernel recorded a device-side error (see moe_get_device_error) */
+} moe_status;
+
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_ERF = 1, MOE_ACT_GELU_TANH = 2 };
+
+/* Device error codes written to the workspace error word. */
+enum {
+  MOE_DEVERR_NONE = 0,
+  MOE_DEVERR_WAIT_TIMEOUT = 1, /* a pipeline barrier wait exceeded its time bound */
+  MOE_DEVERR_BAD_INDEX = 2     /* an expert index outside [0,E) reached a kernel */
+};
+
+/* The problem statement (LLMs-from-scratch 12.1; walkthrough 3.1; Grok-1 book 5.2.3).
+ *   N               tokens (B*T flattened), >= 0
+ *   D, F            model width and expert FFN width, >= 1
+ *   E               experts, 1..64
+ *   k               experts per token, 1..min(E, 8)
+ *   capacity_factor CF; <= 0 means no capacity (every record is kept)
+ *   renormalize     0: gate = softmax over all E (Grok-1); 1: gate renormalised over the
+ *                   selected k (Mixtral / walkthrough 1.2)
+ *   activation      MOE_ACT_* applied to x W1 (SiLU, exact-erf GELU, tanh GELU)
+ *   dtype           MOE_DTYPE_* of X, W1..W3 and every activation buffer
+ * bf16 problems need D and F to be multiples of 8 (16-byte rows for the tensor-memory
+ * copies); fp32 problems need D and F to be multiples of 4. */
+typedef struct {
+  int64_t N;
+  int64_t D;
+  int64_t F;
+  int32_t E;
+  int32_t k;
+  double capacity_factor;
+  int32_t renormalize;
+  int32_t activation;
+  int32_t dtype;
+  int32_t reserved; /* must be 0 */
+} moe_problem;
+
+/* Host only. C = ceil(CF * N * k / E) evaluated in double left to right (walkthrough 3.1);
+ * C = N*k when CF <= 0. */
+moe_status moe_capacity(const moe_problem* p, int64_t* C);
+
+/* Host only. Bytes of workspace every entry point below accepts for problem p (one size for
+ * all of them). The workspace holds the device error word, scratch counters and, for
+ * moe_forward, the intermediate buffers (routing results, X_perm, H, Y). */
+moe_status moe_workspace_size(const moe_problem* p, size_t* bytes);
+
+/* Router + softmax + top-k + gates (Grok-1 book 5.2, 5.2.3; walkthrough 1.1, 1.2;
+ * LLMs-from-scratch 12.1).
+ *   X != NULL : logits = fp32(X) . W_r (+ bias), fp32 accumulation; written to `logits`
+ *               when `logits` != NULL.
+ *   X == NULL : `logits` is read as an INPUT [N,E] (routing from given fp32 logits).
+ *   topk_idx  : the k experts with the largest fp32 logits, in descending order; equal
+ *               logits are ordered by lower expert index.
+ *   topk_gate : renormalize=0: softmax(logits)[idx]; renormalize=1: softmax of the selected
+ *               logits (= probs[idx] / sum of the selected probs).
+ *   prob_colsum (optional, [E]): sum over tokens of the full softmax, for the balance loss
+ *               (walkthrough 2.1); summed in a fixed order.
+ *   W_r may be NULL only when X is NULL. bias (optional, [E] fp32) is added to the logits.
+ * Workspace: moe_workspace_size bytes. */
+moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, const float* bias,
+                     float* logits, int32_t* topk_idx, float* topk_gate, float* prob_colsum,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Load histogram, capacity, slot assignment and permutation (walkthrough 1.3, 3.1, 3.2;
+ * LLMs-from-scratch 12.2; MoE series 2.2).
+ *   load[e]      = number of records (t,j) with topk_idx[t,j] == e (before capacity).
+ *   pos[t,j]     = rank of record (t,j) among expert e's records, records taken slot-major
+ *                  (all j=0 records in token order, then all j=1 records, ...).
+ *   dropped[t,j] = pos[t,j] >= C.
+ *   offsets      = exclusive prefix sum of min(load_e, C); offsets[E] = kept records.
+ *   row_token[offsets[e] + pos[t,j]] = t for every kept record; entries past offsets[E]
+ *                  are not written.
+ *   X_perm[row]  = X[row_token[row]] for row < offsets[E] (skipped when X or X_perm is NULL);
+ *                  rows past offsets[E] are not written.
+ * topk_idx values must lie in [0,E); a value outside is recorded as MOE_DEVERR_BAD_INDEX
+ * and that record is treated as dropped. Bit-exact and deterministic. */
+moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk_idx,
+                        int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                        int32_t* row_token, void* X_perm, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* Grouped gated expert FFN on the expert-contiguous rows (LLMs-from-scratch 12.1; Grok-1
+ * book 5.3.5): for each expert e and each row r in [offsets[e], offsets[e+1]):
+ *   H[r] = act(X_perm[r] W1_e) (.) (X_perm[r] W2_e),   Y[r] = H[r] W3_e.
+ * bf16: tcgen05 tensor-core GEMMs with fp32 accumulation, act and product in fp32, H and Y
+ * rounded to bf16. fp32: CUDA-core fp32 FMA throughout. offsets stay on the device (the
+ * host never learns the per-expert counts). Rows past offsets[E] are not written. */
+moe_status moe_expert_ffn(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                          const void* W1, const void* W2, const void* W3, void* H, void* Y,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* First half of moe_expert_ffn (GEMM1 with the gating fused into its epilogue):
+ *   H[r] = act(X_perm[r] W1_e) (.) (X_perm[r] W2_e)   for r in [offsets[e], offsets[e+1]).
+ * Same precision, layout and row rules as moe_expert_ffn. */
+moe_status moe_expert_up(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                         const void* W1, const void* W2, void* H, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Second half of moe_expert_ffn (GEMM2): Y[r] = H[r] W3_e for r in [offsets[e], offsets[e+1]). */
+moe_status moe_expert_down(const moe_problem* p, const void* H, const int32_t* offsets,
+                           const void* W3, void* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* Gate-weighted combine (Grok-1 book 5.3.5; LLMs-from-scratch 12.2; MoE series 2.2):
+ *   out[t] = sum_{j=0..k-1} [!dropped[t,j]] * topk_gate[t,j] * Y[offsets[topk_idx[t,j]] + pos[t,j]]
+ * accumulated in fp32 in ascending j, rounded once to the output dtype; a token whose
+ * slots are all dropped gets 0. `dropped` may be NULL (nothing dropped). No atomics. */
+moe_status moe_combine(const moe_problem* p, const void* Y, const int32_t* topk_idx,
+                       const float* topk_gate, const int32_t* offsets, const int32_t* pos,
+                       const uint8_t* dropped, void* out, void* stream);
+
+/* The whole layer: moe_route -> moe_dispatch -> moe_expert_ffn -> moe_combine, enqueued on
+ * one stream with no host synchronisation. Intermediates live in the workspace; each of
+ * the optional export pointers (logits .. prob_colsum) may be NULL, otherwise the
+ * corresponding intermediate is also written there. */
+moe_status moe_forward(const moe_problem* p, const void* X, const float* W_r, const float* bias,
+                       const void* W1, const void* W2, const void* W3, void* out, float* logits,
+                       int32_t* topk_idx, float* topk_gate, int32_t* load, int32_t* offsets,
+                       int32_t* pos, uint8_t* dropped, float* prob_colsum, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* moe_forward with HOST activations: X_host [N,D] and out_host [N,D] are host pointers
+ * (page-locked memory gives asynchronous copies), the weights and W_r/bias are device
+ * pointers. Enqueues the host->device copy of X, the forward, and the device->host copy
+ * of out on `stream`, then waits for the stream, so out_host is valid on return. Uses
+ * the workspace (moe_workspace_size + N*D*2*sizeof(element) bytes, see
+ * moe_workspace_size_host). */
+moe_status moe_forward_host(const moe_problem* p, const void* X_host, const float* W_r,
+                            const float* bias, const void* W1, const void* W2, const void* W3,
+                            void* out_host, void* ws, size_t ws_bytes, void* stream);
+
+/* Host only. Workspace bytes for moe_forward_host. */
+moe_status moe_workspace_size_host(const moe_problem* p, size_t* bytes);
+
+/* Zero the device error word of a new workspace (asynchronous, on `stream`). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the device error word of workspace `ws` into *code
+ * (MOE_DEVERR_*) and clears it. Returns MOE_ERR_DEVICE when the word was non-zero. */
+moe_status moe_get_device_error(void* ws, void* stream, int32_t* code);
+
+/* Static strings. */
+const char* moe_status_string(moe_status s);
+const char* moe_last_error(void);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,128 @@
+"""CPU tests of the C ABI: the library builds and loads without a GPU, exports every symbol
+include/moe.h declares, and its host-side logic (capacity, workspace sizing, argument checks)
+behaves as documented. No compute call is made here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from top_routing_expert_fp32_b200 import build
+    build.build()
+    from top_routing_expert_fp32_b200 import abi as a
+    return a
+
+
+def _header_functions():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(abi):
+    declared = _header_functions()
+    assert set(declared) == set(abi.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s(moe_[a-z_]+)$", out, flags=re.M))
+    missing = set(declared) - exported
+    assert not missing, f"declared but not exported: {missing}"
+    for name in declared:
+        assert hasattr(abi.lib, name)
+
+
+def test_library_built_for_sm100a(abi):
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", abi.LIB_PATH],
+                         capture_output=True, text=True)
+    assert out.returncode == 0 and "sm_100a" in out.stdout
+
+
+def test_version_and_status_strings(abi):
+    assert abi.lib.moe_version() >= 100
+    assert abi.lib.moe_status_string(0) == b"ok"
+    assert abi.lib.moe_status_string(3) == b"CUDA error"
+
+
+@pytest.mark.parametrize("N,k,E,cf", [(16384, 2, 64, 1.25), (16384, 1, 64, 1.25), (8, 2, 4, 1.0),
+                                      (10, 2, 3, 1.0), (100, 2, 8, 0.0), (0, 2, 8, 1.25),
+                                      (7, 3, 5, 0.3), (4096, 2, 8, -1.0)])
+def test_capacity_matches_oracle(abi, oracle_lib, N, k, E, cf):
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("c", N=N, D=64, F=64, E=E, k=k, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1, capacity_factor=cf)
+    assert abi.capacity(abi.problem(cfg)) == oracle_lib.capacity(N, k, E, cf)
+
+
+def test_workspace_size_covers_intermediates(abi):
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.CONFIGS["mixtral"]
+    p = abi.problem(cfg)
+    n = abi.workspace_size(p)
+    R = cfg.N * cfg.k
+    assert n >= 2 * R * (2 * cfg.D + cfg.F)  # X_perm, H, Y in bf16
+    assert abi.workspace_size(p, host=True) >= n + 2 * 2 * cfg.N * cfg.D
+    p0 = abi.problem(cfg, N=0)
+    assert abi.workspace_size(p0) >= 256
+
+
+def _call_route(abi, p, ws=None, ws_bytes=0, X=None, W_r=None, logits=None, idx=8, gate=8):
+    return abi.lib.moe_route(ctypes.byref(p), X, W_r, None, logits, idx, gate, None, ws,
+                             ws_bytes, None)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("k", 0, 1), ("k", 9, 1), ("E", 65, 2), ("N", -1, 1), ("D", 0, 1), ("dtype", 7, 1),
+    ("activation", 3, 1), ("renormalize", 2, 1), ("reserved", 1, 1), ("D", 12, 2),
+    ("capacity_factor", float("nan"), 1)])
+def test_invalid_problems_rejected_on_host(abi, field, value, status):
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("c", N=64, D=64, F=64, E=8, k=2, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1)
+    p = abi.problem(cfg)
+    setattr(p, field, value)
+    b = ctypes.c_size_t()
+    assert abi.lib.moe_workspace_size(ctypes.byref(p), ctypes.byref(b)) == status
+    assert len(abi.lib.moe_last_error()) > 0
+
+
+def test_k9_with_large_E_is_unsupported(abi):
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("c", N=64, D=64, F=64, E=16, k=9, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1)
+    b = ctypes.c_size_t()
+    assert abi.lib.moe_workspace_size(ctypes.byref(abi.problem(cfg)), ctypes.byref(b)) == 2
+
+
+def test_null_and_misaligned_pointers_rejected(abi):
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("c", N=64, D=64, F=64, E=8, k=2, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1)
+    p = abi.problem(cfg)
+    need = abi.workspace_size(p)
+    # No workspace.
+    assert _call_route(abi, p, X=4096, W_r=4096) == abi.MOE_ERR_INVALID_ARG
+    # Workspace too small.
+    assert _call_route(abi, p, ws=4096, ws_bytes=need - 1, X=4096, W_r=4096) == \
+        abi.MOE_ERR_INVALID_ARG
+    assert b"too small" in abi.lib.moe_last_error()
+    # Misaligned X.
+    assert _call_route(abi, p, ws=4096, ws_bytes=need, X=4100, W_r=4096) == \
+        abi.MOE_ERR_INVALID_ARG
+    assert b"aligned" in abi.lib.moe_last_error()
+    # Routing from logits needs the logits pointer.
+    assert _call_route(abi, p, ws=4096, ws_bytes=need) == abi.MOE_ERR_INVALID_ARG
+    # Dispatch: X without X_perm.
+    st = abi.lib.moe_dispatch(ctypes.byref(p), 4096, 4096, 4096, 4096, 4096, 4096, None, None,
+                              4096, need, None)
+    assert st == abi.MOE_ERR_INVALID_ARG
+    # Forward: missing weights.
+    st = abi.lib.moe_forward(ctypes.byref(p), 4096, 4096, None, None, 4096, 4096, 4096,
+                             *([None] * 8), 4096, need, None)
+    assert st == abi.MOE_ERR_INVALID_ARG and b"W1" in abi.lib.moe_last_error()

@@ -1,0 +1,154 @@
+"""End-to-end GPU parity of moe_forward (the path the benchmark times) against the oracle.
+
+Small layers are compared on every token. The five named workloads run at their full sizes,
+in the same launch configuration the benchmark uses; the oracle then checks routing for every
+token (bit-exact integers, near-tie flips counted and excluded), dispatch bit-exact, and the
+layer output on a deterministic sample of tokens it computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from top_routing_expert_fp32_b200 import configs, inputs
+from gpu_helpers import (NEAR_TIE, alloc_dispatch_out, alloc_route_out, np_host,
+                         normwise_rel_err, oracle_dtype, to_f64, tol)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from top_routing_expert_fp32_b200 import abi as a
+    return a
+
+
+def run_forward(abi, cfg, inp):
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    r = alloc_route_out(cfg.N, cfg.E, cfg.k)
+    d = alloc_dispatch_out(cfg.N, cfg.E, cfg.k)
+    out = torch.empty((cfg.N, cfg.D), dtype=inp.X.dtype, device="cuda")
+    abi.forward(p, inp.X, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, out, ws,
+                logits=r["logits"], topk_idx=r["idx"], topk_gate=r["gate"], load=d["load"],
+                offsets=d["offsets"], pos=d["pos"], dropped=d["dropped"],
+                prob_colsum=r["colsum"])
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    ex = {k: v.cpu().numpy() for k, v in {**r, **d}.items()}
+    return out, ex
+
+
+def check_layer(cfg, inp, out, ex, sample=None):
+    """Oracle checks; returns a summary dict."""
+    od = oracle_dtype(cfg)
+    Xn = np_host(inp.X)
+    Wr = inp.W_r.cpu().numpy()
+    bias = None if inp.bias is None else inp.bias.cpu().numpy()
+    l64, l32 = oracle.router_logits(Xn, od, Wr, bias)
+    ro = oracle.route(l32, k=cfg.k, renorm=cfg.renormalize)
+    margin = oracle.topk_margin(l64, cfg.k)
+    flips = (ex["idx"] != ro["idx"]).any(1)
+    assert (margin[flips] < NEAR_TIE).all(), "routing differs on a token that is not near-tied"
+    C = oracle.capacity(cfg.N, cfg.k, cfg.E, cfg.capacity_factor)
+    do = oracle.dispatch(ro["idx"], cfg.E, C)
+    if not flips.any():
+        for key in ("load", "offsets", "pos", "dropped"):
+            assert np.array_equal(ex[key], do[key]), key
+    else:  # a flip shifts later positions of the experts involved; compare the rest
+        assert (ex["load"].sum() == cfg.N * cfg.k)
+    same = ~flips & (ex["dropped"] == do["dropped"]).all(1)
+    np.testing.assert_allclose(ex["colsum"], ro["colsum"], rtol=1e-4, atol=1e-3)
+    # layer output on the sampled tokens
+    toks = np.arange(cfg.N) if sample is None else np.asarray(sample)
+    toks = toks[same[toks]]
+    rec_t, rec_e, slot = [], [], []
+    for t in toks:
+        for j in range(cfg.k):
+            if not do["dropped"][t, j]:
+                rec_t.append(t)
+                rec_e.append(ro["idx"][t, j])
+                slot.append((t, j))
+    Y = oracle.expert_ffn(np.array(rec_t, np.int32), np.array(rec_e, np.int32), Xn,
+                          np_host(inp.W1), np_host(inp.W2), np_host(inp.W3), od, cfg.activation)
+    ref = np.zeros((len(toks), cfg.D))
+    row_of = {t: i for i, t in enumerate(toks)}
+    for (t, j), y in zip(slot, Y):
+        ref[row_of[t]] += ro["gate"][t, j] * y
+    got = to_f64(out)[toks]
+    err = normwise_rel_err(got, ref)
+    assert err.max() <= tol(cfg), f"max normwise rel err {err.max():.3g} > {tol(cfg)}"
+    all_dropped = do["dropped"][toks].all(1)
+    assert (got[all_dropped] == 0).all()
+    return dict(flips=int(flips.sum()), max_err=float(err.max()), tokens=len(toks),
+                drop_rate=oracle.drop_rate(do["dropped"]))
+
+
+SMALL = [
+    configs.CONFIGS["tiny_f32"],
+    configs.MoEConfig("small_silu", N=300, D=256, F=512, E=8, k=2, dtype=configs.DTYPE_BF16,
+                      activation=configs.ACT_SILU, renormalize=1),
+    configs.MoEConfig("small_gelu_norenorm", N=257, D=384, F=640, E=8, k=2,
+                      dtype=configs.DTYPE_BF16, activation=configs.ACT_GELU_ERF, renormalize=0),
+    configs.MoEConfig("small_capacity", N=500, D=128, F=256, E=16, k=2, dtype=configs.DTYPE_BF16,
+                      activation=configs.ACT_SILU, renormalize=1, capacity_factor=1.0,
+                      router_bias_var=2.0),
+    configs.MoEConfig("small_capacity_k1", N=500, D=128, F=256, E=16, k=1,
+                      dtype=configs.DTYPE_BF16, activation=configs.ACT_SILU, renormalize=1,
+                      capacity_factor=0.8, router_bias_var=2.0),
+    configs.MoEConfig("small_f32_gelu_tanh", N=96, D=64, F=96, E=5, k=3, dtype=configs.DTYPE_F32,
+                      activation=configs.ACT_GELU_TANH, renormalize=0, capacity_factor=0.9),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=[c.name for c in SMALL])
+def test_forward_small_all_tokens(abi, cfg):
+    inp = inputs.make_inputs(cfg, "cuda")
+    out, ex = run_forward(abi, cfg, inp)
+    s = check_layer(cfg, inp, out, ex)
+    assert s["tokens"] >= cfg.N - 2 * s["flips"] - 8
+
+
+def test_forward_deterministic_and_host_entry(abi):
+    cfg = SMALL[3]
+    inp = inputs.make_inputs(cfg, "cuda")
+    out1, _ = run_forward(abi, cfg, inp)
+    out2, _ = run_forward(abi, cfg, inp)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    p = abi.problem(cfg)
+    ws = abi.workspace(p, host=True)
+    xh = inp.X.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws)
+    assert torch.equal(oh.view(torch.int16), out1.cpu().view(torch.int16))
+
+
+def test_forward_zero_tokens(abi):
+    cfg = SMALL[1].with_(N=0)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    inp = inputs.make_inputs(SMALL[1].with_(N=1), "cuda")
+    out = torch.empty((1, cfg.D), dtype=torch.bfloat16, device="cuda")
+    abi.forward(p, inp.X, inp.W_r, None, inp.W1, inp.W2, inp.W3, out, ws)
+    torch.cuda.synchronize()
+
+
+def _sample(cfg, n=12):
+    s = set(np.linspace(0, cfg.N - 1, n).astype(int).tolist())
+    return sorted(s)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "decode", "mixtral", "capacity", "capacity_k1",
+                                  "grok1"])
+def test_forward_named_workload_full_size(abi, name):
+    cfg = configs.CONFIGS[name]
+    inp = inputs.make_inputs(cfg, "cuda")
+    out, ex = run_forward(abi, cfg, inp)
+    sample = None if cfg.N <= 64 else _sample(cfg)
+    if cfg.capacity_factor > 0:   # include tokens that lost one or both slots
+        d = ex["dropped"]
+        extra = list(np.where(d.all(1))[0][:2]) + list(np.where(d.any(1) & ~d.all(1))[0][:2])
+        sample = sorted(set(sample) | set(int(t) for t in extra))
+    s = check_layer(cfg, inp, out, ex, sample)
+    print(f"\n{name}: {s}")
+    del inp
+    torch.cuda.empty_cache()

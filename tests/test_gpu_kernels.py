@@ -1,0 +1,260 @@
+"""GPU parity of each kernel behind the C ABI against the CPU oracle, at sizes the oracle
+finishes in seconds that span several tiles and ragged tails, plus edge cases.
+Integer outputs bit-exact; floating point within the stated tolerances."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from top_routing_expert_fp32_b200 import configs, inputs
+from gpu_helpers import (NEAR_TIE, TOL_BF16, alloc_dispatch_out, alloc_route_out, np_host,
+                         normwise_rel_err, oracle_dtype, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from top_routing_expert_fp32_b200 import abi as a
+    return a
+
+
+def _cfg(N, D, F, E, k, dtype=configs.DTYPE_BF16, act=0, renorm=1, cf=0.0, bias_var=0.0):
+    return configs.MoEConfig("t", N=N, D=D, F=F, E=E, k=k, dtype=dtype, activation=act,
+                             renormalize=renorm, capacity_factor=cf, router_bias_var=bias_var)
+
+
+# ------------------------------------------------------------------ routing from given logits
+
+@pytest.mark.parametrize("N,E,k,renorm,ties", [
+    (1, 1, 1, 1, False), (7, 3, 2, 0, False), (64, 4, 2, 1, True), (1000, 8, 2, 1, False),
+    (1000, 8, 2, 0, True), (4097, 8, 1, 1, False), (333, 13, 5, 0, True), (2048, 64, 2, 1, False),
+    (2050, 64, 8, 0, True), (100, 64, 1, 1, True), (65, 16, 8, 0, False)])
+def test_route_from_logits_bitexact(abi, oracle_lib, N, E, k, renorm, ties):
+    if ties:
+        rng = np.random.default_rng(N + E)
+        l32 = rng.integers(-2, 3, size=(N, E)).astype(np.float32)
+    else:
+        l32 = inputs.make_logits(N, E, seed=N * 7 + E).numpy()
+    cfg = _cfg(N, 64, 64, E, k, renorm=renorm)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    o = alloc_route_out(N, E, k)
+    o["logits"].copy_(torch.from_numpy(l32))
+    abi.route(p, None, None, None, o["logits"], o["idx"], o["gate"], o["colsum"], ws)
+    torch.cuda.synchronize()
+    ref = oracle_lib.route(l32, k=k, renorm=renorm)
+    assert np.array_equal(o["idx"].cpu().numpy(), ref["idx"])
+    np.testing.assert_allclose(o["gate"].cpu().numpy(), ref["gate"], rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(o["colsum"].cpu().numpy(), ref["colsum"], rtol=1e-5, atol=1e-5)
+    assert abi.device_error(ws) == 0
+
+
+@pytest.mark.parametrize("dtype,N,D,E,k,renorm,bias_var", [
+    (configs.DTYPE_BF16, 515, 256, 8, 2, 1, 0.0), (configs.DTYPE_BF16, 1000, 2048, 64, 2, 1, 2.0),
+    (configs.DTYPE_F32, 64, 64, 4, 2, 1, 0.0), (configs.DTYPE_BF16, 77, 72, 6, 3, 0, 0.0),
+    (configs.DTYPE_F32, 130, 100, 13, 1, 1, 1.0), (configs.DTYPE_BF16, 257, 6144, 8, 2, 0, 0.0)])
+def test_route_from_x(abi, oracle_lib, dtype, N, D, E, k, renorm, bias_var):
+    cfg = _cfg(N, D, 64, E, k, dtype=dtype, renorm=renorm, bias_var=bias_var)
+    inp = inputs.make_inputs(cfg, "cuda", seed=3, weights=False)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    o = alloc_route_out(N, E, k)
+    abi.route(p, inp.X, inp.W_r, inp.bias, o["logits"], o["idx"], o["gate"], o["colsum"], ws)
+    torch.cuda.synchronize()
+    Xn = np_host(inp.X)
+    l64, l32 = oracle_lib.router_logits(Xn, oracle_dtype(cfg), inp.W_r.cpu().numpy(),
+                                        None if inp.bias is None else inp.bias.cpu().numpy())
+    # fp32 accumulation error bound: relative to sum_d |x_d w_de|.
+    scale = np.abs(to_f64(inp.X)) @ np.abs(inp.W_r.cpu().double().numpy())
+    got_l = o["logits"].cpu().numpy().astype(np.float64)
+    assert (np.abs(got_l - l64) <= 1e-5 * scale + 1e-6).all()
+    ref = oracle_lib.route(l32, k=k, renorm=renorm)
+    margin = oracle_lib.topk_margin(l64, k)
+    got_idx = o["idx"].cpu().numpy()
+    diff = (got_idx != ref["idx"]).any(1)
+    assert (margin[diff] < NEAR_TIE).all(), "top-k mismatch on a token that is not near-tied"
+    same = ~diff
+    np.testing.assert_allclose(o["gate"].cpu().numpy()[same], ref["gate"][same], rtol=2e-5,
+                               atol=1e-6)
+    np.testing.assert_allclose(o["colsum"].cpu().numpy(), ref["colsum"], rtol=1e-4, atol=1e-4)
+
+
+# ------------------------------------------------------------------ dispatch (bit-exact)
+
+def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, X=None):
+    l32 = inputs.make_logits(N, E, seed=seed).numpy()
+    if skew:
+        l32 = l32 + (np.arange(E, dtype=np.float32)[::-1] * skew)
+    idx = oracle_lib.route(l32, k=k, renorm=1)["idx"]
+    if all_one:
+        idx = np.tile(np.arange(k, dtype=np.int32), (N, 1))
+    dtype = configs.DTYPE_F32 if (X is not None and X.dtype == torch.float32) else configs.DTYPE_BF16
+    cfg = _cfg(N, X.shape[1] if X is not None else 64, 64, E, k, dtype=dtype, cf=cf)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    d = alloc_dispatch_out(N, E, k)
+    idx_d = torch.from_numpy(idx).cuda()
+    X_perm = None
+    if X is not None:
+        X_perm = torch.full((N * k, X.shape[1]), float("nan"), dtype=X.dtype, device="cuda")
+    abi.dispatch(p, X, idx_d, d["load"], d["offsets"], d["pos"], d["dropped"], d["row_token"],
+                 X_perm, ws)
+    torch.cuda.synchronize()
+    C = abi.capacity(p)
+    assert C == oracle_lib.capacity(N, k, E, cf)
+    ref = oracle_lib.dispatch(idx, E, C)
+    assert np.array_equal(d["load"].cpu().numpy(), ref["load"])
+    assert np.array_equal(d["offsets"].cpu().numpy(), ref["offsets"])
+    assert np.array_equal(d["pos"].cpu().numpy(), ref["pos"])
+    assert np.array_equal(d["dropped"].cpu().numpy(), ref["dropped"])
+    nk = int(ref["offsets"][E])
+    assert np.array_equal(d["row_token"].cpu().numpy()[:nk], ref["row_token"])
+    assert abi.device_error(ws) == 0
+    return d, ref, X_perm
+
+
+@pytest.mark.parametrize("N,E,k,cf,skew", [
+    (1, 1, 1, 0.0, 0), (5, 3, 2, 0.3, 0), (64, 4, 2, 0.0, 0), (1000, 8, 2, 0.0, 0),
+    (1000, 8, 2, 1.0, 0.5), (5000, 8, 2, 1.25, 0.3), (16384, 64, 2, 1.25, 0.05),
+    (16384, 64, 1, 1.25, 0.05), (3001, 13, 3, 0.7, 0.2), (2049, 64, 8, 1.0, 0.0),
+    (1025, 2, 1, 0.5, 0)])
+def test_dispatch_bitexact(abi, oracle_lib, N, E, k, cf, skew):
+    _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=N + E + k, skew=skew)
+
+
+def test_dispatch_all_records_to_one_expert_set(abi, oracle_lib):
+    d, ref, _ = _dispatch_case(abi, oracle_lib, 3000, 8, 2, 1.25, seed=1, all_one=True)
+    assert ref["dropped"].any()
+
+
+def test_dispatch_zero_tokens(abi):
+    cfg = _cfg(0, 64, 64, 8, 2)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    d = alloc_dispatch_out(1, 8, 2)
+    d["load"].fill_(5)
+    d["offsets"].fill_(5)
+    idx = torch.zeros((1, 2), dtype=torch.int32, device="cuda")
+    abi.dispatch(p, None, idx, d["load"], d["offsets"], d["pos"], d["dropped"], d["row_token"],
+                 None, ws)
+    torch.cuda.synchronize()
+    assert (d["load"] == 0).all() and (d["offsets"] == 0).all()
+
+
+def test_dispatch_bad_index_reported(abi, oracle_lib):
+    N, E, k = 300, 8, 2
+    idx = oracle_lib.route(inputs.make_logits(N, E, seed=4).numpy(), k=k, renorm=1)["idx"].copy()
+    idx[17, 1] = E          # out of range
+    idx[200, 0] = -3        # out of range
+    cfg = _cfg(N, 64, 64, E, k)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    d = alloc_dispatch_out(N, E, k)
+    abi.dispatch(p, None, torch.from_numpy(idx).cuda(), d["load"], d["offsets"], d["pos"],
+                 d["dropped"], d["row_token"], None, ws)
+    assert abi.device_error(ws) == abi.DEVERR_BAD_INDEX
+    dr = d["dropped"].cpu().numpy()
+    assert dr[17, 1] == 1 and dr[200, 0] == 1
+    assert d["load"].cpu().numpy().sum() == N * k - 2
+    assert abi.device_error(ws) == 0  # cleared
+
+
+@pytest.mark.parametrize("N,D,E,k,cf,dtype", [
+    (1000, 4096, 8, 2, 0.0, configs.DTYPE_BF16), (777, 8, 4, 2, 0.5, configs.DTYPE_BF16),
+    (300, 16384, 8, 2, 1.0, configs.DTYPE_BF16), (64, 64, 4, 2, 0.0, configs.DTYPE_F32),
+    (2500, 2048, 64, 2, 1.25, configs.DTYPE_BF16), (129, 6144, 8, 1, 0.0, configs.DTYPE_BF16)])
+def test_gather_exact(abi, oracle_lib, N, D, E, k, cf, dtype):
+    X = inputs.randn((N, D), 1.0, inputs.torch_dtype(dtype), "cuda", seed=5, tid=1)
+    d, ref, X_perm = _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=9, X=X)
+    nk = int(ref["offsets"][E])
+    rt = torch.from_numpy(ref["row_token"]).long().cuda()
+    assert torch.equal(X_perm[:nk].view(torch.int16 if X.dtype == torch.bfloat16 else torch.int32),
+                       X[rt].view(torch.int16 if X.dtype == torch.bfloat16 else torch.int32))
+    if nk < N * k:   # rows past the kept records are left untouched
+        assert torch.isnan(X_perm[nk:].float()).all()
+
+
+# ------------------------------------------------------------------ grouped expert FFN
+
+def _ffn_case(abi, oracle_lib, counts, D, F, act, dtype=configs.DTYPE_BF16, seed=0):
+    E = len(counts)
+    R = int(sum(counts))
+    cfg = _cfg(max(R, 1), D, F, E, 1, dtype=dtype, act=act)
+    tdt = inputs.torch_dtype(dtype)
+    Xp = inputs.randn((max(R, 1), D), 1.0, tdt, "cuda", seed, 1)
+    W1 = inputs.randn((E, D, F), 1 / math.sqrt(D), tdt, "cuda", seed, 3)
+    W2 = inputs.randn((E, D, F), 1 / math.sqrt(D), tdt, "cuda", seed, 4)
+    W3 = inputs.randn((E, F, D), 1 / math.sqrt(F), tdt, "cuda", seed, 5)
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32,
+                           device="cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    H = torch.full((max(R, 1), F), float("nan"), dtype=tdt, device="cuda")
+    Y = torch.full((max(R, 1), D), float("nan"), dtype=tdt, device="cuda")
+    abi.expert_ffn(p, Xp, offsets, W1, W2, W3, H, Y, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    if R == 0:
+        return
+    rec_e = np.repeat(np.arange(E, dtype=np.int32), counts)
+    ref = oracle_lib.expert_ffn(np.arange(R, dtype=np.int32), rec_e, np_host(Xp), np_host(W1),
+                                np_host(W2), np_host(W3), oracle_dtype(cfg), act)
+    err = normwise_rel_err(to_f64(Y[:R]), ref)
+    tol = TOL_BF16 if dtype == configs.DTYPE_BF16 else 1e-5
+    assert err.max() <= tol, f"max normwise rel err {err.max():.3g}"
+    return err
+
+
+@pytest.mark.parametrize("counts,D,F,act", [
+    ([128], 64, 256, configs.ACT_SILU),
+    ([128], 128, 128, configs.ACT_SILU),
+    ([0, 1, 300], 128, 256, configs.ACT_SILU),
+    ([129, 127, 128, 0, 5, 256, 1, 64], 256, 384, configs.ACT_GELU_ERF),
+    ([70, 0, 33], 72, 200, configs.ACT_GELU_TANH),
+    ([513, 400], 1024, 512, configs.ACT_SILU),
+    ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
+])
+def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, counts, D, F, act):
+    _ffn_case(abi, oracle_lib, counts, D, F, act)
+
+
+def test_expert_ffn_f32(abi, oracle_lib):
+    err = _ffn_case(abi, oracle_lib, [40, 0, 57, 31], 64, 128, configs.ACT_SILU,
+                    dtype=configs.DTYPE_F32)
+    assert err.max() <= 1e-5
+
+
+def test_expert_ffn_empty(abi, oracle_lib):
+    _ffn_case(abi, oracle_lib, [0, 0, 0], 64, 128, configs.ACT_SILU)
+
+
+# ------------------------------------------------------------------ combine
+
+@pytest.mark.parametrize("N,D,E,k,cf,dtype", [
+    (1000, 4096, 8, 2, 0.0, configs.DTYPE_BF16), (500, 2048, 64, 2, 1.0, configs.DTYPE_BF16),
+    (64, 64, 4, 2, 0.0, configs.DTYPE_F32), (300, 72, 5, 3, 0.4, configs.DTYPE_BF16),
+    (257, 1024, 8, 1, 0.5, configs.DTYPE_F32)])
+def test_combine(abi, oracle_lib, N, D, E, k, cf, dtype):
+    tdt = inputs.torch_dtype(dtype)
+    d, ref, _ = _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=11)
+    R = N * k
+    Y = inputs.randn((R, D), 1.0, tdt, "cuda", 12, 1)
+    rng = np.random.default_rng(3)
+    gate = torch.from_numpy(rng.random((N, k)).astype(np.float32)).cuda()
+    idx = oracle_lib.route(inputs.make_logits(N, E, seed=11).numpy(), k=k, renorm=1)["idx"]
+    cfg = _cfg(N, D, 64, E, k, dtype=dtype, cf=cf)
+    p = abi.problem(cfg)
+    out = torch.empty((N, D), dtype=tdt, device="cuda")
+    abi.combine(p, Y, torch.from_numpy(idx).cuda(), gate, d["offsets"], d["pos"], d["dropped"],
+                out)
+    torch.cuda.synchronize()
+    rows = ref["offsets"][idx] + ref["pos"]
+    Yrec = to_f64(Y)[np.where(ref["dropped"] == 1, 0, rows)]
+    oref = oracle_lib.combine(gate.cpu().double().numpy(), ref["dropped"], Yrec)
+    err = normwise_rel_err(to_f64(out), oref)
+    assert err.max() <= (8e-3 if dtype == configs.DTYPE_BF16 else 1e-6)
+    allgone = ref["dropped"].all(1)
+    assert (to_f64(out)[allgone] == 0).all()

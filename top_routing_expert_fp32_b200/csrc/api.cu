@@ -1,0 +1,491 @@
+// C ABI of the MoE FFN forward library (declared in include/moe.h): argument validation,
+// workspace layout, and the enqueueing of the kernels in the pages' order
+// (route -> dispatch -> expert FFN -> combine).
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace moe
+
+namespace {
+
+using namespace moe;
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t ns = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    uint64_t ms = 2000;
+    if (const char* s = std::getenv("MOE_WAIT_TIMEOUT_MS")) {
+      const long long v = std::atoll(s);
+      if (v > 0) ms = static_cast<uint64_t>(v);
+    }
+    ns = ms * 1000000ull;
+  });
+  return ns;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t elem_size(const moe_problem& p) { return p.dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+// Device workspace regions (byte offsets from the workspace base).
+struct Layout {
+  size_t err, colsum_part, counts, idx, gate, pos, dropped, load, offsets, row_token, xperm, h, y;
+  size_t total;       // moe_forward and every other entry point
+  size_t xin, xout;   // moe_forward_host only
+  size_t total_host;
+};
+
+Layout make_layout(const moe_problem& p) {
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  const size_t R = static_cast<size_t>(p.N) * static_cast<size_t>(p.k);
+  const size_t es = elem_size(p);
+  L.err = take(256);
+  L.colsum_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)) * p.E);
+  L.counts = take(sizeof(int32_t) * static_cast<size_t>(dispatch_num_chunks(R)) * p.E);
+  L.idx = take(sizeof(int32_t) * R);
+  L.gate = take(sizeof(float) * R);
+  L.pos = take(sizeof(int32_t) * R);
+  L.dropped = take(R);
+  L.load = take(sizeof(int32_t) * p.E);
+  L.offsets = take(sizeof(int32_t) * (p.E + 1));
+  L.row_token = take(sizeof(int32_t) * R);
+  L.xperm = take(es * R * static_cast<size_t>(p.D));
+  L.h = take(es * R * static_cast<size_t>(p.F));
+  L.y = take(es * R * static_cast<size_t>(p.D));
+  L.total = o;
+  L.xin = take(es * static_cast<size_t>(p.N) * static_cast<size_t>(p.D));
+  L.xout = take(es * static_cast<size_t>(p.N) * static_cast<size_t>(p.D));
+  L.total_host = o;
+  return L;
+}
+
+moe_status check_problem(const moe_problem* p) {
+  if (p == nullptr) return fail(MOE_ERR_INVALID_ARG, "problem is NULL");
+  if (p->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved field must be 0");
+  if (p->N < 0) return fail(MOE_ERR_INVALID_ARG, "N < 0");
+  if (p->D < 1 || p->F < 1) return fail(MOE_ERR_INVALID_ARG, "D and F must be >= 1");
+  if (p->E < 1) return fail(MOE_ERR_INVALID_ARG, "E < 1");
+  if (p->k < 1 || p->k > p->E) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, E]");
+  if (p->E > 64) return fail(MOE_ERR_UNSUPPORTED, "E > 64");
+  if (p->k > 8) return fail(MOE_ERR_UNSUPPORTED, "k > 8");
+  if (p->dtype != MOE_DTYPE_F32 && p->dtype != MOE_DTYPE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "unknown dtype");
+  if (p->activation < MOE_ACT_SILU || p->activation > MOE_ACT_GELU_TANH)
+    return fail(MOE_ERR_INVALID_ARG, "unknown activation");
+  if (p->renormalize != 0 && p->renormalize != 1)
+    return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (std::isnan(p->capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+  if (p->N * static_cast<int64_t>(p->k) > INT32_MAX)
+    return fail(MOE_ERR_UNSUPPORTED, "N*k exceeds 2^31-1 records");
+  if (p->D > (1 << 24) || p->F > (1 << 24)) return fail(MOE_ERR_UNSUPPORTED, "D or F > 2^24");
+  const int64_t vec = p->dtype == MOE_DTYPE_BF16 ? 8 : 4;
+  if (p->D % vec != 0 || p->F % vec != 0)
+    return fail(MOE_ERR_UNSUPPORTED,
+                p->dtype == MOE_DTYPE_BF16 ? "bf16 needs D and F multiples of 8"
+                                           : "fp32 needs D and F multiples of 4");
+  return MOE_OK;
+}
+
+bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+moe_status need(const void* ptr, const char* name, uintptr_t align = 16) {
+  if (ptr == nullptr) return fail(MOE_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  if (!aligned(ptr, align))
+    return fail(MOE_ERR_INVALID_ARG, std::string(name) + " is not " + std::to_string(align) +
+                                         "-byte aligned");
+  return MOE_OK;
+}
+
+moe_status opt(const void* ptr, const char* name, uintptr_t align = 16) {
+  return ptr == nullptr ? MOE_OK : need(ptr, name, align);
+}
+
+#define MOE_TRY(expr)              \
+  do {                             \
+    const moe_status _s = (expr);  \
+    if (_s != MOE_OK) return _s;   \
+  } while (0)
+
+#define MOE_CUDA(expr, where)                        \
+  do {                                               \
+    const cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+moe_status check_ws(const moe_problem& p, const void* ws, size_t ws_bytes, bool host) {
+  MOE_TRY(need(ws, "ws", 256));
+  const Layout L = make_layout(p);
+  const size_t want = host ? L.total_host : L.total;
+  if (ws_bytes < want)
+    return fail(MOE_ERR_INVALID_ARG,
+                "workspace too small: " + std::to_string(ws_bytes) + " < " + std::to_string(want));
+  return MOE_OK;
+}
+
+moe_status check_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  MOE_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "attr");
+  MOE_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "attr");
+  if (major != 10 || minor != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "requires an sm_100a (B200) GPU");
+  return MOE_OK;
+}
+
+int64_t capacity_of(const moe_problem& p) {
+  const int64_t R = p.N * static_cast<int64_t>(p.k);
+  if (p.capacity_factor <= 0.0) return R;
+  return static_cast<int64_t>(
+      std::ceil(p.capacity_factor * static_cast<double>(p.N) * static_cast<double>(p.k) /
+                static_cast<double>(p.E)));
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status run_up(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                  const void* W1, const void* W2, void* H, int* err, cudaStream_t stream) {
+  if (p.dtype == MOE_DTYPE_BF16) {
+    MOE_TRY(check_sm100());
+    MOE_CUDA(launch_ffn_up_sm100(p, X_perm, offsets, W1, W2, H, err, wait_timeout_ns(), stream),
+             "expert up-projection (tcgen05)");
+  } else {
+    MOE_CUDA(launch_ffn_up_f32(p, X_perm, offsets, W1, W2, H, stream), "expert up-projection");
+  }
+  return MOE_OK;
+}
+
+moe_status run_down(const moe_problem& p, const void* H, const int32_t* offsets, const void* W3,
+                    void* Y, int* err, cudaStream_t stream) {
+  if (p.dtype == MOE_DTYPE_BF16) {
+    MOE_TRY(check_sm100());
+    MOE_CUDA(launch_ffn_down_sm100(p, H, offsets, W3, Y, err, wait_timeout_ns(), stream),
+             "expert down-projection (tcgen05)");
+  } else {
+    MOE_CUDA(launch_ffn_down_f32(p, H, offsets, W3, Y, stream), "expert down-projection");
+  }
+  return MOE_OK;
+}
+
+moe_status run_ffn(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                   const void* W1, const void* W2, const void* W3, void* H, void* Y, int* err,
+                   cudaStream_t stream) {
+  MOE_TRY(run_up(p, X_perm, offsets, W1, W2, H, err, stream));
+  return run_down(p, H, offsets, W3, Y, err, stream);
+}
+
+moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, const float* bias,
+                        const void* W1, const void* W2, const void* W3, void* out, float* logits,
+                        int32_t* topk_idx, float* topk_gate, int32_t* load, int32_t* offsets,
+                        int32_t* pos, uint8_t* dropped, float* prob_colsum, void* ws,
+                        cudaStream_t stream) {
+  const Layout L = make_layout(p);
+  int* err = at<int>(ws, L.err);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* gate = topk_gate ? topk_gate : at<float>(ws, L.gate);
+  int32_t* ld = load ? load : at<int32_t>(ws, L.load);
+  int32_t* off = offsets ? offsets : at<int32_t>(ws, L.offsets);
+  int32_t* ps = pos ? pos : at<int32_t>(ws, L.pos);
+  uint8_t* dr = dropped ? dropped : at<uint8_t>(ws, L.dropped);
+  int32_t* row_token = at<int32_t>(ws, L.row_token);
+  void* xperm = at<void>(ws, L.xperm);
+  void* h = at<void>(ws, L.h);
+  void* y = at<void>(ws, L.y);
+  if (p.N == 0) {
+    MOE_CUDA(launch_slot_assign(p, 0, idx, at<int32_t>(ws, L.counts), ld, off, ps, dr, row_token,
+                                err, stream),
+             "dispatch");
+    if (prob_colsum) MOE_CUDA(cudaMemsetAsync(prob_colsum, 0, sizeof(float) * p.E, stream), "memset");
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_route(p, X, W_r, bias, logits, idx, gate, at<float>(ws, L.colsum_part),
+                        prob_colsum, err, stream),
+           "route");
+  MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps, dr,
+                              row_token, err, stream),
+           "slot assign");
+  MOE_CUDA(launch_gather(p, X, row_token, off, xperm, err, stream), "gather");
+  MOE_TRY(run_ffn(p, xperm, off, W1, W2, W3, h, y, err, stream));
+  MOE_CUDA(launch_combine(p, y, idx, gate, off, ps, dr, out, err, stream), "combine");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_capacity(const moe_problem* p, int64_t* C) {
+  MOE_TRY(check_problem(p));
+  if (C == nullptr) return fail(MOE_ERR_INVALID_ARG, "C is NULL");
+  *C = capacity_of(*p);
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_problem* p, size_t* bytes) {
+  MOE_TRY(check_problem(p));
+  if (bytes == nullptr) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = make_layout(*p).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size_host(const moe_problem* p, size_t* bytes) {
+  MOE_TRY(check_problem(p));
+  if (bytes == nullptr) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = make_layout(*p).total_host;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, const float* bias,
+                     float* logits, int32_t* topk_idx, float* topk_gate, float* prob_colsum,
+                     void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  if (X != nullptr) {
+    MOE_TRY(need(X, "X"));
+    MOE_TRY(need(W_r, "W_r"));
+    MOE_TRY(opt(logits, "logits", 4));
+  } else {
+    MOE_TRY(need(logits, "logits (input when X is NULL)", 4));
+  }
+  MOE_TRY(opt(bias, "bias", 4));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(topk_gate, "topk_gate", 4));
+  MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
+  const Layout L = make_layout(*p);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p->N == 0) {
+    if (prob_colsum) MOE_CUDA(cudaMemsetAsync(prob_colsum, 0, sizeof(float) * p->E, s), "memset");
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_route(*p, X, W_r, bias, logits, topk_idx, topk_gate, at<float>(ws, L.colsum_part),
+                        prob_colsum, at<int>(ws, L.err), s),
+           "route");
+  return MOE_OK;
+}
+
+moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk_idx,
+                        int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                        int32_t* row_token, void* X_perm, void* ws, size_t ws_bytes,
+                        void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(load, "load", 4));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(pos, "pos", 4));
+  MOE_TRY(need(dropped, "dropped", 1));
+  MOE_TRY(opt(row_token, "row_token", 4));
+  const bool gather = X != nullptr && X_perm != nullptr;
+  if ((X == nullptr) != (X_perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "X and X_perm must both be given or both be NULL");
+  if (gather) {
+    MOE_TRY(need(X, "X"));
+    MOE_TRY(need(X_perm, "X_perm"));
+  }
+  const Layout L = make_layout(*p);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = at<int>(ws, L.err);
+  int32_t* rt = row_token ? row_token : at<int32_t>(ws, L.row_token);
+  MOE_CUDA(launch_slot_assign(*p, capacity_of(*p), topk_idx, at<int32_t>(ws, L.counts), load,
+                              offsets, pos, dropped, rt, err, s),
+           "slot assign");
+  if (gather) MOE_CUDA(launch_gather(*p, X, rt, offsets, X_perm, err, s), "gather");
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                          const void* W1, const void* W2, const void* W3, void* H, void* Y,
+                          void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X_perm, "X_perm"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W1, "W1"));
+  MOE_TRY(need(W2, "W2"));
+  MOE_TRY(need(W3, "W3"));
+  MOE_TRY(need(H, "H"));
+  MOE_TRY(need(Y, "Y"));
+  if (p->N == 0) return MOE_OK;
+  const Layout L = make_layout(*p);
+  return run_ffn(*p, X_perm, offsets, W1, W2, W3, H, Y, at<int>(ws, L.err),
+                 static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_up(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                         const void* W1, const void* W2, void* H, void* ws, size_t ws_bytes,
+                         void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X_perm, "X_perm"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W1, "W1"));
+  MOE_TRY(need(W2, "W2"));
+  MOE_TRY(need(H, "H"));
+  if (p->N == 0) return MOE_OK;
+  const Layout L = make_layout(*p);
+  return run_up(*p, X_perm, offsets, W1, W2, H, at<int>(ws, L.err),
+                static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_down(const moe_problem* p, const void* H, const int32_t* offsets,
+                           const void* W3, void* Y, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(H, "H"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W3, "W3"));
+  MOE_TRY(need(Y, "Y"));
+  if (p->N == 0) return MOE_OK;
+  const Layout L = make_layout(*p);
+  return run_down(*p, H, offsets, W3, Y, at<int>(ws, L.err), static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_problem* p, const void* Y, const int32_t* topk_idx,
+                       const float* topk_gate, const int32_t* offsets, const int32_t* pos,
+                       const uint8_t* dropped, void* out, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(need(Y, "Y"));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(topk_gate, "topk_gate", 4));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(pos, "pos", 4));
+  MOE_TRY(opt(dropped, "dropped", 1));
+  MOE_TRY(need(out, "out"));
+  MOE_CUDA(launch_combine(*p, Y, topk_idx, topk_gate, offsets, pos, dropped, out, nullptr,
+                          static_cast<cudaStream_t>(stream)),
+           "combine");
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_problem* p, const void* X, const float* W_r, const float* bias,
+                       const void* W1, const void* W2, const void* W3, void* out, float* logits,
+                       int32_t* topk_idx, float* topk_gate, int32_t* load, int32_t* offsets,
+                       int32_t* pos, uint8_t* dropped, float* prob_colsum, void* ws,
+                       size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X, "X"));
+  MOE_TRY(need(W_r, "W_r"));
+  MOE_TRY(opt(bias, "bias", 4));
+  MOE_TRY(need(W1, "W1"));
+  MOE_TRY(need(W2, "W2"));
+  MOE_TRY(need(W3, "W3"));
+  MOE_TRY(need(out, "out"));
+  MOE_TRY(opt(logits, "logits", 4));
+  MOE_TRY(opt(topk_idx, "topk_idx", 4));
+  MOE_TRY(opt(topk_gate, "topk_gate", 4));
+  MOE_TRY(opt(load, "load", 4));
+  MOE_TRY(opt(offsets, "offsets", 4));
+  MOE_TRY(opt(pos, "pos", 4));
+  MOE_TRY(opt(dropped, "dropped", 1));
+  MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
+  return forward_impl(*p, X, W_r, bias, W1, W2, W3, out, logits, topk_idx, topk_gate, load,
+                      offsets, pos, dropped, prob_colsum, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_host(const moe_problem* p, const void* X_host, const float* W_r,
+                            const float* bias, const void* W1, const void* W2, const void* W3,
+                            void* out_host, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, true));
+  if (p->N > 0) {
+    MOE_TRY(need(X_host, "X_host", 1));
+    MOE_TRY(need(out_host, "out_host", 1));
+  }
+  MOE_TRY(need(W_r, "W_r"));
+  MOE_TRY(opt(bias, "bias", 4));
+  MOE_TRY(need(W1, "W1"));
+  MOE_TRY(need(W2, "W2"));
+  MOE_TRY(need(W3, "W3"));
+  const Layout L = make_layout(*p);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = elem_size(*p) * static_cast<size_t>(p->N) * static_cast<size_t>(p->D);
+  void* xin = at<void>(ws, L.xin);
+  void* xout = at<void>(ws, L.xout);
+  if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(xin, X_host, bytes, cudaMemcpyHostToDevice, s), "H2D");
+  MOE_TRY(forward_impl(*p, xin, W_r, bias, W1, W2, W3, xout, nullptr, nullptr, nullptr, nullptr,
+                       nullptr, nullptr, nullptr, nullptr, ws, s));
+  if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, s), "D2H");
+  MOE_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(need(ws, "ws", 256));
+  if (ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace smaller than 256 bytes");
+  MOE_CUDA(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)), "memset");
+  return MOE_OK;
+}
+
+moe_status moe_get_device_error(void* ws, void* stream, int32_t* code) {
+  if (ws == nullptr || code == nullptr) return fail(MOE_ERR_INVALID_ARG, "ws or code is NULL");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  int32_t v = 0;
+  MOE_CUDA(cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost), "read error word");
+  *code = v;
+  if (v != 0) {
+    MOE_CUDA(cudaMemset(ws, 0, sizeof(v)), "clear error word");
+    return fail(MOE_ERR_DEVICE, "device error code " + std::to_string(v));
+  }
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported problem";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+int32_t moe_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,286 @@
+// Dispatch: expert load histogram, capacity, slot-major position assignment, drop mask,
+// expert-contiguous row map, and the permutation of token rows into expert order.
+//   MoE formula-to-code walkthrough 1.3 (load = bincount of the routed experts), 3.1
+//   (capacity), 3.2 (dispatch with a dropped mask); LLMs-from-scratch ch.12, 12.2 (N*k
+//   dispatch records); MoE series (GShard/Mixtral/Switch) 2.2 (overflow).
+//
+// Record order is slot-major: r = j*N + t (all rank-0 records in token order, then rank 1 ...).
+// pos(t,j) = number of earlier records (in that order) routed to the same expert.
+//   pass 1 (count): records are split into chunks of kDispatchChunk; each block counts its
+//                   chunk per expert (integer shared-memory counters: order-free, exact).
+//   pass 2 (assign): each block sums the counts of the chunks before it (a few hundred ints),
+//                   then walks its chunk in tiles of 1024 records; inside a tile, warps rank
+//                   equal experts with __match_any_sync, and a per-expert scan over the 32
+//                   warps orders the warps. The result is the stable counting-sort rank --
+//                   bit-exact and independent of scheduling.
+// Gather: one warp per block; lane 0 streams 16-KB pieces of rows global -> shared -> global
+// with bulk copies (cp.async.bulk), keeping up to kGatherStages pieces in flight.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxE = 64;
+constexpr int kAssignThreads = 1024;  // 32 warps
+constexpr int kCountThreads = 256;
+
+__global__ void __launch_bounds__(kCountThreads)
+    count_kernel(const int32_t* __restrict__ idx, int64_t N, int k, int E, int64_t R,
+                 int32_t* __restrict__ counts, int* err) {
+  __shared__ int hist[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kDispatchChunk;
+  const int64_t r1 = std::min<int64_t>(r0 + kDispatchChunk, R);
+  for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+    const int64_t j = r / N, t = r - j * N;
+    const int e = idx[t * k + j];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else record_error(err, MOE_DEVERR_BAD_INDEX);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(kAssignThreads)
+    assign_kernel(const int32_t* __restrict__ idx, int64_t N, int k, int E, int64_t R,
+                  int64_t C, int nchunks, const int32_t* __restrict__ counts,
+                  int32_t* __restrict__ load, int32_t* __restrict__ offsets,
+                  int32_t* __restrict__ pos, uint8_t* __restrict__ dropped,
+                  int32_t* __restrict__ row_token) {
+  __shared__ int s_base[kMaxE];   // records of expert e in earlier chunks
+  __shared__ int s_off[kMaxE + 1];  // first row of expert e in the expert-contiguous order
+  __shared__ int s_wpre[32][kMaxE];  // per-warp running prefix of the current tile
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int base = 0, total = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = counts[static_cast<int64_t>(c) * E + e];
+      if (c < static_cast<int>(blockIdx.x)) base += v;
+      total += v;
+    }
+    s_base[e] = base;
+    s_wpre[0][e] = total;  // temporary: totals, consumed below
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = run;
+      const int64_t tot = s_wpre[0][e];
+      run += static_cast<int>(tot < C ? tot : C);
+    }
+    s_off[E] = run;
+    if (blockIdx.x == 0) {
+      for (int e = 0; e < E; ++e) {
+        load[e] = s_wpre[0][e];
+        offsets[e] = s_off[e];
+      }
+      offsets[E] = run;
+    }
+  }
+  __syncthreads();
+
+  int running = 0;  // thread e < E: records of expert e seen in earlier tiles of this chunk
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kDispatchChunk;
+  const int64_t r1 = std::min<int64_t>(r0 + kDispatchChunk, R);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int64_t tile = r0; tile < r1; tile += kAssignThreads) {
+    for (int i = threadIdx.x; i < 32 * kMaxE; i += kAssignThreads) (&s_wpre[0][0])[i] = 0;
+    __syncthreads();
+    const int64_t r = tile + threadIdx.x;
+    const bool valid = r < r1;
+    int64_t j = 0, t = 0;
+    int e = -1;
+    if (valid) {
+      j = r / N;
+      t = r - j * N;
+      e = idx[t * k + j];
+      if (e < 0 || e >= E) e = -1;  // recorded by the count pass
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -2);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && e >= 0 && rank == 0) s_wpre[warp][e] = __popc(peers);
+    __syncthreads();
+    if (threadIdx.x < E) {
+      const int ee = threadIdx.x;
+      int run = running;
+      for (int w = 0; w < 32; ++w) {
+        const int c = s_wpre[w][ee];
+        s_wpre[w][ee] = run;
+        run += c;
+      }
+      running = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int64_t rec = t * k + j;
+      if (e >= 0) {
+        const int p = s_base[e] + s_wpre[warp][e] + rank;
+        const bool drop = p >= C;
+        pos[rec] = p;
+        dropped[rec] = drop ? 1 : 0;
+        if (!drop && row_token != nullptr) row_token[s_off[e] + p] = static_cast<int32_t>(t);
+      } else {
+        pos[rec] = -1;
+        dropped[rec] = 1;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+constexpr int kGatherStages = 4;
+constexpr uint32_t kPieceBytes = 16384;
+constexpr uint64_t kGatherTimeoutNs = 2000000000ull;
+
+// One warp per block. Pieces q = blockIdx.x + i*gridDim.x, i = 0, 1, ...; piece q covers
+// bytes [ (q % P) * kPieceBytes, ... ) of row q / P.
+__global__ void __launch_bounds__(32)
+    gather_kernel(const uint8_t* __restrict__ X, const int32_t* __restrict__ row_token,
+                  const int32_t* __restrict__ offsets, int E, uint32_t row_bytes,
+                  uint8_t* __restrict__ X_perm, int* err) {
+  extern __shared__ __align__(128) uint8_t g_smem[];
+  __shared__ __align__(8) uint64_t bars[kGatherStages];
+  const int lane = threadIdx.x;
+  const int64_t rows = offsets[E];
+  const int64_t P = (row_bytes + kPieceBytes - 1) / kPieceBytes;
+  const int64_t total = rows * P;
+  if (static_cast<int64_t>(blockIdx.x) >= total) return;
+  const int64_t n = (total - blockIdx.x + gridDim.x - 1) / gridDim.x;  // pieces of this block
+
+  if (lane == 0) {
+    for (int s = 0; s < kGatherStages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  auto piece = [&](int64_t i, int64_t& row, uint32_t& off, uint32_t& bytes) {
+    const int64_t q = blockIdx.x + i * gridDim.x;
+    row = q / P;
+    off = static_cast<uint32_t>((q - row * P) * kPieceBytes);
+    const uint32_t rest = row_bytes - off;
+    bytes = rest < kPieceBytes ? rest : kPieceBytes;
+  };
+  // Token of the row of load index i, fetched 32 at a time by the whole warp.
+  int tok_batch = -1;
+  int64_t batch_base = -1;
+  auto token_of = [&](int64_t i) -> int {
+    const int64_t b = i & ~static_cast<int64_t>(31);
+    if (b != batch_base) {
+      batch_base = b;
+      const int64_t li = b + lane;
+      tok_batch = 0;
+      if (li < n) {
+        int64_t row;
+        uint32_t off, bytes;
+        piece(li, row, off, bytes);
+        tok_batch = row_token[row];
+      }
+    }
+    return __shfl_sync(0xffffffffu, tok_batch, static_cast<int>(i - b));
+  };
+  auto issue_load = [&](int64_t i) {
+    int64_t row;
+    uint32_t off, bytes;
+    piece(i, row, off, bytes);
+    const int tok = token_of(i);
+    if (lane == 0) {
+      const int s = static_cast<int>(i % kGatherStages);
+      mbar_arrive_expect_tx(&bars[s], bytes);
+      bulk_g2s(g_smem + s * kPieceBytes, X + static_cast<int64_t>(tok) * row_bytes + off, bytes,
+               &bars[s]);
+    }
+  };
+
+  const int64_t pro = std::min<int64_t>(n, kGatherStages);
+  for (int64_t i = 0; i < pro; ++i) issue_load(i);
+  int64_t issued = pro;  // loads [0, issued) have been issued
+  int64_t i = 0;
+  bool ok = true;
+  for (; i < n; ++i) {
+    const int s = static_cast<int>(i % kGatherStages);
+    const uint32_t parity = static_cast<uint32_t>((i / kGatherStages) & 1);
+    if (lane == 0) ok = mbar_wait(&bars[s], parity, kGatherTimeoutNs);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) {
+      if (lane == 0) record_error(err, MOE_DEVERR_WAIT_TIMEOUT);
+      break;
+    }
+    if (lane == 0) {
+      int64_t row;
+      uint32_t off, bytes;
+      piece(i, row, off, bytes);
+      bulk_s2g(X_perm + row * row_bytes + off, g_smem + s * kPieceBytes, bytes);
+      bulk_commit();
+    }
+    const int64_t nxt = i - 1 + kGatherStages;  // refill the stage read by store i-1
+    if (i >= 1 && nxt < n) {
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      issue_load(nxt);
+      issued = nxt + 1;
+    }
+  }
+  if (lane == 0) {
+    bulk_wait_all();
+    // After a timeout, loads [i, issued) may still be landing in shared memory: wait for
+    // each of them (bounded) before the block exits.
+    for (int64_t L = i; !ok && L < issued; ++L)
+      (void)mbar_wait(&bars[L % kGatherStages], static_cast<uint32_t>((L / kGatherStages) & 1),
+                      kGatherTimeoutNs / 16);
+  }
+}
+
+}  // namespace
+
+int dispatch_num_chunks(int64_t records) {
+  return static_cast<int>(std::max<int64_t>(1, (records + kDispatchChunk - 1) / kDispatchChunk));
+}
+
+cudaError_t launch_slot_assign(const moe_problem& p, int64_t capacity, const int32_t* idx,
+                               int32_t* chunk_counts, int32_t* load, int32_t* offsets,
+                               int32_t* pos, uint8_t* dropped, int32_t* row_token, int* err,
+                               cudaStream_t stream) {
+  const int64_t R = p.N * p.k;
+  if (R == 0) {
+    cudaError_t e = cudaMemsetAsync(load, 0, sizeof(int32_t) * p.E, stream);
+    if (e != cudaSuccess) return e;
+    return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.E + 1), stream);
+  }
+  const int nchunks = dispatch_num_chunks(R);
+  count_kernel<<<nchunks, kCountThreads, 0, stream>>>(idx, p.N, p.k, p.E, R, chunk_counts, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  assign_kernel<<<nchunks, kAssignThreads, 0, stream>>>(idx, p.N, p.k, p.E, R, capacity, nchunks,
+                                                       chunk_counts, load, offsets, pos, dropped,
+                                                       row_token);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const moe_problem& p, const void* X, const int32_t* row_token,
+                          const int32_t* offsets, void* X_perm, int* err, cudaStream_t stream) {
+  const int64_t R = p.N * p.k;
+  if (R == 0) return cudaSuccess;
+  const uint32_t elem = p.dtype == MOE_DTYPE_BF16 ? 2u : 4u;
+  const uint32_t row_bytes = static_cast<uint32_t>(p.D) * elem;
+  const int64_t P = (row_bytes + kPieceBytes - 1) / kPieceBytes;
+  const int64_t max_pieces = R * P;
+  const int grid = static_cast<int>(std::min<int64_t>(max_pieces, int64_t(num_sms()) * 3));
+  const size_t smem = kGatherStages * kPieceBytes;
+  cudaError_t e = cudaFuncSetAttribute(
+      gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  gather_kernel<<<grid, 32, smem, stream>>>(static_cast<const uint8_t*>(X), row_token, offsets,
+                                            p.E, row_bytes, static_cast<uint8_t*>(X_perm), err);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,60 @@
+// Host-side launchers of the kernels behind the C ABI. All pointers are device pointers;
+// every launcher enqueues on `stream` and returns the CUDA error of the launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Upper bound on router partial-sum blocks (the launcher never exceeds it).
+int route_num_blocks(int64_t N, int E);
+
+// Router GEMV + softmax + top-k + gates. X == nullptr: `logits` is an input.
+// colsum_partial: [route_num_blocks][E] floats (or nullptr when prob_colsum is nullptr).
+cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
+                         float* logits, int32_t* idx, float* gate, float* colsum_partial,
+                         float* prob_colsum, int* err, cudaStream_t stream);
+
+// Records are processed in chunks of this many for the slot assignment.
+constexpr int kDispatchChunk = 2048;
+
+int dispatch_num_chunks(int64_t records);
+
+// Histogram + prefix sums + slot-major capacity positions (+ row -> token map).
+cudaError_t launch_slot_assign(const moe_problem& p, int64_t capacity, const int32_t* idx,
+                               int32_t* chunk_counts, int32_t* load, int32_t* offsets,
+                               int32_t* pos, uint8_t* dropped, int32_t* row_token, int* err,
+                               cudaStream_t stream);
+
+// X_perm[row] = X[row_token[row]] for row < offsets[E] (bulk-copy staged through shared memory).
+cudaError_t launch_gather(const moe_problem& p, const void* X, const int32_t* row_token,
+                          const int32_t* offsets, void* X_perm, int* err, cudaStream_t stream);
+
+// Grouped expert GEMMs, bf16 operands, tcgen05 tensor cores.
+//   up:   H = act(X_perm W1_e) (.) (X_perm W2_e)      down: Y = H W3_e
+cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                                const void* W1, const void* W2, void* H, int* err,
+                                uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_ffn_down_sm100(const moe_problem& p, const void* H, const int32_t* offsets,
+                                  const void* W3, void* Y, int* err, uint64_t timeout_ns,
+                                  cudaStream_t stream);
+
+// The same two steps in fp32 on CUDA cores.
+cudaError_t launch_ffn_up_f32(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                              const void* W1, const void* W2, void* H, cudaStream_t stream);
+cudaError_t launch_ffn_down_f32(const moe_problem& p, const void* H, const int32_t* offsets,
+                                const void* W3, void* Y, cudaStream_t stream);
+
+// Gate-weighted combine of each token's k expert rows.
+cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* idx,
+                           const float* gate, const int32_t* offsets, const int32_t* pos,
+                           const uint8_t* dropped, void* out, int* err, cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace moe
