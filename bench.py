@@ -395,12 +395,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=None)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override N (smaller cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     from top_routing_expert_fp32_b200 import configs
     cfg = configs.CONFIGS[args.workload or configs.BENCH_WORKLOAD]
+    if args.tokens is not None:
+        cfg = cfg.with_(N=args.tokens, name=f"{cfg.name}_n{args.tokens}")
     world, rank, local = dist_env()
 
     if args.impl == "reference":
