@@ -145,6 +145,28 @@ moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk
                         int32_t* row_token, void* X_perm, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* moe_dispatch for callers that cannot give the library any device memory of their own:
+ * code that may no longer call cudaMalloc once it runs (an allocation synchronises the device
+ * and can stall every stream of a serving loop), or a host whose device memory is all owned by
+ * its own pool and lent out only as the tensors it computes on. Same arguments, results and
+ * guarantees as moe_dispatch, minus the workspace: the per-chunk expert counters live in a
+ * fixed 64 KiB array inside the library (held on every GPU that loads the library until the
+ * process exits). There is no counterpart on the pages; this is a deployment variant.
+ *   - row_token is required (it is an output here, not workspace).
+ *   - Limit: ceil(N*k / 2048) * E <= 16384 counters (e.g. N*k <= 524288 records at E = 64);
+ *     larger problems return MOE_ERR_UNSUPPORTED -- use moe_dispatch.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one array: calls that may overlap on the GPU (different streams,
+ *     or different host threads on one device) race and must be serialised by the caller.
+ *     Each call rewrites every counter it reads, so no clearing is needed between calls.
+ *   - Out-of-range expert indices are treated as dropped but not reported (there is no
+ *     workspace error word).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+moe_status moe_dispatch_noalloc(const moe_problem* p, const void* X, const int32_t* topk_idx,
+                                int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                                int32_t* row_token, void* X_perm, void* stream);
+
 /* Grouped gated expert FFN on the expert-contiguous rows (LLMs-from-scratch 12.1; Grok-1
  * book 5.3.5): for each expert e and each row r in [offsets[e], offsets[e+1]):
  *   H[r] = act(X_perm[r] W1_e) (.) (X_perm[r] W2_e),   Y[r] = H[r] W3_e.

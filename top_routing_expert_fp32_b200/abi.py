@@ -23,7 +23,7 @@ DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_INDEX = range(3)
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_workspace_size_host", "moe_route",
-           "moe_dispatch", "moe_expert_ffn", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_host",
+           "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_workspace_init", "moe_get_device_error", "moe_status_string", "moe_last_error",
            "moe_version")
 
@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_size_host": [PP, ctypes.POINTER(S)],
         "moe_route": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_dispatch": [PP, P, P, P, P, P, P, P, P, P, S, P],
+        "moe_dispatch_noalloc": [PP, P, P, P, P, P, P, P, P, P],
         "moe_expert_ffn": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_up": [PP, P, P, P, P, P, P, S, P],
         "moe_expert_down": [PP, P, P, P, P, P, S, P],
@@ -136,6 +137,14 @@ def dispatch(p, X, topk_idx, load, offsets, pos, dropped, row_token, X_perm, ws,
     _check(lib.moe_dispatch(ctypes.byref(p), _ptr(X), _ptr(topk_idx), _ptr(load), _ptr(offsets),
                             _ptr(pos), _ptr(dropped), _ptr(row_token), _ptr(X_perm), _ptr(ws),
                             ws.numel(), _stream(stream)))
+
+
+def dispatch_noalloc(p, X, topk_idx, load, offsets, pos, dropped, row_token, X_perm,
+                     stream=None):
+    """moe_dispatch without a workspace (counters in a fixed array inside the library)."""
+    _check(lib.moe_dispatch_noalloc(ctypes.byref(p), _ptr(X), _ptr(topk_idx), _ptr(load),
+                                    _ptr(offsets), _ptr(pos), _ptr(dropped), _ptr(row_token),
+                                    _ptr(X_perm), _stream(stream)))
 
 
 def expert_ffn(p, X_perm, offsets, W1, W2, W3, H, Y, ws, stream=None):

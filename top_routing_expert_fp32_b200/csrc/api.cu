@@ -489,3 +489,10 @@ const char* moe_last_error(void) { return g_last_error.c_str(); }
 int32_t moe_version(void) { return 100; }
 
 }  // extern "C"
+
+namespace moe {
+
+// Lets entry points defined in other files report through moe_last_error().
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
+}  // namespace moe

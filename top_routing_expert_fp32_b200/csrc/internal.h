@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <string>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -56,5 +58,8 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
                            const uint8_t* dropped, void* out, int* err, cudaStream_t stream);
 
 int num_sms();
+
+// Message returned by moe_last_error() on the calling thread.
+void set_last_error(const std::string& msg);
 
 }  // namespace moe
