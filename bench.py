@@ -397,6 +397,8 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="override N (smaller cases for profiling)")
+    ap.add_argument("--ffn", type=int, default=None,
+                    help="override F (smaller weight footprint for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -405,6 +407,8 @@ def main():
     cfg = configs.CONFIGS[args.workload or configs.BENCH_WORKLOAD]
     if args.tokens is not None:
         cfg = cfg.with_(N=args.tokens, name=f"{cfg.name}_n{args.tokens}")
+    if args.ffn is not None:
+        cfg = cfg.with_(F=args.ffn, name=f"{cfg.name}_f{args.ffn}")
     world, rank, local = dist_env()
 
     if args.impl == "reference":
