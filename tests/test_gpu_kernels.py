@@ -55,7 +55,9 @@ def test_route_from_logits_bitexact(abi, oracle_lib, N, E, k, renorm, ties):
 @pytest.mark.parametrize("dtype,N,D,E,k,renorm,bias_var", [
     (configs.DTYPE_BF16, 515, 256, 8, 2, 1, 0.0), (configs.DTYPE_BF16, 1000, 2048, 64, 2, 1, 2.0),
     (configs.DTYPE_F32, 64, 64, 4, 2, 1, 0.0), (configs.DTYPE_BF16, 77, 72, 6, 3, 0, 0.0),
-    (configs.DTYPE_F32, 130, 100, 13, 1, 1, 1.0), (configs.DTYPE_BF16, 257, 6144, 8, 2, 0, 0.0)])
+    (configs.DTYPE_F32, 130, 100, 13, 1, 1, 1.0), (configs.DTYPE_BF16, 257, 6144, 8, 2, 0, 0.0),
+    (configs.DTYPE_BF16, 600, 520, 33, 3, 1, 1.0), (configs.DTYPE_F32, 300, 200, 24, 2, 0, 0.0),
+    (configs.DTYPE_BF16, 64, 4096, 8, 2, 1, 0.0), (configs.DTYPE_BF16, 129, 1000, 64, 8, 0, 2.0)])
 def test_route_from_x(abi, oracle_lib, dtype, N, D, E, k, renorm, bias_var):
     cfg = _cfg(N, D, 64, E, k, dtype=dtype, renorm=renorm, bias_var=bias_var)
     inp = inputs.make_inputs(cfg, "cuda", seed=3, weights=False)
