@@ -218,8 +218,12 @@ def _ffn_case(abi, oracle_lib, counts, D, F, act, dtype=configs.DTYPE_BF16, seed
     ([70, 0, 33], 72, 200, configs.ACT_GELU_TANH),
     ([513, 400], 1024, 512, configs.ACT_SILU),
     ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
+    ([700, 0, 257, 1100], 512, 768, configs.ACT_GELU_ERF),
 ])
-def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, counts, D, F, act):
+@pytest.mark.parametrize("tile_rows", ["128", "256"])
+def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, monkeypatch, counts, D, F, act, tile_rows):
+    # 128: one CTA per tile; 256: CTA pairs (tcgen05 cta_group::2) sharing one tile.
+    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
     _ffn_case(abi, oracle_lib, counts, D, F, act)
 
 

@@ -23,6 +23,9 @@
 // Every barrier wait is bounded in time; on a timeout the CTA records
 // MOE_DEVERR_WAIT_TIMEOUT, unwinds, drains its MMAs and frees its TMEM.
 #include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -31,26 +34,34 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;                            // tile rows (UMMA M)
+constexpr int kRows = 128;                         // rows of A (and accumulator lanes) per CTA
 constexpr int BN = 256;                            // UMMA N
 constexpr int BK = 64;                             // k-block: one 128-byte swizzle row of bf16
 constexpr int UK = 16;                             // K of one tcgen05.mma kind::f16
-constexpr int kStages = 4;
-constexpr int kABytes = BM * BK * 2;               // 16 KB
+constexpr int kABytes = kRows * BK * 2;            // 16 KB
 constexpr int kBoxBytes = 64 * BK * 2;             // 8 KB: 64 columns x 64 k-rows
-constexpr int kBBytes = 4 * kBoxBytes;             // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;     // 48 KB
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr int kMaxE = 64;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers etc*/;
 
-// Instruction descriptor, kind::f16: D fp32, A bf16, B bf16, A K-major, B MN-major,
-// N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                            (static_cast<uint32_t>(BN >> 3) << 17) |
-                            (static_cast<uint32_t>(BM >> 4) << 24);
+// Per-variant shape: a single CTA computes 128-row tiles with the whole B; a CTA pair
+// computes 256-row tiles, each CTA holding its 128 A rows and half of the B columns.
+template <bool PAIR>
+struct Shape {
+  static constexpr int kTileRows = PAIR ? 256 : 128;
+  static constexpr int kBBoxes = PAIR ? 2 : 4;                       // 64-col B boxes per CTA
+  static constexpr int kStages = PAIR ? 7 : 4;  // fills the 227 KB of shared memory
+  static constexpr int kBBytes = kBBoxes * kBoxBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTxBytes = PAIR ? 2 * kStageBytes : kStageBytes;  // per stage, both CTAs
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
+  // Instruction descriptor, kind::f16: D fp32, A bf16, B bf16, A K-major, B MN-major,
+  // N = 256, M = tile rows.
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
+                                     (1u << 16) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                                     (static_cast<uint32_t>(kTileRows >> 4) << 24);
+};
 
 struct GemmParams {
   const int32_t* offsets;  // [E+1] expert segments of the A rows
@@ -62,19 +73,20 @@ struct GemmParams {
   uint64_t timeout_ns;
 };
 
-template <bool DUAL, int ACT>
+template <bool DUAL, int ACT, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_sm100(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+  using S = Shape<PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint8_t* sB = smem + S::kStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::kStages * S::kBBytes);
+  uint64_t* empty = full + S::kStages;
+  uint64_t* tfull = empty + S::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
@@ -86,6 +98,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int n_blocks = (p.n_out + NT - 1) / NT;
   const int num_kb = (p.K + BK - 1) / BK;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the CTA that issues the MMAs
+  const bool mma_cta = rank == 0;
+  const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -93,22 +109,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e = 0; e < p.E; ++e) {
       s_tile_start[e] = acc;
       const int m = s_seg[e + 1] - s_seg[e];
-      acc += ((m + BM - 1) / BM) * n_blocks;
+      acc += ((m + S::kTileRows - 1) / S::kTileRows) * n_blocks;
     }
     s_tile_start[p.E] = acc;
   }
   __syncthreads();
   const int total_tiles = s_tile_start[p.E];
-  if (static_cast<int>(blockIdx.x) >= total_tiles) return;  // uniform: before any allocation
+  // Uniform over the block (and over the pair: both CTAs see the same tile list).
+  if (first_tile >= total_tiles) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -117,11 +134,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (DUAL) prefetch_tensormap(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(s_tmem, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s_tmem, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR) cluster_sync_all();  // barriers and TMEM of both CTAs ready before any remote use
+  else __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
@@ -130,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     e = 0;
     while (e < p.E - 1 && tile >= s_tile_start[e + 1]) ++e;
     const int local = tile - s_tile_start[e];
-    const int m_tiles = (s_seg[e + 1] - s_seg[e] + BM - 1) / BM;
+    const int m_tiles = (s_seg[e + 1] - s_seg[e] + S::kTileRows - 1) / S::kTileRows;
     n_blk = local / m_tiles;
     m_blk = local - n_blk * m_tiles;
   };
@@ -140,10 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < total_tiles; tile += tile_stride) {
         int e, m_blk, n_blk;
         decode(tile, e, m_blk, n_blk);
-        const int row0 = s_seg[e] + m_blk * BM;
+        const int row0 = s_seg[e] + m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
         const int n0 = n_blk * NT;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns)) {
@@ -151,22 +175,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
           uint8_t* a_dst = sA + stage * kABytes;
-          uint8_t* b_dst = sB + stage * kBBytes;
+          uint8_t* b_dst = sB + stage * S::kBBytes;
           const int k0 = kb * BK;
-          tma_load_2d(a_dst, &tmA, &full[stage], k0, row0);
-          if (DUAL) {
-            tma_load_3d(b_dst, &tmB0, &full[stage], n0, k0, e);
-            tma_load_3d(b_dst + kBoxBytes, &tmB0, &full[stage], n0 + 64, k0, e);
-            tma_load_3d(b_dst + 2 * kBoxBytes, &tmB1, &full[stage], n0, k0, e);
-            tma_load_3d(b_dst + 3 * kBoxBytes, &tmB1, &full[stage], n0 + 64, k0, e);
+          if (PAIR) {
+            // Both CTAs' bytes are counted on the MMA CTA's barrier.
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (mma_cta) mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
+            tma_load_2d_pair(a_dst, &tmA, bar, k0, row0);
+            if (DUAL) {  // CTA 0 holds the W1 columns, CTA 1 the W2 columns
+              const CUtensorMap* m = rank == 0 ? &tmB0 : &tmB1;
+              tma_load_3d_pair(b_dst, m, bar, n0, k0, e);
+              tma_load_3d_pair(b_dst + kBoxBytes, m, bar, n0 + 64, k0, e);
+            } else {     // CTA r holds columns [n0 + 128r, n0 + 128r + 128)
+              const int nc = n0 + static_cast<int>(rank) * 128;
+              tma_load_3d_pair(b_dst, &tmB0, bar, nc, k0, e);
+              tma_load_3d_pair(b_dst + kBoxBytes, &tmB0, bar, nc + 64, k0, e);
+            }
           } else {
+            mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
+            tma_load_2d(a_dst, &tmA, &full[stage], k0, row0);
+            if (DUAL) {
+              tma_load_3d(b_dst, &tmB0, &full[stage], n0, k0, e);
+              tma_load_3d(b_dst + kBoxBytes, &tmB0, &full[stage], n0 + 64, k0, e);
+              tma_load_3d(b_dst + 2 * kBoxBytes, &tmB1, &full[stage], n0, k0, e);
+              tma_load_3d(b_dst + 3 * kBoxBytes, &tmB1, &full[stage], n0 + 64, k0, e);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tma_load_3d(b_dst + j * kBoxBytes, &tmB0, &full[stage], n0 + 64 * j, k0, e);
+              for (int j = 0; j < 4; ++j)
+                tma_load_3d(b_dst + j * kBoxBytes, &tmB0, &full[stage], n0 + 64 * j, k0, e);
+            }
           }
-          if (++stage == kStages) {
+          if (++stage == S::kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -174,12 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ---------------------------------------------------- MMA issuer
+    if (lane == 0 && mma_cta) {  // ------------------------------------------- MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
+      for (int tile = first_tile; ok && tile < total_tiles; tile += tile_stride, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
@@ -197,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after_sync();
           const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+          const uint32_t b_addr = smem_u32(sB + stage * S::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
             // A: K-major SW128, advance 16 elements = 32 bytes inside the swizzle row.
@@ -205,25 +245,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             // B: MN-major SW128, 64-column blocks kBoxBytes apart (LBO), 8-row k groups
             // 1024 bytes apart (SBO); advance 16 k-rows = 2048 bytes.
             const uint64_t bd = smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
-            umma_bf16_ss(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            if (PAIR) umma_bf16_ss_pair(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            else umma_bf16_ss(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);  // frees the smem stage once these MMAs have read it
-          if (++stage == kStages) {
+          // frees the smem stage (of both CTAs) once these MMAs have read it
+          if (PAIR) umma_commit_pair(&empty[stage], 0x3);
+          else umma_commit(&empty[stage]);
+          if (++stage == S::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) umma_commit(&tfull[acc]);  // accumulator complete
+        if (ok) {  // accumulator complete
+          if (PAIR) umma_commit_pair(&tfull[acc], 0x3);
+          else umma_commit(&tfull[acc]);
+        }
       }
       // Every MMA issued by this thread has completed once `drain` flips.
-      umma_commit(drain);
+      if (PAIR) umma_commit_pair(drain, 0x1);
+      else umma_commit(drain);
       if (!mbar_wait(drain, 0, p.timeout_ns)) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
     }
   } else {  // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // this warp may access TMEM lanes [32q, 32q+32)
     const int r = q * 32 + lane;
+    const uint32_t tempty_mma0 = PAIR ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
     int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+    for (int tile = first_tile; tile < total_tiles; tile += tile_stride, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, p.timeout_ns);
@@ -231,12 +279,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
         break;
       }
+      __syncwarp();
       tc_fence_after_sync();
       int e, m_blk, n_blk;
       decode(tile, e, m_blk, n_blk);
-      const int rows = min(BM, s_seg[e + 1] - s_seg[e] - m_blk * BM);
+      const int first_row = m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
+      const int rows = min(kRows, s_seg[e + 1] - s_seg[e] - first_row);
       const bool valid = r < rows;
-      const int64_t grow = static_cast<int64_t>(s_seg[e]) + m_blk * BM + r;
+      const int64_t grow = static_cast<int64_t>(s_seg[e]) + first_row + r;
       const int n0 = n_blk * NT;
       __nv_bfloat16* orow = p.out + grow * p.n_out + n0;
       const uint32_t t_row =
@@ -284,15 +334,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) {  // this warp is done with the accumulator
+        if (PAIR) mbar_arrive_cluster(tempty_mma0 + static_cast<uint32_t>(acc * 8));
+        else mbar_arrive(&tempty[acc]);
+      }
     }
   }
 
-  __syncthreads();
+  __syncwarp();  // role branches leave warps 0 and 1 divergent; the barrier below is .aligned
+  if (PAIR) cluster_sync_all();  // no CTA of the pair leaves while the other may signal it
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -341,14 +398,90 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, uint64_t n, uint64_t k, uint64
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool DUAL, int ACT>
+// Clusters of two that fit on the device at once for this kernel (cached per kernel).
+template <typename Kern>
+int max_pair_clusters(Kern kern, int smem) {
+  static int cached = 0;
+  if (cached > 0) return cached;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * num_sms());
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = num_sms() / 2;
+  }
+  cached = n;
+  return n;
+}
+
+template <bool DUAL, int ACT, bool PAIR>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const GemmParams& gp, int grid, cudaStream_t stream) {
-  auto kern = grouped_gemm_sm100<DUAL, ACT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+                        const GemmParams& gp, int64_t tiles_upper, cudaStream_t stream) {
+  using S = Shape<PAIR>;
+  auto kern = grouped_gemm_sm100<DUAL, ACT, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(a, b0, b1, gp);
-  return cudaGetLastError();
+  if (!PAIR) {
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_upper)));
+    kern<<<grid, kThreads, S::kSmemBytes, stream>>>(a, b0, b1, gp);
+    return cudaGetLastError();
+  }
+  const int clusters = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(max_pair_clusters(kern, S::kSmemBytes), tiles_upper)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = S::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, gp);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Tile shape: CTA pairs (256-row tiles) pay off when experts hold many rows; 128-row tiles
+// waste less on small or capacity-limited experts. MOE_GEMM_TILE_ROWS=128|256 overrides.
+bool use_pairs(const moe_problem& p) {
+  if (const char* env = std::getenv("MOE_GEMM_TILE_ROWS")) {
+    if (std::strcmp(env, "256") == 0) return true;
+    if (std::strcmp(env, "128") == 0) return false;
+  }
+  const int64_t R = p.N * p.k;
+  int64_t per_expert = R / p.E;
+  if (p.capacity_factor > 0.0) {
+    const int64_t C = static_cast<int64_t>(std::ceil(p.capacity_factor * static_cast<double>(p.N) *
+                                                     static_cast<double>(p.k) / static_cast<double>(p.E)));
+    per_expert = std::min(per_expert, C);
+  }
+  return per_expert >= 768;
+}
+
+template <bool DUAL, int ACT>
+cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUtensorMap& b0,
+                         const CUtensorMap& b1, const GemmParams& gp, int n_tile,
+                         cudaStream_t stream) {
+  const int64_t R = p.N * p.k;
+  const int64_t n_blocks = (gp.n_out + n_tile - 1) / n_tile;
+  if (use_pairs(p)) {
+    const int64_t tiles = ((R + 255) / 256 + p.E) * n_blocks;
+    return launch_gemm<DUAL, ACT, true>(a, b0, b1, gp, tiles, stream);
+  }
+  const int64_t tiles = ((R + 127) / 128 + p.E) * n_blocks;
+  return launch_gemm<DUAL, ACT, false>(a, b0, b1, gp, tiles, stream);
 }
 
 }  // namespace
@@ -360,10 +493,9 @@ cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const 
   if (R == 0) return cudaSuccess;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tA, tW1, tW2;
-  if (!make_map_2d(&tA, X_perm, p.D, R, BM) || !make_map_3d(&tW1, W1, p.F, p.D, p.E) ||
+  if (!make_map_2d(&tA, X_perm, p.D, R, kRows) || !make_map_3d(&tW1, W1, p.F, p.D, p.E) ||
       !make_map_3d(&tW2, W2, p.F, p.D, p.E))
     return cudaErrorInvalidValue;
-  const int64_t row_blocks = (R + BM - 1) / BM + p.E;  // upper bound over any split of R
   GemmParams g;
   g.offsets = offsets;
   g.out = static_cast<__nv_bfloat16*>(H);
@@ -372,14 +504,13 @@ cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const 
   g.n_out = static_cast<int>(p.F);
   g.err = err;
   g.timeout_ns = timeout_ns;
-  const int grid = static_cast<int>(std::min<int64_t>(num_sms(), row_blocks * ((p.F + 127) / 128)));
   switch (p.activation) {
     case MOE_ACT_SILU:
-      return launch_gemm<true, MOE_ACT_SILU>(tA, tW1, tW2, g, grid, stream);
+      return launch_shape<true, MOE_ACT_SILU>(p, tA, tW1, tW2, g, 128, stream);
     case MOE_ACT_GELU_ERF:
-      return launch_gemm<true, MOE_ACT_GELU_ERF>(tA, tW1, tW2, g, grid, stream);
+      return launch_shape<true, MOE_ACT_GELU_ERF>(p, tA, tW1, tW2, g, 128, stream);
     default:
-      return launch_gemm<true, MOE_ACT_GELU_TANH>(tA, tW1, tW2, g, grid, stream);
+      return launch_shape<true, MOE_ACT_GELU_TANH>(p, tA, tW1, tW2, g, 128, stream);
   }
 }
 
@@ -390,9 +521,8 @@ cudaError_t launch_ffn_down_sm100(const moe_problem& p, const void* H, const int
   if (R == 0) return cudaSuccess;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tA, tW3;
-  if (!make_map_2d(&tA, H, p.F, R, BM) || !make_map_3d(&tW3, W3, p.D, p.F, p.E))
+  if (!make_map_2d(&tA, H, p.F, R, kRows) || !make_map_3d(&tW3, W3, p.D, p.F, p.E))
     return cudaErrorInvalidValue;
-  const int64_t row_blocks = (R + BM - 1) / BM + p.E;
   GemmParams g;
   g.offsets = offsets;
   g.out = static_cast<__nv_bfloat16*>(Y);
@@ -401,8 +531,7 @@ cudaError_t launch_ffn_down_sm100(const moe_problem& p, const void* H, const int
   g.n_out = static_cast<int>(p.D);
   g.err = err;
   g.timeout_ns = timeout_ns;
-  const int grid = static_cast<int>(std::min<int64_t>(num_sms(), row_blocks * ((p.D + 255) / 256)));
-  return launch_gemm<false, MOE_ACT_SILU>(tA, tW3, tW3, g, grid, stream);
+  return launch_shape<false, MOE_ACT_SILU>(p, tA, tW3, tW3, g, 256, stream);
 }
 
 }  // namespace moe
