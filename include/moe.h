@@ -153,7 +153,7 @@ moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk
  * fixed 64 KiB array inside the library (held on every GPU that loads the library until the
  * process exits). There is no counterpart on the pages; this is a deployment variant.
  *   - row_token is required (it is an output here, not workspace).
- *   - Limit: ceil(N*k / 2048) * E <= 16384 counters (e.g. N*k <= 524288 records at E = 64);
+ *   - Limit: ceil(N*k / 1024) * E <= 16384 counters (e.g. N*k <= 262144 records at E = 64);
  *     larger problems return MOE_ERR_UNSUPPORTED -- use moe_dispatch.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.

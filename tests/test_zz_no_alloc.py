@@ -25,7 +25,7 @@ def _cfg(N, E, k, cf, D=64):
 
 def test_noalloc_rejects_oversized_problems_on_host():
     abi = _abi()
-    p = abi.problem(_cfg(300000, 64, 2, 1.25))   # ceil(600000/2048)*64 = 18752 > 16384
+    p = abi.problem(_cfg(300000, 64, 2, 1.25))   # ceil(600000/1024)*64 = 37504 > 16384
     st = abi.lib.moe_dispatch_noalloc(ctypes.byref(p), None, 8, 8, 8, 8, 8, 8, None, None)
     assert st == abi.MOE_ERR_UNSUPPORTED
     assert b"exceeds the fixed scratch" in abi.lib.moe_last_error()

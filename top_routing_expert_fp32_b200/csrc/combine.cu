@@ -50,7 +50,7 @@ struct Vec16<float> {
   }
 };
 
-template <typename T>
+template <typename T, int KMAX, bool BATCH>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4* __restrict__ Y, const int32_t* __restrict__ idx,
                    const float* __restrict__ gate, const int32_t* __restrict__ offsets,
@@ -74,20 +74,40 @@ __global__ void __launch_bounds__(kThreads)
     s_g[j] = gate[rec];
   }
   __syncthreads();
-  for (int64_t c = threadIdx.x; c < chunks_per_row; c += kThreads) {
-    float acc[V];
+  // With BATCH (long rows), kBatch chunks per thread are loaded (all k rows) before any is
+  // used, so a thread keeps about 8 16-byte loads in flight instead of one round trip per
+  // chunk; short rows keep the register count (and occupancy) of one chunk at a time.
+  constexpr int kBatch = (!BATCH || KMAX >= 8) ? 1 : 8 / KMAX;
+  for (int64_t c0 = threadIdx.x; c0 < chunks_per_row; c0 += kThreads * kBatch) {
+    uint4 yv[kBatch][KMAX];
 #pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int64_t row = s_row[j];
-      if (row < 0) continue;
-      float y[V];
-      Vec16<T>::unpack(__ldg(Y + row * chunks_per_row + c), y);
-      const float g = s_g[j];
+    for (int b = 0; b < kBatch; ++b) {
+      const int64_t c = c0 + b * kThreads;
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = fmaf(g, y[i], acc[i]);
+      for (int j = 0; j < KMAX; ++j) {
+        yv[b][j] = make_uint4(0u, 0u, 0u, 0u);
+        if (j < k && c < chunks_per_row && s_row[j] >= 0)
+          yv[b][j] = __ldg(Y + s_row[j] * chunks_per_row + c);
+      }
     }
-    out[t * chunks_per_row + c] = Vec16<T>::pack(acc);
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int64_t c = c0 + b * kThreads;
+      if (c >= chunks_per_row) break;
+      float acc[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j >= k || s_row[j] < 0) continue;
+        float y[V];
+        Vec16<T>::unpack(yv[b][j], y);
+        const float g = s_g[j];
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(g, y[i], acc[i]);
+      }
+      out[t * chunks_per_row + c] = Vec16<T>::pack(acc);
+    }
   }
 }
 
@@ -100,14 +120,32 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
   const int64_t elem = p.dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int64_t chunks = p.D * elem / 16;
   const dim3 grid(static_cast<unsigned>(p.N));
-  if (p.dtype == MOE_DTYPE_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint4*>(Y), idx, gate, offsets, pos, dropped, static_cast<uint4*>(out),
-        p.N, p.k, p.E, chunks, err);
-  else
-    combine_kernel<float><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint4*>(Y), idx, gate, offsets, pos, dropped, static_cast<uint4*>(out),
-        p.N, p.k, p.E, chunks, err);
+  const uint4* y = static_cast<const uint4*>(Y);
+  uint4* o = static_cast<uint4*>(out);
+  const bool batch = chunks >= 4 * kThreads;
+#define MOE_COMBINE(T, KM)                                                                     \
+  do {                                                                                         \
+    if (batch)                                                                                 \
+      combine_kernel<T, KM, true><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,   \
+                                                                 dropped, o, p.N, p.k, p.E,    \
+                                                                 chunks, err);                 \
+    else                                                                                       \
+      combine_kernel<T, KM, false><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,  \
+                                                                  dropped, o, p.N, p.k, p.E,   \
+                                                                  chunks, err);                \
+  } while (0)
+  if (p.dtype == MOE_DTYPE_BF16) {
+    if (p.k <= 1) MOE_COMBINE(__nv_bfloat16, 1);
+    else if (p.k <= 2) MOE_COMBINE(__nv_bfloat16, 2);
+    else if (p.k <= 4) MOE_COMBINE(__nv_bfloat16, 4);
+    else MOE_COMBINE(__nv_bfloat16, 8);
+  } else {
+    if (p.k <= 1) MOE_COMBINE(float, 1);
+    else if (p.k <= 2) MOE_COMBINE(float, 2);
+    else if (p.k <= 4) MOE_COMBINE(float, 4);
+    else MOE_COMBINE(float, 8);
+  }
+#undef MOE_COMBINE
   return cudaGetLastError();
 }
 

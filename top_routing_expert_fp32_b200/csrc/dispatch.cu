@@ -24,7 +24,7 @@ namespace moe {
 namespace {
 
 constexpr int kMaxE = 64;
-constexpr int kAssignThreads = 1024;  // 32 warps
+constexpr int kAssignThreads = 1024;  // 32 warps: one tile = one chunk
 constexpr int kCountThreads = 256;
 
 __global__ void __launch_bounds__(kCountThreads)
@@ -35,12 +35,24 @@ __global__ void __launch_bounds__(kCountThreads)
   __syncthreads();
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kDispatchChunk;
   const int64_t r1 = std::min<int64_t>(r0 + kDispatchChunk, R);
-  for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
-    const int64_t j = r / N, t = r - j * N;
-    const int e = idx[t * k + j];
-    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
-    else record_error(err, MOE_DEVERR_BAD_INDEX);
+  constexpr int kPer = kDispatchChunk / kCountThreads;  // records per thread, loaded together
+  int ev[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int64_t r = r0 + threadIdx.x + static_cast<int64_t>(u) * kCountThreads;
+    ev[u] = -1;
+    if (r < r1) {
+      const int64_t j = r / N, t = r - j * N;
+      ev[u] = idx[t * k + j];
+      if (ev[u] < 0 || ev[u] >= E) {
+        record_error(err, MOE_DEVERR_BAD_INDEX);
+        ev[u] = -1;
+      }
+    }
   }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u)
+    if (ev[u] >= 0) atomicAdd(&hist[ev[u]], 1);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
@@ -137,27 +149,29 @@ __global__ void __launch_bounds__(kAssignThreads)
   }
 }
 
-constexpr int kGatherStages = 4;
-constexpr uint32_t kPieceBytes = 16384;
+constexpr int kGatherMaxStages = 16;
+constexpr uint32_t kMaxPieceBytes = 16384;
+constexpr uint32_t kGatherSmem = 64 * 1024;
 constexpr uint64_t kGatherTimeoutNs = 2000000000ull;
 
-// One warp per block. Pieces q = blockIdx.x + i*gridDim.x, i = 0, 1, ...; piece q covers
-// bytes [ (q % P) * kPieceBytes, ... ) of row q / P.
+// One warp per block. A row is copied in pieces of piece_bytes (= the row when it is at most
+// 16 KB); piece q = blockIdx.x + i*gridDim.x covers bytes [(q % P) * piece_bytes, ...) of row
+// q / P. `stages` pieces (64 KB of shared memory / piece size, at most 16) are in flight.
 __global__ void __launch_bounds__(32)
     gather_kernel(const uint8_t* __restrict__ X, const int32_t* __restrict__ row_token,
                   const int32_t* __restrict__ offsets, int E, uint32_t row_bytes,
-                  uint8_t* __restrict__ X_perm, int* err) {
+                  uint32_t piece_bytes, int stages, uint8_t* __restrict__ X_perm, int* err) {
   extern __shared__ __align__(128) uint8_t g_smem[];
-  __shared__ __align__(8) uint64_t bars[kGatherStages];
+  __shared__ __align__(8) uint64_t bars[kGatherMaxStages];
   const int lane = threadIdx.x;
   const int64_t rows = offsets[E];
-  const int64_t P = (row_bytes + kPieceBytes - 1) / kPieceBytes;
+  const int64_t P = (row_bytes + piece_bytes - 1) / piece_bytes;
   const int64_t total = rows * P;
   if (static_cast<int64_t>(blockIdx.x) >= total) return;
   const int64_t n = (total - blockIdx.x + gridDim.x - 1) / gridDim.x;  // pieces of this block
 
   if (lane == 0) {
-    for (int s = 0; s < kGatherStages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
   }
   __syncwarp();
@@ -165,9 +179,9 @@ __global__ void __launch_bounds__(32)
   auto piece = [&](int64_t i, int64_t& row, uint32_t& off, uint32_t& bytes) {
     const int64_t q = blockIdx.x + i * gridDim.x;
     row = q / P;
-    off = static_cast<uint32_t>((q - row * P) * kPieceBytes);
+    off = static_cast<uint32_t>((q - row * P) * piece_bytes);
     const uint32_t rest = row_bytes - off;
-    bytes = rest < kPieceBytes ? rest : kPieceBytes;
+    bytes = rest < piece_bytes ? rest : piece_bytes;
   };
   // Token of the row of load index i, fetched 32 at a time by the whole warp.
   int tok_batch = -1;
@@ -193,21 +207,21 @@ __global__ void __launch_bounds__(32)
     piece(i, row, off, bytes);
     const int tok = token_of(i);
     if (lane == 0) {
-      const int s = static_cast<int>(i % kGatherStages);
+      const int s = static_cast<int>(i % stages);
       mbar_arrive_expect_tx(&bars[s], bytes);
-      bulk_g2s(g_smem + s * kPieceBytes, X + static_cast<int64_t>(tok) * row_bytes + off, bytes,
-               &bars[s]);
+      bulk_g2s(g_smem + static_cast<uint32_t>(s) * piece_bytes,
+               X + static_cast<int64_t>(tok) * row_bytes + off, bytes, &bars[s]);
     }
   };
 
-  const int64_t pro = std::min<int64_t>(n, kGatherStages);
+  const int64_t pro = n < stages ? n : stages;
   for (int64_t i = 0; i < pro; ++i) issue_load(i);
   int64_t issued = pro;  // loads [0, issued) have been issued
   int64_t i = 0;
   bool ok = true;
   for (; i < n; ++i) {
-    const int s = static_cast<int>(i % kGatherStages);
-    const uint32_t parity = static_cast<uint32_t>((i / kGatherStages) & 1);
+    const int s = static_cast<int>(i % stages);
+    const uint32_t parity = static_cast<uint32_t>((i / stages) & 1);
     if (lane == 0) ok = mbar_wait(&bars[s], parity, kGatherTimeoutNs);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     if (!ok) {
@@ -218,10 +232,11 @@ __global__ void __launch_bounds__(32)
       int64_t row;
       uint32_t off, bytes;
       piece(i, row, off, bytes);
-      bulk_s2g(X_perm + row * row_bytes + off, g_smem + s * kPieceBytes, bytes);
+      bulk_s2g(X_perm + row * row_bytes + off, g_smem + static_cast<uint32_t>(s) * piece_bytes,
+               bytes);
       bulk_commit();
     }
-    const int64_t nxt = i - 1 + kGatherStages;  // refill the stage read by store i-1
+    const int64_t nxt = i - 1 + stages;  // refill the stage read by store i-1
     if (i >= 1 && nxt < n) {
       if (lane == 0) bulk_wait_read<1>();
       __syncwarp();
@@ -234,7 +249,7 @@ __global__ void __launch_bounds__(32)
     // After a timeout, loads [i, issued) may still be landing in shared memory: wait for
     // each of them (bounded) before the block exits.
     for (int64_t L = i; !ok && L < issued; ++L)
-      (void)mbar_wait(&bars[L % kGatherStages], static_cast<uint32_t>((L / kGatherStages) & 1),
+      (void)mbar_wait(&bars[L % stages], static_cast<uint32_t>((L / stages) & 1),
                       kGatherTimeoutNs / 16);
   }
 }
@@ -271,15 +286,18 @@ cudaError_t launch_gather(const moe_problem& p, const void* X, const int32_t* ro
   if (R == 0) return cudaSuccess;
   const uint32_t elem = p.dtype == MOE_DTYPE_BF16 ? 2u : 4u;
   const uint32_t row_bytes = static_cast<uint32_t>(p.D) * elem;
-  const int64_t P = (row_bytes + kPieceBytes - 1) / kPieceBytes;
+  const uint32_t piece = row_bytes < kMaxPieceBytes ? row_bytes : kMaxPieceBytes;
+  const int stages = static_cast<int>(std::min<uint32_t>(kGatherMaxStages, kGatherSmem / piece));
+  const int64_t P = (row_bytes + piece - 1) / piece;
   const int64_t max_pieces = R * P;
   const int grid = static_cast<int>(std::min<int64_t>(max_pieces, int64_t(num_sms()) * 3));
-  const size_t smem = kGatherStages * kPieceBytes;
+  const size_t smem = static_cast<size_t>(stages) * piece;
   cudaError_t e = cudaFuncSetAttribute(
-      gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGatherSmem));
   if (e != cudaSuccess) return e;
   gather_kernel<<<grid, 32, smem, stream>>>(static_cast<const uint8_t*>(X), row_token, offsets,
-                                            p.E, row_bytes, static_cast<uint8_t*>(X_perm), err);
+                                            p.E, row_bytes, piece, stages,
+                                            static_cast<uint8_t*>(X_perm), err);
   return cudaGetLastError();
 }
 

@@ -23,7 +23,7 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
                          float* prob_colsum, int* err, cudaStream_t stream);
 
 // Records are processed in chunks of this many for the slot assignment.
-constexpr int kDispatchChunk = 2048;
+constexpr int kDispatchChunk = 1024;
 
 int dispatch_num_chunks(int64_t records);
 

@@ -16,7 +16,7 @@
 
 namespace {
 
-// Per-chunk expert counters: ceil(N*k / 2048) * E int32 values must fit.
+// Per-chunk expert counters: ceil(N*k / 1024) * E int32 values must fit.
 constexpr int kScratchInts = 16384;  // 64 KiB
 static __device__ __align__(256) int32_t g_dispatch_counts[kScratchInts];
 
@@ -72,7 +72,7 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_problem* p, const void* X,
   const int64_t need = static_cast<int64_t>(moe::dispatch_num_chunks(records)) * p->E;
   if (need > kScratchInts)
     return noalloc_fail(MOE_ERR_UNSUPPORTED,
-                        "ceil(N*k/2048)*E = " + std::to_string(need) +
+                        "ceil(N*k/1024)*E = " + std::to_string(need) +
                             " exceeds the fixed scratch of " + std::to_string(kScratchInts) +
                             " counters; use moe_dispatch with a workspace");
   int32_t* counts = nullptr;
