@@ -61,6 +61,11 @@ struct Shape {
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
                                      (1u << 16) | (static_cast<uint32_t>(BN >> 3) << 17) |
                                      (static_cast<uint32_t>(kTileRows >> 4) << 24);
+  // Single-CTA tiles whose rows all fit in 64 (an expert's last row block) use M = 64: the
+  // accumulator then holds row 16q + l in TMEM lane 32q + l (lanes 0-15 of each quarter).
+  static constexpr uint32_t kIdesc64 = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
+                                       (1u << 16) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                                       (static_cast<uint32_t>(64 >> 4) << 24);
 };
 
 struct GemmParams {
@@ -229,6 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+        uint32_t idesc = S::kIdesc;
+        if (!PAIR) {
+          int e, m_blk, n_blk;
+          decode(tile, e, m_blk, n_blk);
+          if (s_seg[e + 1] - s_seg[e] - m_blk * kRows <= 64) idesc = S::kIdesc64;
+        }
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
             record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
@@ -245,8 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // B: MN-major SW128, 64-column blocks kBoxBytes apart (LBO), 8-row k groups
             // 1024 bytes apart (SBO); advance 16 k-rows = 2048 bytes.
             const uint64_t bd = smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
-            if (PAIR) umma_bf16_ss_pair(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0 ? 1u : 0u);
-            else umma_bf16_ss(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            if (PAIR) umma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else umma_bf16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           // frees the smem stage (of both CTAs) once these MMAs have read it
           if (PAIR) umma_commit_pair(&empty[stage], 0x3);
@@ -268,7 +279,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {  // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // this warp may access TMEM lanes [32q, 32q+32)
-    const int r = q * 32 + lane;
     const uint32_t tempty_mma0 = PAIR ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
     int it = 0;
     for (int tile = first_tile; tile < total_tiles; tile += tile_stride, ++it) {
@@ -285,6 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode(tile, e, m_blk, n_blk);
       const int first_row = m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
       const int rows = min(kRows, s_seg[e + 1] - s_seg[e] - first_row);
+      // Row held by this thread's TMEM lane (M = 64 tiles use lanes 0-15 of each quarter).
+      const bool half = !PAIR && rows <= 64;
+      const int r = half ? (lane < 16 ? 16 * q + lane : kRows) : q * 32 + lane;
       const bool valid = r < rows;
       const int64_t grow = static_cast<int64_t>(s_seg[e]) + first_row + r;
       const int n0 = n_blk * NT;
