@@ -5,7 +5,7 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl re
 A step is one pass of the whole hot path (route -> dispatch -> expert up/down -> combine)
 over one batch of the workload, enqueued through the C ABI with CUDA events between the
 kernels (the same kernels moe_forward launches). Inputs are resident in HBM; L2 is flushed
-(a 512 MiB write) between timed steps, outside the per-step events. Rank 0 prints one JSON
+(a 512 MiB write, then a read of it) between timed steps, outside the per-step events. Rank 0 prints one JSON
 line. With N>1 (torchrun) every rank runs an independent replica on its own GPU (the layer
 has no data-path collective); value = tokens of all ranks / max-over-ranks time.
 
@@ -244,6 +244,13 @@ def run_gpu(args, cfg, world, rank, device):
     Y = torch.empty((R, D), dtype=tdt, device=device)
     out = torch.empty((N, D), dtype=tdt, device=device)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.int32, device=device)
+    flush_sum = torch.empty((), dtype=torch.int64, device=device)
+
+    def flush_l2():
+        # Write 512 MiB (evicts X, H, Y), then read it back so that the dirty lines the write
+        # leaves in L2 are written back here, not inside the next step's first kernel.
+        flush.fill_(1)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
     stream = torch.cuda.current_stream(device)
 
     names = ["route", "dispatch", "up", "down", "combine"]
@@ -267,7 +274,7 @@ def run_gpu(args, cfg, world, rank, device):
 
     for _ in range(args.warmup):
         step(new_events())
-        flush.fill_(1)
+        flush_l2()
     torch.cuda.synchronize(device)
     if abi.device_error(ws) != 0:
         raise RuntimeError("device error during warm-up")
@@ -281,7 +288,7 @@ def run_gpu(args, cfg, world, rank, device):
         ev = new_events()
         step(ev)
         evs.append(ev)
-        flush.fill_(1)   # outside the step's events: evicts X, H, Y from L2
+        flush_l2()   # outside the step's events
     torch.cuda.synchronize(device)
     barrier(device)
     t_wall1 = time.time()
@@ -321,22 +328,33 @@ def run_gpu(args, cfg, world, rank, device):
     ffn_ms = mean["up"] + mean["down"]
     gemm_tflops = 6.0 * kept * D * F / ffn_ms / 1e9
 
-    if cfg.dtype == configs.DTYPE_BF16 and kept >= 4 * 128:
-        dom = "up"
+    # Roofline of the up-projection kernel: the larger of its FLOPs at the bf16 peak and its
+    # algorithmic bytes at the HBM peak (A rows read once, the weights of every expert that
+    # keeps a row read once, H written once).
+    used = int((offsets[1:] - offsets[:-1] > 0).sum().item())
+    bytes_up = kept * D * es + used * 2.0 * D * F * es + kept * F * es
+    t_tensor = flops_up / (tc * 1e12) if cfg.dtype == configs.DTYPE_BF16 else 0.0
+    t_hbm = bytes_up / (hbm * 1e9)
+    dom = "up"
+    psrc = (f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback")
+    if t_tensor >= t_hbm:
         roof = {"kernel": "grouped_gemm_sm100<dual> (expert up-projection + gating)",
                 "bound": "tensor", "achieved": kern["up"]["TFLOP/s"], "peak": tc,
                 "unit": "TFLOP/s", "frac": kern["up"]["TFLOP/s"] / tc,
-                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
-                if peak_src == "measured" else "fallback",
-                "flops_per_launch": flops_up}
+                "peak_source": psrc + ", bf16 burst", "flops_per_launch": flops_up}
     else:
-        # decode-sized / fp32: bound by streaming the expert weights through HBM
-        dom = "up"
-        wbytes = 2.0 * E * D * F * es
-        gbs = wbytes / mean["up"] / 1e6
-        roof = {"kernel": "expert up-projection (weight streaming)", "bound": "hbm",
-                "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                "peak_source": peak_src, "bytes_per_launch": wbytes}
+        gbs = bytes_up / mean["up"] / 1e6
+        roof = {"kernel": "expert up-projection (bound by streaming the used experts' weights)",
+                "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                "frac": gbs / hbm, "peak_source": psrc, "bytes_per_launch": bytes_up}
+    roof["min_us"] = {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6}
+    roof["experts_used"] = used
+    # Same two-sided bound for both GEMMs: frac_roofline = bound time / measured time.
+    bytes_down = kept * F * es + used * 1.0 * D * F * es + kept * D * es
+    for n, fl, by in (("up", flops_up, bytes_up), ("down", flops_down, bytes_down)):
+        t_min = max(fl / (tc * 1e12) if cfg.dtype == configs.DTYPE_BF16 else 0.0,
+                    by / (hbm * 1e9))
+        kern[n]["frac_roofline"] = t_min * 1e3 / mean[n]
     roof["traffic"] = traffic_from_profile("up", cfg.name)
 
     # end-to-end through the public host-buffer entry point
@@ -350,7 +368,7 @@ def run_gpu(args, cfg, world, rank, device):
     e1 = torch.cuda.Event(enable_timing=True)
     e_total = 0.0
     for _ in range(args.steps):
-        flush.fill_(1)
+        flush_l2()
         e0.record(stream)
         abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
         e1.record(stream)
@@ -371,7 +389,7 @@ def run_gpu(args, cfg, world, rank, device):
                 + (", bias~N(0,2)" if cfg.router_bias_var > 0 else ""),
         "config": {"workload": workload_desc(cfg), "tokens_per_gpu": N,
                    "parallelism": f"replicas x{world} (no data-path collective)",
-                   "l2": "flushed between steps (512 MiB write outside the step events)",
+                   "l2": "flushed between steps (512 MiB write + read-back, outside the step events)",
                    "kept_records": kept,
                    "grouped_gemm_TFLOP/s": gemm_tflops,
                    "grouped_gemm_frac_bf16_peak": gemm_tflops / tc,

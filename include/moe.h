@@ -113,7 +113,8 @@ moe_status moe_workspace_size(const moe_problem* p, size_t* bytes);
 /* Router + softmax + top-k + gates (Grok-1 book 5.2, 5.2.3; walkthrough 1.1, 1.2;
  * LLMs-from-scratch 12.1).
  *   X != NULL : logits = fp32(X) . W_r (+ bias), fp32 accumulation; written to `logits`
- *               when `logits` != NULL.
+ *               when `logits` != NULL. bf16 X runs on the tensor cores with W_r split into
+ *               three bf16 terms (products exact, sums in fp32); fp32 X on fp32 FMA.
  *   X == NULL : `logits` is read as an INPUT [N,E] (routing from given fp32 logits).
  *   topk_idx  : the k experts with the largest fp32 logits, in descending order; equal
  *               logits are ordered by lower expert index.
@@ -121,7 +122,8 @@ moe_status moe_workspace_size(const moe_problem* p, size_t* bytes);
  *               logits (= probs[idx] / sum of the selected probs).
  *   prob_colsum (optional, [E]): sum over tokens of the full softmax, for the balance loss
  *               (walkthrough 2.1); summed in a fixed order.
- *   W_r may be NULL only when X is NULL. bias (optional, [E] fp32) is added to the logits.
+ *   W_r may be NULL only when X is NULL. bias (optional, [E] fp32) is added to computed
+ *   logits; given logits (X == NULL) are used as they are.
  * Workspace: moe_workspace_size bytes. */
 moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, const float* bias,
                      float* logits, int32_t* topk_idx, float* topk_gate, float* prob_colsum,

@@ -57,7 +57,9 @@ def test_route_from_logits_bitexact(abi, oracle_lib, N, E, k, renorm, ties):
     (configs.DTYPE_F32, 64, 64, 4, 2, 1, 0.0), (configs.DTYPE_BF16, 77, 72, 6, 3, 0, 0.0),
     (configs.DTYPE_F32, 130, 100, 13, 1, 1, 1.0), (configs.DTYPE_BF16, 257, 6144, 8, 2, 0, 0.0),
     (configs.DTYPE_BF16, 600, 520, 33, 3, 1, 1.0), (configs.DTYPE_F32, 300, 200, 24, 2, 0, 0.0),
-    (configs.DTYPE_BF16, 64, 4096, 8, 2, 1, 0.0), (configs.DTYPE_BF16, 129, 1000, 64, 8, 0, 2.0)])
+    (configs.DTYPE_BF16, 64, 4096, 8, 2, 1, 0.0), (configs.DTYPE_BF16, 129, 1000, 64, 8, 0, 2.0),
+    (configs.DTYPE_BF16, 20000, 136, 64, 2, 1, 2.0), (configs.DTYPE_BF16, 300, 64, 1, 1, 1, 0.0),
+    (configs.DTYPE_BF16, 1111, 328, 13, 4, 0, 1.0)])
 def test_route_from_x(abi, oracle_lib, dtype, N, D, E, k, renorm, bias_var):
     cfg = _cfg(N, D, 64, E, k, dtype=dtype, renorm=renorm, bias_var=bias_var)
     inp = inputs.make_inputs(cfg, "cuda", seed=3, weights=False)
@@ -225,6 +227,19 @@ def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, monkeypatch, counts, D, F, act
     # 128: one CTA per tile; 256: CTA pairs (tcgen05 cta_group::2) sharing one tile.
     monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
     _ffn_case(abi, oracle_lib, counts, D, F, act)
+
+
+@pytest.mark.parametrize("counts,D,F", [
+    ([129, 127, 128, 0, 5, 256, 1, 64], 256, 384),
+    ([700, 0, 257, 1100], 512, 768),
+    ([3, 0, 200, 1, 64, 65, 0, 128, 7], 128, 1280),
+])
+@pytest.mark.parametrize("tile_rows,ngroup", [("128", "2"), ("128", "4"), ("256", "3")])
+def test_expert_ffn_tile_groups(abi, oracle_lib, monkeypatch, counts, D, F, tile_rows, ngroup):
+    # Tiles visited in groups of column blocks (a shorter last group included).
+    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
+    monkeypatch.setenv("MOE_GEMM_NGROUP", ngroup)
+    _ffn_case(abi, oracle_lib, counts, D, F, configs.ACT_SILU, seed=3)
 
 
 def test_expert_ffn_f32(abi, oracle_lib):

@@ -63,7 +63,8 @@ size_t elem_size(const moe_problem& p) { return p.dtype == MOE_DTYPE_BF16 ? 2 : 
 
 // Device workspace regions (byte offsets from the workspace base).
 struct Layout {
-  size_t err, colsum_part, counts, idx, gate, pos, dropped, load, offsets, row_token, xperm, h, y;
+  size_t err, colsum_part, wt, zpart, counts, idx, gate, pos, dropped, load, offsets, row_token,
+      xperm, h, y;
   size_t total;       // moe_forward and every other entry point
   size_t xin, xout;   // moe_forward_host only
   size_t total_host;
@@ -81,6 +82,8 @@ Layout make_layout(const moe_problem& p) {
   const size_t es = elem_size(p);
   L.err = take(256);
   L.colsum_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)) * p.E);
+  L.wt = take(route_tc_wt_bytes(p));
+  L.zpart = take(route_tc_zpart_bytes(p));
   L.counts = take(sizeof(int32_t) * static_cast<size_t>(dispatch_num_chunks(R)) * p.E);
   L.idx = take(sizeof(int32_t) * R);
   L.gate = take(sizeof(float) * R);
@@ -241,7 +244,8 @@ moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, c
     return MOE_OK;
   }
   MOE_CUDA(launch_route(p, X, W_r, bias, logits, idx, gate, at<float>(ws, L.colsum_part),
-                        prob_colsum, err, stream),
+                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), at<float>(ws, L.zpart), err,
+                        wait_timeout_ns(), stream),
            "route");
   MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps, dr,
                               row_token, err, stream),
@@ -300,7 +304,8 @@ moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, cons
     return MOE_OK;
   }
   MOE_CUDA(launch_route(*p, X, W_r, bias, logits, topk_idx, topk_gate, at<float>(ws, L.colsum_part),
-                        prob_colsum, at<int>(ws, L.err), s),
+                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), at<float>(ws, L.zpart),
+                        at<int>(ws, L.err), wait_timeout_ns(), s),
            "route");
   return MOE_OK;
 }

@@ -17,8 +17,12 @@
 //                   fp32, bf16 rounding, masked 16-byte stores (rows past the expert's segment
 //                   are never written). The accumulator is double buffered, so the epilogue
 //                   of tile i overlaps the main loop of tile i+1.
-// Tiles: per expert ceil(M_e/128) row blocks x ceil(N/NT) column blocks, enumerated expert by
-// expert with row blocks innermost (consecutive CTAs share a weight column block through L2).
+// Tiles: per expert ceil(M_e/128) row blocks x ceil(N/NT) column blocks. The column blocks
+// are cut into groups of G; tiles run group by group, inside a group expert by expert, then
+// column block, with row blocks innermost (consecutive CTAs share a weight column block
+// through L2). G = all column blocks gives plain expert-by-expert order; a small G makes the
+// CTAs resident at any moment work on several experts at once, so experts with few rows
+// (bound by streaming their weights) run beside experts with many rows (bound by the MMAs).
 // Per-expert row counts are read from device memory: the host never learns them.
 // Every barrier wait is bounded in time; on a timeout the CTA records
 // MOE_DEVERR_WAIT_TIMEOUT, unwinds, drains its MMAs and frees its TMEM.
@@ -74,6 +78,7 @@ struct GemmParams {
   int E;
   int K;                   // reduction length (D for GEMM1, F for GEMM2)
   int n_out;               // output columns (F for GEMM1, D for GEMM2)
+  int n_group;             // column blocks per tile group (>= 1)
   int* err;
   uint64_t timeout_ns;
 };
@@ -95,8 +100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
-  int* s_tile_start = reinterpret_cast<int*>(s_tmem + 1);  // [E+1]
-  int* s_seg = s_tile_start + (kMaxE + 1);                 // [E+1]
+  int* s_mstart = reinterpret_cast<int*>(s_tmem + 1);  // [E+1] first row block of expert e
+  int* s_seg = s_mstart + (kMaxE + 1);                 // [E+1]
 
   constexpr int NT = DUAL ? 128 : 256;  // output columns per tile
   const int warp = threadIdx.x >> 5;
@@ -112,14 +117,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     for (int e = 0; e <= p.E; ++e) s_seg[e] = p.offsets[e];
     for (int e = 0; e < p.E; ++e) {
-      s_tile_start[e] = acc;
+      s_mstart[e] = acc;
       const int m = s_seg[e + 1] - s_seg[e];
-      acc += ((m + S::kTileRows - 1) / S::kTileRows) * n_blocks;
+      acc += (m + S::kTileRows - 1) / S::kTileRows;
     }
-    s_tile_start[p.E] = acc;
+    s_mstart[p.E] = acc;
   }
   __syncthreads();
-  const int total_tiles = s_tile_start[p.E];
+  const int m_total = s_mstart[p.E];
+  const int total_tiles = m_total * n_blocks;
+  const int group = min(max(p.n_group, 1), n_blocks);
+  const int group_tiles = m_total * group;
   // Uniform over the block (and over the pair: both CTAs see the same tile list).
   if (first_tile >= total_tiles) return;
 
@@ -154,14 +162,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
-  // tile -> (expert, row block, column block)
+  // tile -> (expert, row block, column block). Group c holds g column blocks (g = group but
+  // for a shorter last group); inside it expert e owns g * m_tiles(e) consecutive tiles.
   auto decode = [&](int tile, int& e, int& m_blk, int& n_blk) {
+    const int c = tile / group_tiles;
+    const int g = min(group, n_blocks - c * group);
+    int local = tile - c * group_tiles;
     e = 0;
-    while (e < p.E - 1 && tile >= s_tile_start[e + 1]) ++e;
-    const int local = tile - s_tile_start[e];
-    const int m_tiles = (s_seg[e + 1] - s_seg[e] + S::kTileRows - 1) / S::kTileRows;
-    n_blk = local / m_tiles;
-    m_blk = local - n_blk * m_tiles;
+    while (e < p.E - 1 && local >= s_mstart[e + 1] * g) ++e;
+    local -= s_mstart[e] * g;
+    const int m_tiles = s_mstart[e + 1] - s_mstart[e];
+    const int n_in = local / m_tiles;
+    m_blk = local - n_in * m_tiles;
+    n_blk = c * group + n_in;
   };
 
   if (warp == 0) {
@@ -483,12 +496,26 @@ bool use_pairs(const moe_problem& p) {
   return per_expert >= 768;
 }
 
+// Column blocks per tile group. Experts that hold many rows (CTA-pair tiles) keep the
+// expert-by-expert order, which keeps an expert's A rows in L2 across its column blocks.
+// Otherwise groups of kGroup blocks mix experts of all sizes among the resident CTAs.
+// MOE_GEMM_NGROUP=<n> overrides (testing and tuning).
+int column_group(bool pairs, int64_t n_blocks) {
+  constexpr int kGroup = 8;
+  if (const char* env = std::getenv("MOE_GEMM_NGROUP")) {
+    const int g = std::atoi(env);
+    if (g > 0) return static_cast<int>(std::min<int64_t>(g, n_blocks));
+  }
+  return static_cast<int>(pairs ? n_blocks : std::min<int64_t>(kGroup, n_blocks));
+}
+
 template <bool DUAL, int ACT>
 cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUtensorMap& b0,
-                         const CUtensorMap& b1, const GemmParams& gp, int n_tile,
+                         const CUtensorMap& b1, GemmParams gp, int n_tile,
                          cudaStream_t stream) {
   const int64_t R = p.N * p.k;
   const int64_t n_blocks = (gp.n_out + n_tile - 1) / n_tile;
+  gp.n_group = column_group(use_pairs(p), n_blocks);
   if (use_pairs(p)) {
     const int64_t tiles = ((R + 255) / 256 + p.E) * n_blocks;
     return launch_gemm<DUAL, ACT, true>(a, b0, b1, gp, tiles, stream);
@@ -498,6 +525,19 @@ cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUten
 }
 
 }  // namespace
+
+bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                             uint32_t box_cols, uint32_t box_rows) {
+  if (encode_fn() == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
                                 const void* W1, const void* W2, void* H, int* err,

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -16,11 +17,27 @@ namespace moe {
 // Upper bound on router partial-sum blocks (the launcher never exceeds it).
 int route_num_blocks(int64_t N, int E);
 
-// Router GEMV + softmax + top-k + gates. X == nullptr: `logits` is an input.
+// Router logits + softmax + top-k + gates. X == nullptr: `logits` is an input.
 // colsum_partial: [route_num_blocks][E] floats (or nullptr when prob_colsum is nullptr).
+// wt / zpart: scratch of the tensor-core logits (route_tc_*_bytes), used for bf16 X.
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          float* logits, int32_t* idx, float* gate, float* colsum_partial,
-                         float* prob_colsum, int* err, cudaStream_t stream);
+                         float* prob_colsum, __nv_bfloat16* wt, float* zpart, int* err,
+                         uint64_t timeout_ns, cudaStream_t stream);
+
+// Tensor-core router logits for bf16 X: splits W_r into three bf16 terms (wt), then writes
+// S split-K slices of partial logits zpart[S][N][Ep] (Ep = E rounded up to 8).
+bool route_tc_supported(const moe_problem& p);
+size_t route_tc_wt_bytes(const moe_problem& p);
+size_t route_tc_zpart_bytes(const moe_problem& p);
+cudaError_t launch_route_tc_logits(const moe_problem& p, const void* X, const float* W_r,
+                                   __nv_bfloat16* wt, float* zpart, int* S_out, int* Ep_out,
+                                   int* err, uint64_t timeout_ns, cudaStream_t stream);
+
+// 2-D bf16 tensor map (cols contiguous, row stride cols * 2 bytes), box box_cols x box_rows,
+// 128-byte swizzle, out-of-range elements read as zero.
+bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                             uint32_t box_cols, uint32_t box_rows);
 
 // Records are processed in chunks of this many for the slot assignment.
 constexpr int kDispatchChunk = 1024;

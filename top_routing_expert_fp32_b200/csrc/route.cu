@@ -3,15 +3,15 @@
 //   Grok-1 book ch.5, 5.2 (fp32 router, softmax, TopK) and 5.2.3 (two gate variants);
 //   MoE formula-to-code walkthrough 1.1-1.2; LLMs-from-scratch ch.12, 12.1.
 //
-// Two logit kernels, chosen by E (both fp32 FMA with fp32 accumulation):
-//   narrow (E <= 16, bound by reading X from HBM): a block owns G tokens (G*EB = 64
-//     accumulators per lane) and its 4 warps split the model dimension D, each lane reading
-//     16-byte chunks (a warp reads one contiguous 512-byte segment per token per step). W_r
-//     rows come through L1. A 5-step butterfly leaves 2 finished partial logits per lane; the
-//     4 warps' partials are added in a fixed order through shared memory.
-//   wide (E > 16, bound by fp32 FMA throughput): a block computes a 64-token x 64-expert tile
-//     as a small SGEMM over D in 32-wide slices staged through shared memory (X converted to
-//     fp32 once, stored transposed), each thread a 4x4 register tile.
+// bf16 X: the logits run on the tensor cores (route_tc.cu) and this file's selection kernel
+// finishes. fp32 X: two logit kernels, chosen by E (both fp32 FMA with fp32 accumulation):
+//   narrow (E <= 16, bound by reading X): persistent 512-thread blocks, one per SM, with W_r
+//     resident in shared memory; a warp owns G = 32/EB tokens and a slice of D, lanes stream
+//     16-byte chunks of X, a butterfly leaves one finished partial per lane, and the K slices
+//     are added in a fixed order through shared memory.
+//   wide (E > 16, bound by fp32 FMA throughput): a block computes a 128-token x 64-expert
+//     tile as a small SGEMM over D in 32-wide slices staged through shared memory, each
+//     thread an 8x8 register tile, two K halves added in a fixed order.
 // Then one thread per token does softmax + top-k + gates from shared memory. Blocks are
 // persistent over token tiles and keep a fixed-order partial sum of the softmax probabilities
 // per expert (for the balance-loss statistic); a second tiny kernel adds the partials in block
@@ -32,7 +32,9 @@ struct RouteArgs {
   const void* X;
   const float* W_r;
   const float* bias;
-  const float* logits_in;  // X == nullptr: given logits
+  const float* logits_in;  // selection kernel input: S slices [S][N][in_stride]
+  int S;                   // slices added in order (1 for given logits)
+  int in_stride;           // floats per token row of logits_in (>= E)
   float* logits_out;       // may be nullptr
   int32_t* idx;
   float* gate;
@@ -44,20 +46,9 @@ struct RouteArgs {
   int renorm;
 };
 
-// 16 bytes of X: 8 bf16 or 4 fp32 values.
+// 16 bytes of X: 4 fp32 values.
 template <typename XT>
 struct XVec;
-template <>
-struct XVec<__nv_bfloat16> {
-  static constexpr int kElems = 8;
-  __device__ static float get(const uint4& v, int j) {
-    const uint32_t w = (&v.x)[j >> 1];
-    return bf16_bits_to_float((j & 1) ? (w >> 16) : (w & 0xFFFFu));
-  }
-  __device__ static float one(const void* X, int64_t i) {
-    return bf16_bits_to_float(static_cast<const uint16_t*>(X)[i]);
-  }
-};
 template <>
 struct XVec<float> {
   static constexpr int kElems = 4;
@@ -489,16 +480,25 @@ __global__ void __launch_bounds__(kWideThreads) route_wide_kernel(RouteArgs a) {
 
 constexpr int kSelThreads = 64;
 
+// Logits of a token = sum of its S slices in slice order (+ bias): given logits (S = 1, no
+// bias) or the tensor-core router's split-K partials.
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(RouteArgs a) {
   __shared__ float s_z[kSelThreads][kMaxE + 1];
   float colsum_acc = 0.f;
   const int E = a.E;
+  const int64_t slice = a.N * a.in_stride;
   for (int64_t tile = blockIdx.x; tile * kSelThreads < a.N; tile += gridDim.x) {
     const int64_t t0 = tile * kSelThreads;
     for (int i = threadIdx.x; i < kSelThreads * E; i += kSelThreads) {
       const int tl = i / E;
       const int e = i % E;
-      if (t0 + tl < a.N) s_z[tl][e] = a.logits_in[(t0 + tl) * E + e];
+      if (t0 + tl < a.N) {
+        const float* z = a.logits_in + (t0 + tl) * a.in_stride + e;
+        float v = z[0];
+        for (int s = 1; s < a.S; ++s) v += z[s * slice];
+        if (a.bias != nullptr) v += __ldg(a.bias + e);
+        s_z[tl][e] = v;
+      }
     }
     __syncthreads();
     select_tile(a, s_z, kSelThreads, t0, colsum_acc);
@@ -589,14 +589,16 @@ int route_num_blocks(int64_t N, int E) {
 
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          float* logits, int32_t* idx, float* gate, float* colsum_partial,
-                         float* prob_colsum, int* err, cudaStream_t stream) {
-  (void)err;
+                         float* prob_colsum, __nv_bfloat16* wt, float* zpart, int* err,
+                         uint64_t timeout_ns, cudaStream_t stream) {
   if (p.N == 0) return cudaSuccess;
   RouteArgs a;
   a.X = X;
   a.W_r = W_r;
   a.bias = bias;
   a.logits_in = X == nullptr ? logits : nullptr;
+  a.S = 1;
+  a.in_stride = p.E;
   a.logits_out = X != nullptr ? logits : nullptr;
   a.idx = idx;
   a.gate = gate;
@@ -606,10 +608,22 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
   a.E = p.E;
   a.k = p.k;
   a.renorm = p.renormalize;
-  const Kind kind = kind_of(X, p.E, a.D);
-  const bool bf16 = p.dtype == MOE_DTYPE_BF16;
+  Kind kind = kind_of(X, p.E, a.D);
   int grid = 1;
   cudaError_t e = cudaSuccess;
+  if (X != nullptr && route_tc_supported(p)) {
+    // bf16 activations: logits on the tensor cores (bf16x3 split of W_r), then selection.
+    int S = 1, Ep = p.E;
+    e = launch_route_tc_logits(p, X, W_r, wt, zpart, &S, &Ep, err, timeout_ns, stream);
+    if (e != cudaSuccess) return e;
+    a.X = nullptr;
+    a.logits_in = zpart;
+    a.S = S;
+    a.in_stride = Ep;
+    kind = Kind::kSelect;
+  } else if (X == nullptr) {
+    a.bias = nullptr;  // given logits are used as they are
+  }
   if (kind == Kind::kSelect) {
     grid = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>((p.N + kSelThreads - 1) / kSelThreads, kMaxBlocks)));
@@ -621,14 +635,12 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
     const int tpb = (kNarrowWarps / ks) * (32 / EB);
     grid = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>(std::min<int64_t>((p.N + tpb - 1) / tpb, num_sms()), kMaxBlocks)));
-    e = bf16 ? launch_narrow<__nv_bfloat16>(a, EB, ks, stream)
-             : launch_narrow<float>(a, EB, ks, stream);
+    e = launch_narrow<float>(a, EB, ks, stream);  // fp32 X (bf16 X takes the tensor cores)
   } else {
     grid = static_cast<int>(
         std::max<int64_t>(1, std::min<int64_t>((p.N + kWT - 1) / kWT, kMaxBlocks)));
     const bool vecw = (p.E % 4) == 0;
-    e = bf16 ? launch_wide<__nv_bfloat16>(a, grid, vecw, stream)
-             : launch_wide<float>(a, grid, vecw, stream);
+    e = launch_wide<float>(a, grid, vecw, stream);
   }
   if (e != cudaSuccess) return e;
   if (prob_colsum != nullptr) {
