@@ -45,6 +45,12 @@ def lib():
         i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
         L.oracle_capacity.argtypes = [i64, i32, i32, f64]
         L.oracle_capacity.restype = i64
+        L.oracle_capacity_min.argtypes = [i64, i32, i32, f64, i64]
+        L.oracle_capacity_min.restype = i64
+        L.oracle_dispatch_order.argtypes = [i64, i32, i32, i64, i32, P, P, P, P, P, P]
+        L.oracle_dispatch_order.restype = None
+        L.oracle_combine_policy.argtypes = [i64, i32, i64, P, P, i32, P, P]
+        L.oracle_combine_policy.restype = None
         L.oracle_router_logits.argtypes = [i64, i64, i32, P, i32, P, P, P, P]
         L.oracle_router_logits.restype = None
         L.oracle_route.argtypes = [i64, i32, i32, i32, P, P, P, P, P]
@@ -61,8 +67,8 @@ def lib():
         L.oracle_balance_loss.restype = f64
         L.oracle_drop_rate.argtypes = [i64, i32, P]
         L.oracle_drop_rate.restype = f64
-        L.oracle_forward.argtypes = [i64, i64, i64, i32, i32, f64, i32, i32, i32,
-                                     P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.oracle_forward.argtypes = [i64, i64, i64, i32, i32, f64, i64, i32, i32, i32, i32,
+                                     i32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.oracle_forward.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
@@ -96,8 +102,14 @@ def num_threads() -> int:
     return int(lib().oracle_num_threads())
 
 
-def capacity(N: int, k: int, E: int, cf: float) -> int:
-    return int(lib().oracle_capacity(N, k, E, float(cf)))
+# Capacity policies: slot order of the position assignment, and what a token's kept slots
+# weigh when another of its slots was dropped.
+SLOT_MAJOR, TOKEN_MAJOR = 0, 1
+DROP_ZERO, DROP_RENORM_KEPT = 0, 1
+
+
+def capacity(N: int, k: int, E: int, cf: float, min_capacity: int = 0) -> int:
+    return int(lib().oracle_capacity_min(N, k, E, float(cf), int(min_capacity)))
 
 
 def router_logits(X: np.ndarray, x_dtype: int, W_r: np.ndarray, bias=None):
@@ -136,8 +148,9 @@ def topk_margin(logits64: np.ndarray, k: int) -> np.ndarray:
     return m
 
 
-def dispatch(idx: np.ndarray, E: int, C: int):
-    """Slot-major capacity dispatch. Returns dict(load, offsets, pos, dropped, row_token)."""
+def dispatch(idx: np.ndarray, E: int, C: int, order: int = SLOT_MAJOR):
+    """Capacity dispatch (slot-major or token-major). Returns dict(load, offsets, pos, dropped,
+    row_token)."""
     idx = _c(idx, np.int32)
     N, k = idx.shape
     load = np.empty((E,), np.int32)
@@ -145,8 +158,8 @@ def dispatch(idx: np.ndarray, E: int, C: int):
     pos = np.empty((N, k), np.int32)
     dropped = np.empty((N, k), np.uint8)
     row_token = np.full((N * k,), -1, np.int32)
-    lib().oracle_dispatch(N, k, E, C, _p(idx), _p(load), _p(offsets), _p(pos), _p(dropped),
-                          _p(row_token))
+    lib().oracle_dispatch_order(N, k, E, C, order, _p(idx), _p(load), _p(offsets), _p(pos),
+                                _p(dropped), _p(row_token))
     return dict(load=load, offsets=offsets, pos=pos, dropped=dropped,
                 row_token=row_token[: int(offsets[E])].copy())
 
@@ -165,14 +178,15 @@ def expert_ffn(rec_token, rec_expert, X, W1, W2, W3, dtype: int, act: int) -> np
     return Y
 
 
-def combine(gate, dropped, Yrec) -> np.ndarray:
+def combine(gate, dropped, Yrec, policy: int = DROP_ZERO) -> np.ndarray:
     gate = _c(gate, np.float64)
     N, k = gate.shape
     Yrec = _c(Yrec, np.float64)
     D = Yrec.shape[-1]
     dr = None if dropped is None else _c(dropped, np.uint8)
     out = np.empty((N, D), np.float64)
-    lib().oracle_combine(N, k, D, _p(gate), _p(dr), _p(Yrec.reshape(N * k, D)), _p(out))
+    lib().oracle_combine_policy(N, k, D, _p(gate), _p(dr), policy, _p(Yrec.reshape(N * k, D)),
+                                _p(out))
     return out
 
 
@@ -190,7 +204,8 @@ def drop_rate(dropped) -> float:
 
 
 def forward(X, W_r, bias, W1, W2, W3, *, k: int, cf: float, renorm: int, act: int,
-            dtype: int):
+            dtype: int, min_capacity: int = 0, order: int = SLOT_MAJOR,
+            drop_policy: int = DROP_ZERO):
     """Whole layer in fp64. Returns dict(out [N,D] f64, logits32, idx, gate, load, offsets,
     pos, dropped, colsum)."""
     X, W1, W2, W3 = (_elems(a, dtype) for a in (X, W1, W2, W3))
@@ -208,7 +223,8 @@ def forward(X, W_r, bias, W1, W2, W3, *, k: int, cf: float, renorm: int, act: in
     pos = np.empty((N, k), np.int32)
     dropped = np.empty((N, k), np.uint8)
     colsum = np.empty((E,), np.float64)
-    rc = lib().oracle_forward(N, D, F, E, k, float(cf), renorm, act, dtype, _p(X), _p(W_r),
+    rc = lib().oracle_forward(N, D, F, E, k, float(cf), int(min_capacity), order, drop_policy,
+                              renorm, act, dtype, _p(X), _p(W_r),
                               _p(b), _p(W1), _p(W2), _p(W3), _p(out), _p(l32), _p(idx),
                               _p(gate), _p(load), _p(offsets), _p(pos), _p(dropped),
                               _p(colsum))

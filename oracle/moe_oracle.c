@@ -21,9 +21,14 @@
  * Readings where the pages are silent (each listed in the design notes):
  *   - top-k ties: lower expert index first; selection is made on the fp32 logits (softmax is
  *     strictly increasing, so the set equals the set selected on probabilities);
- *   - capacity slots are assigned slot-major: every rank-0 record in token order, then every
- *     rank-1 record, ... (the walkthrough's loop with its two loops swapped);
- *   - a dropped record contributes zero; the other slot keeps its gate unchanged;
+ *   - capacity slots are assigned slot-major by default: every rank-0 record in token order,
+ *     then every rank-1 record, ... (the walkthrough's loop with its two loops swapped);
+ *     token-major order (the walkthrough's own loop, [W] 3.2) is the other policy;
+ *   - a dropped record contributes zero; by default the other slots keep their gates
+ *     unchanged; the other policy ([GS] 2.2 case A, (w1, w2) -> (1, 0) when one of the two
+ *     experts overflows) renormalises the gates of a token's kept slots to sum 1 whenever at
+ *     least one slot was dropped and one was kept;
+ *   - capacity = max(ceil(CF*N*K/E), min_capacity) ([GS] 2.1), min_capacity = 0 by default;
  *   - balance loss f_i = load_i / (N*k), P_i = mean full-softmax probability.
  *
  * Every floating-point step accumulates in double in the order the definition states.
@@ -75,6 +80,14 @@ static int all_finite_f32(const float* v, int64_t n) {
 int64_t oracle_capacity(int64_t N, int32_t k, int32_t E, double cf) {
   if (cf <= 0.0) return N * (int64_t)k;
   return (int64_t)ceil(cf * (double)N * (double)k / (double)E);
+}
+
+/* GShard's form ([GS] 2.1): capacity = max(S/E * K * capacity_factor, min_capacity), the first
+ * term rounded up as above. With CF <= 0 there is no capacity and min_capacity is unused. */
+int64_t oracle_capacity_min(int64_t N, int32_t k, int32_t E, double cf, int64_t min_capacity) {
+  const int64_t c = oracle_capacity(N, k, E, cf);
+  if (cf <= 0.0) return c;
+  return c > min_capacity ? c : min_capacity;
 }
 
 /* ---------------------------------------------------------------- router  [G5] 5.2 */
@@ -207,17 +220,30 @@ void oracle_topk_margin(int64_t N, int32_t E, int32_t k, const double* logits64,
  * load[e]    = number of records routed to e (before capacity)      ([W] 1.3)
  * offsets    = exclusive prefix sum of kept_e = min(load_e, C); offsets[E] = kept records
  * row_token[offsets[e] + pos] = t for every kept record (expert-contiguous order). */
-void oracle_dispatch(int64_t N, int32_t k, int32_t E, int64_t C, const int32_t* idx,
-                     int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
-                     int32_t* row_token) {
+/* One routing record (t, j): its position is the number of records routed to the same expert
+ * before it in the visiting order; it is dropped when that position reaches C. */
+static void visit_record(int64_t t, int32_t j, int32_t k, int64_t C, const int32_t* idx,
+                         int64_t* count, int32_t* pos, uint8_t* dropped) {
+  int32_t e = idx[t * k + j];
+  int64_t p = count[e]++;
+  pos[t * k + j] = (int32_t)p;
+  dropped[t * k + j] = (uint8_t)(p >= C);
+}
+
+/* order 0 (slot-major): all rank-0 records in token order, then rank 1, ...
+ * order 1 (token-major, the walkthrough's loop [W] 3.2): token by token, its slots in rank
+ * order. */
+void oracle_dispatch_order(int64_t N, int32_t k, int32_t E, int64_t C, int32_t order,
+                           const int32_t* idx, int32_t* load, int32_t* offsets, int32_t* pos,
+                           uint8_t* dropped, int32_t* row_token) {
   int64_t* count = (int64_t*)calloc((size_t)E, sizeof(int64_t));
-  for (int32_t j = 0; j < k; ++j)
-    for (int64_t t = 0; t < N; ++t) {
-      int32_t e = idx[t * k + j];
-      int64_t p = count[e]++;
-      pos[t * k + j] = (int32_t)p;
-      dropped[t * k + j] = (uint8_t)(p >= C);
-    }
+  if (order == 1) {
+    for (int64_t t = 0; t < N; ++t)
+      for (int32_t j = 0; j < k; ++j) visit_record(t, j, k, C, idx, count, pos, dropped);
+  } else {
+    for (int32_t j = 0; j < k; ++j)
+      for (int64_t t = 0; t < N; ++t) visit_record(t, j, k, C, idx, count, pos, dropped);
+  }
   offsets[0] = 0;
   for (int32_t e = 0; e < E; ++e) {
     load[e] = (int32_t)count[e];
@@ -229,6 +255,12 @@ void oracle_dispatch(int64_t N, int32_t k, int32_t E, int64_t C, const int32_t* 
       for (int32_t j = 0; j < k; ++j)
         if (!dropped[t * k + j]) row_token[offsets[idx[t * k + j]] + pos[t * k + j]] = (int32_t)t;
   free(count);
+}
+
+void oracle_dispatch(int64_t N, int32_t k, int32_t E, int64_t C, const int32_t* idx,
+                     int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                     int32_t* row_token) {
+  oracle_dispatch_order(N, k, E, C, 0, idx, load, offsets, pos, dropped, row_token);
 }
 
 /* ---------------------------------------------------------------- expert FFN  [L12] 12.1 */
@@ -291,20 +323,37 @@ void oracle_expert_ffn(int64_t n_rec, const int32_t* rec_token, const int32_t* r
 /* out[t] = sum_{j=0}^{k-1} [not dropped(t,j)] * gate[t,j] * y(t,j)   (j ascending; a token
  * accumulates its k contributions, [L12] 12.2; a dropped slot adds nothing, [GS] 2.2).
  * Yrec holds one row per record in record order (t*k + j). */
-void oracle_combine(int64_t N, int32_t k, int64_t D, const double* gate,
-                    const uint8_t* dropped, const double* Yrec, double* out) {
+/* out[t] = sum over kept slots j of g'[t,j] * Y[t,j]. policy 0: g' = g. policy 1 ([GS] 2.2
+ * case A): when a token has both dropped and kept slots, g'[t,j] = g[t,j] / (sum of the kept
+ * slots' gates), so that the kept gates sum to 1 ((w1, w2) -> (1, 0) for top-2). */
+void oracle_combine_policy(int64_t N, int32_t k, int64_t D, const double* gate,
+                           const uint8_t* dropped, int32_t policy, const double* Yrec,
+                           double* out) {
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < N; ++t) {
     double* o = out + t * D;
     for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    double kept_sum = 0.0;
+    int32_t kept = 0;
+    for (int32_t j = 0; j < k; ++j)
+      if (!(dropped && dropped[t * k + j])) {
+        kept_sum += gate[t * k + j];
+        ++kept;
+      }
+    const int reweight = policy == 1 && kept > 0 && kept < k;
     for (int32_t j = 0; j < k; ++j) {
       const int64_t r = t * k + j;
       if (dropped && dropped[r]) continue;
-      const double g = gate[r];
+      const double g = reweight ? gate[r] / kept_sum : gate[r];
       const double* y = Yrec + r * D;
       for (int64_t d = 0; d < D; ++d) o[d] += g * y[d];
     }
   }
+}
+
+void oracle_combine(int64_t N, int32_t k, int64_t D, const double* gate,
+                    const uint8_t* dropped, const double* Yrec, double* out) {
+  oracle_combine_policy(N, k, D, gate, dropped, 0, Yrec, out);
 }
 
 /* ---------------------------------------------------------------- diagnostics  [W] 2, 3.3 */
@@ -331,10 +380,12 @@ double oracle_drop_rate(int64_t N, int32_t k, const uint8_t* dropped) {
 /* ---------------------------------------------------------------- whole layer */
 
 /* The full forward in the pages' order: logits -> softmax -> top-k (+renorm) -> load ->
- * capacity -> slot-major dispatch -> gated expert FFN per kept record -> gate-weighted
- * combine. out [N,D] doubles (before any rounding to the output dtype). Every other output
- * pointer is optional. Returns 0, or -1 on a non-finite logit. */
+ * capacity (with min_capacity) -> dispatch in the given order -> gated expert FFN per kept
+ * record -> gate-weighted combine under the drop policy. out [N,D] doubles (before any
+ * rounding to the output dtype). Every other output pointer is optional. Returns 0, or -1 on
+ * a non-finite logit. */
 int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double cf,
+                   int64_t min_capacity, int32_t order, int32_t drop_policy,
                    int32_t renorm, int32_t act, int32_t dtype, const void* X, const float* W_r,
                    const float* bias, const void* W1, const void* W2, const void* W3,
                    double* out, float* logits32_out, int32_t* idx_out, double* gate_out,
@@ -354,8 +405,8 @@ int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double
   if (oracle_route(N, E, k, renorm, l32, idx, gate, NULL, prob_colsum_out) != 0) {
     rc = -1;
   } else {
-    const int64_t C = oracle_capacity(N, k, E, cf);
-    oracle_dispatch(N, k, E, C, idx, load, offs, pos, drp, NULL);
+    const int64_t C = oracle_capacity_min(N, k, E, cf, min_capacity);
+    oracle_dispatch_order(N, k, E, C, order, idx, load, offs, pos, drp, NULL);
     /* expert outputs of the kept records, one row per record (dropped rows stay zero) */
     int64_t nk = 0;
     for (int64_t r = 0; r < R; ++r) nk += drp[r] ? 0 : 1;
@@ -377,7 +428,7 @@ int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double
       memcpy(Yrec + r * D, Yk + q * D, sizeof(double) * (size_t)D);
       ++q;
     }
-    oracle_combine(N, k, D, gate, drp, Yrec, out);
+    oracle_combine_policy(N, k, D, gate, drp, drop_policy, Yrec, out);
     free(rt);
     free(re);
     free(Yk);
