@@ -201,7 +201,9 @@ def oracle_tokens_per_s(cfg, budget_s: float = 12.0):
     def run(n):
         t = time.perf_counter()
         oracle.forward(X[:n], Wr, b, W1, W2, W3, k=cfg.k, cf=cfg.capacity_factor,
-                       renorm=cfg.renormalize, act=cfg.activation, dtype=od)
+                       renorm=cfg.renormalize, act=cfg.activation, dtype=od,
+                       min_capacity=cfg.min_capacity, order=cfg.capacity_order,
+                       drop_policy=cfg.drop_policy)
         return time.perf_counter() - t
 
     n = min(cfg.N, max(1, oracle.num_threads()))

@@ -3,9 +3,10 @@
  *
  * The layer (one data-parallel hot path, single GPU):
  *   logits = X W_r (+bias) in fp32 -> softmax over E -> top-k -> gates (optionally
- *   renormalised over the selected set) -> per-expert load -> capacity ceil(CF*N*k/E) with a
- *   slot-major drop mask -> expert-contiguous permutation of the N*k records -> per-expert
- *   gated FFN [act(x W1_e) (.) (x W2_e)] W3_e -> gate-weighted sum back to the N tokens.
+ *   renormalised over the selected set) -> per-expert load -> capacity
+ *   max(ceil(CF*N*k/E), min_capacity) with a slot-major or token-major drop mask ->
+ *   expert-contiguous permutation of the N*k records -> per-expert gated FFN
+ *   [act(x W1_e) (.) (x W2_e)] W3_e -> gate-weighted sum back to the N tokens.
  *
  * Sources, cited by page title and section:
  *   - Grok-1 book ch.5 "MoE routing & experts": 5.2 (fp32 router x.W_r, softmax, TopK),
@@ -17,7 +18,8 @@
  *   - MoE formula-to-code walkthrough: 1.1 (stable softmax), 1.2 (top-k ordered by
  *     descending score, renormalisation), 1.3 (expert load), 2.1 (balance loss), 3.1
  *     (capacity), 3.2 (dispatch with a dropped mask), 3.3 (drop rate).
- *   - MoE series (GShard/Mixtral/Switch): 2.2 (an overflowed slot contributes nothing).
+ *   - MoE series (GShard/Mixtral/Switch): 2.1 (capacity with min_capacity), 2.2 (an
+ *     overflowed slot contributes nothing; case A: the kept expert takes the whole weight).
  *
  * Conventions shared by every entry point:
  *   - Array pointers are DEVICE pointers unless the entry point says otherwise. The caller
@@ -68,6 +70,10 @@ typedef enum {
 
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_ERF = 1, MOE_ACT_GELU_TANH = 2 };
+/* Order in which routing records take capacity positions (walkthrough 3.2; MoE series 2.2). */
+enum { MOE_ORDER_SLOT_MAJOR = 0, MOE_ORDER_TOKEN_MAJOR = 1 };
+/* Weights of a token's kept slots when another of its slots was dropped (MoE series 2.2). */
+enum { MOE_DROP_ZERO = 0, MOE_DROP_RENORM_KEPT = 1 };
 
 /* Device error codes written to the workspace error word. */
 enum {
@@ -86,6 +92,15 @@ enum {
  *                   selected k (Mixtral / walkthrough 1.2)
  *   activation      MOE_ACT_* applied to x W1 (SiLU, exact-erf GELU, tanh GELU)
  *   dtype           MOE_DTYPE_* of X, W1..W3 and every activation buffer
+ *   capacity_order  MOE_ORDER_SLOT_MAJOR: all rank-0 records in token order take positions
+ *                   first, then rank 1, ... (every token's first choice has priority);
+ *                   MOE_ORDER_TOKEN_MAJOR: token by token, each token's slots in rank order
+ *                   (the walkthrough's dispatch loop, 3.2)
+ *   drop_policy     MOE_DROP_ZERO: a dropped slot contributes nothing and the kept slots keep
+ *                   their gates; MOE_DROP_RENORM_KEPT: when a token has dropped and kept
+ *                   slots, the kept gates are divided by their sum (GShard case A, MoE series
+ *                   2.2: (w1, w2) -> (1, 0) when the second expert overflows)
+ *   min_capacity    >= 0; the capacity is max(ceil(CF*N*k/E), min_capacity) (MoE series 2.1)
  * bf16 problems need D and F to be multiples of 8 (16-byte rows for the tensor-memory
  * copies); fp32 problems need D and F to be multiples of 4. */
 typedef struct {
@@ -98,11 +113,14 @@ typedef struct {
   int32_t renormalize;
   int32_t activation;
   int32_t dtype;
+  int32_t capacity_order;
+  int32_t drop_policy;
   int32_t reserved; /* must be 0 */
+  int64_t min_capacity;
 } moe_problem;
 
-/* Host only. C = ceil(CF * N * k / E) evaluated in double left to right (walkthrough 3.1);
- * C = N*k when CF <= 0. */
+/* Host only. C = max(ceil(CF * N * k / E), min_capacity), the first term evaluated in double
+ * left to right (walkthrough 3.1; MoE series 2.1); C = N*k when CF <= 0. */
 moe_status moe_capacity(const moe_problem* p, int64_t* C);
 
 /* Host only. Bytes of workspace every entry point below accepts for problem p (one size for
@@ -132,8 +150,9 @@ moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, cons
 /* Load histogram, capacity, slot assignment and permutation (walkthrough 1.3, 3.1, 3.2;
  * LLMs-from-scratch 12.2; MoE series 2.2).
  *   load[e]      = number of records (t,j) with topk_idx[t,j] == e (before capacity).
- *   pos[t,j]     = rank of record (t,j) among expert e's records, records taken slot-major
- *                  (all j=0 records in token order, then all j=1 records, ...).
+ *   pos[t,j]     = rank of record (t,j) among expert e's records, records taken in
+ *                  p->capacity_order: slot-major (all j=0 records in token order, then all
+ *                  j=1 records, ...) or token-major (t ascending, j ascending within t).
  *   dropped[t,j] = pos[t,j] >= C.
  *   offsets      = exclusive prefix sum of min(load_e, C); offsets[E] = kept records.
  *   row_token[offsets[e] + pos[t,j]] = t for every kept record; entries past offsets[E]
@@ -191,9 +210,11 @@ moe_status moe_expert_down(const moe_problem* p, const void* H, const int32_t* o
                            const void* W3, void* Y, void* ws, size_t ws_bytes, void* stream);
 
 /* Gate-weighted combine (Grok-1 book 5.3.5; LLMs-from-scratch 12.2; MoE series 2.2):
- *   out[t] = sum_{j=0..k-1} [!dropped[t,j]] * topk_gate[t,j] * Y[offsets[topk_idx[t,j]] + pos[t,j]]
- * accumulated in fp32 in ascending j, rounded once to the output dtype; a token whose
- * slots are all dropped gets 0. `dropped` may be NULL (nothing dropped). No atomics. */
+ *   out[t] = sum_{j=0..k-1} [!dropped[t,j]] * g[t,j] * Y[offsets[topk_idx[t,j]] + pos[t,j]]
+ * with g = topk_gate, except under MOE_DROP_RENORM_KEPT for a token with both dropped and kept
+ * slots: g[t,j] = topk_gate[t,j] / (sum of its kept slots' gates, fp32, ascending j).
+ * Accumulated in fp32 in ascending j, rounded once to the output dtype; a token whose slots
+ * are all dropped gets 0. `dropped` may be NULL (nothing dropped). No atomics. */
 moe_status moe_combine(const moe_problem* p, const void* Y, const int32_t* topk_idx,
                        const float* topk_gate, const int32_t* offsets, const int32_t* pos,
                        const uint8_t* dropped, void* out, void* stream);

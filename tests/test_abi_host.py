@@ -45,7 +45,7 @@ def test_library_built_for_sm100a(abi):
 
 
 def test_version_and_status_strings(abi):
-    assert abi.lib.moe_version() >= 100
+    assert abi.lib.moe_version() >= 110
     assert abi.lib.moe_status_string(0) == b"ok"
     assert abi.lib.moe_status_string(3) == b"CUDA error"
 
@@ -58,6 +58,32 @@ def test_capacity_matches_oracle(abi, oracle_lib, N, k, E, cf):
     cfg = configs.MoEConfig("c", N=N, D=64, F=64, E=E, k=k, dtype=configs.DTYPE_BF16,
                             activation=0, renormalize=1, capacity_factor=cf)
     assert abi.capacity(abi.problem(cfg)) == oracle_lib.capacity(N, k, E, cf)
+
+
+@pytest.mark.parametrize("N,k,E,cf,minc", [(8, 2, 4, 0.5, 3), (8, 2, 4, 1.0, 3), (16384, 2, 64, 1.0, 256),
+                                           (100, 2, 8, 0.0, 1000), (5, 2, 3, 0.3, 2)])
+def test_capacity_with_floor_matches_oracle(abi, oracle_lib, N, k, E, cf, minc):
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("c", N=N, D=64, F=64, E=E, k=k, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1, capacity_factor=cf, min_capacity=minc)
+    assert abi.capacity(abi.problem(cfg)) == oracle_lib.capacity(N, k, E, cf, minc)
+
+
+def test_problem_struct_matches_header_layout(abi, tmp_path):
+    # The ctypes mirror must have the C header's size and field offsets (gcc, host only).
+    import subprocess
+    fields = [f for f, _ in abi.moe_problem._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "moe.h"\nint main(void) {\n'
+                   '  printf("%zu", sizeof(moe_problem));\n' +
+                   "".join(f'  printf(" %zu", offsetof(moe_problem, {f}));\n' for f in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
+    assert got[0] == ctypes.sizeof(abi.moe_problem)
+    assert got[1:] == [getattr(abi.moe_problem, f).offset for f in fields]
 
 
 def test_workspace_size_covers_intermediates(abi):
@@ -80,7 +106,8 @@ def _call_route(abi, p, ws=None, ws_bytes=0, X=None, W_r=None, logits=None, idx=
 @pytest.mark.parametrize("field,value,status", [
     ("k", 0, 1), ("k", 9, 1), ("E", 65, 2), ("N", -1, 1), ("D", 0, 1), ("dtype", 7, 1),
     ("activation", 3, 1), ("renormalize", 2, 1), ("reserved", 1, 1), ("D", 12, 2),
-    ("capacity_factor", float("nan"), 1)])
+    ("capacity_factor", float("nan"), 1), ("capacity_order", 2, 1), ("drop_policy", -1, 1),
+    ("min_capacity", -5, 1)])
 def test_invalid_problems_rejected_on_host(abi, field, value, status):
     from top_routing_expert_fp32_b200 import configs
     cfg = configs.MoEConfig("c", N=64, D=64, F=64, E=8, k=2, dtype=configs.DTYPE_BF16,

@@ -49,8 +49,8 @@ def check_layer(cfg, inp, out, ex, sample=None):
     margin = oracle.topk_margin(l64, cfg.k)
     flips = (ex["idx"] != ro["idx"]).any(1)
     assert (margin[flips] < NEAR_TIE).all(), "routing differs on a token that is not near-tied"
-    C = oracle.capacity(cfg.N, cfg.k, cfg.E, cfg.capacity_factor)
-    do = oracle.dispatch(ro["idx"], cfg.E, C)
+    C = oracle.capacity(cfg.N, cfg.k, cfg.E, cfg.capacity_factor, cfg.min_capacity)
+    do = oracle.dispatch(ro["idx"], cfg.E, C, order=cfg.capacity_order)
     if not flips.any():
         for key in ("load", "offsets", "pos", "dropped"):
             assert np.array_equal(ex[key], do[key]), key
@@ -72,8 +72,15 @@ def check_layer(cfg, inp, out, ex, sample=None):
                           np_host(inp.W1), np_host(inp.W2), np_host(inp.W3), od, cfg.activation)
     ref = np.zeros((len(toks), cfg.D))
     row_of = {t: i for i, t in enumerate(toks)}
+    # Gates as the combine applies them (MoE series 2.2 case A under DROP_RENORM_KEPT).
+    g_eff = ro["gate"].copy()
+    if cfg.drop_policy == configs.DROP_RENORM_KEPT:
+        kept = do["dropped"] == 0
+        partial = kept.any(1) & ~kept.all(1)
+        ksum = (ro["gate"] * kept).sum(1)
+        g_eff[partial] = ro["gate"][partial] / ksum[partial, None]
     for (t, j), y in zip(slot, Y):
-        ref[row_of[t]] += ro["gate"][t, j] * y
+        ref[row_of[t]] += g_eff[t, j] * y
     got = to_f64(out)[toks]
     err = normwise_rel_err(got, ref)
     assert err.max() <= tol(cfg), f"max normwise rel err {err.max():.3g} > {tol(cfg)}"
@@ -97,6 +104,24 @@ SMALL = [
                       capacity_factor=0.8, router_bias_var=2.0),
     configs.MoEConfig("small_f32_gelu_tanh", N=96, D=64, F=96, E=5, k=3, dtype=configs.DTYPE_F32,
                       activation=configs.ACT_GELU_TANH, renormalize=0, capacity_factor=0.9),
+    # capacity policies: token-major positions, GShard case-A reweight, min_capacity floor
+    configs.MoEConfig("small_token_major", N=500, D=128, F=256, E=16, k=2,
+                      dtype=configs.DTYPE_BF16, activation=configs.ACT_SILU, renormalize=1,
+                      capacity_factor=1.0, router_bias_var=2.0,
+                      capacity_order=configs.ORDER_TOKEN_MAJOR),
+    configs.MoEConfig("small_gshard", N=500, D=128, F=256, E=16, k=2,
+                      dtype=configs.DTYPE_BF16, activation=configs.ACT_SILU, renormalize=1,
+                      capacity_factor=0.5, router_bias_var=2.0,
+                      capacity_order=configs.ORDER_TOKEN_MAJOR,
+                      drop_policy=configs.DROP_RENORM_KEPT, min_capacity=40),
+    configs.MoEConfig("small_case_a_k3_norenorm", N=300, D=128, F=192, E=8, k=3,
+                      dtype=configs.DTYPE_BF16, activation=configs.ACT_GELU_ERF, renormalize=0,
+                      capacity_factor=0.6, router_bias_var=1.0,
+                      drop_policy=configs.DROP_RENORM_KEPT),
+    configs.MoEConfig("small_f32_token_major_case_a", N=96, D=64, F=96, E=5, k=3,
+                      dtype=configs.DTYPE_F32, activation=configs.ACT_SILU, renormalize=1,
+                      capacity_factor=0.7, capacity_order=configs.ORDER_TOKEN_MAJOR,
+                      drop_policy=configs.DROP_RENORM_KEPT),
 ]
 
 
@@ -138,7 +163,7 @@ def _sample(cfg, n=12):
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "decode", "mixtral", "capacity", "capacity_k1",
-                                  "grok1"])
+                                  "capacity_gshard", "grok1"])
 def test_forward_named_workload_full_size(abi, name):
     cfg = configs.CONFIGS[name]
     inp = inputs.make_inputs(cfg, "cuda")

@@ -21,9 +21,12 @@ def abi():
     return a
 
 
-def _cfg(N, D, F, E, k, dtype=configs.DTYPE_BF16, act=0, renorm=1, cf=0.0, bias_var=0.0):
+def _cfg(N, D, F, E, k, dtype=configs.DTYPE_BF16, act=0, renorm=1, cf=0.0, bias_var=0.0,
+         order=configs.ORDER_SLOT_MAJOR, drop_policy=configs.DROP_ZERO, min_capacity=0):
     return configs.MoEConfig("t", N=N, D=D, F=F, E=E, k=k, dtype=dtype, activation=act,
-                             renormalize=renorm, capacity_factor=cf, router_bias_var=bias_var)
+                             renormalize=renorm, capacity_factor=cf, router_bias_var=bias_var,
+                             capacity_order=order, drop_policy=drop_policy,
+                             min_capacity=min_capacity)
 
 
 # ------------------------------------------------------------------ routing from given logits
@@ -88,7 +91,8 @@ def test_route_from_x(abi, oracle_lib, dtype, N, D, E, k, renorm, bias_var):
 
 # ------------------------------------------------------------------ dispatch (bit-exact)
 
-def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, X=None):
+def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, X=None,
+                   order=configs.ORDER_SLOT_MAJOR, min_capacity=0):
     l32 = inputs.make_logits(N, E, seed=seed).numpy()
     if skew:
         l32 = l32 + (np.arange(E, dtype=np.float32)[::-1] * skew)
@@ -96,7 +100,8 @@ def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, 
     if all_one:
         idx = np.tile(np.arange(k, dtype=np.int32), (N, 1))
     dtype = configs.DTYPE_F32 if (X is not None and X.dtype == torch.float32) else configs.DTYPE_BF16
-    cfg = _cfg(N, X.shape[1] if X is not None else 64, 64, E, k, dtype=dtype, cf=cf)
+    cfg = _cfg(N, X.shape[1] if X is not None else 64, 64, E, k, dtype=dtype, cf=cf,
+               order=order, min_capacity=min_capacity)
     p = abi.problem(cfg)
     ws = abi.workspace(p)
     d = alloc_dispatch_out(N, E, k)
@@ -108,8 +113,8 @@ def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, 
                  X_perm, ws)
     torch.cuda.synchronize()
     C = abi.capacity(p)
-    assert C == oracle_lib.capacity(N, k, E, cf)
-    ref = oracle_lib.dispatch(idx, E, C)
+    assert C == oracle_lib.capacity(N, k, E, cf, min_capacity)
+    ref = oracle_lib.dispatch(idx, E, C, order=order)
     assert np.array_equal(d["load"].cpu().numpy(), ref["load"])
     assert np.array_equal(d["offsets"].cpu().numpy(), ref["offsets"])
     assert np.array_equal(d["pos"].cpu().numpy(), ref["pos"])
@@ -127,6 +132,22 @@ def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, 
     (1025, 2, 1, 0.5, 0)])
 def test_dispatch_bitexact(abi, oracle_lib, N, E, k, cf, skew):
     _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=N + E + k, skew=skew)
+
+
+@pytest.mark.parametrize("N,E,k,cf,skew,minc", [
+    (5, 3, 2, 0.3, 0, 0), (1000, 8, 2, 1.0, 0.5, 0), (5000, 8, 2, 1.25, 0.3, 700),
+    (16384, 64, 2, 1.0, 0.05, 256), (3001, 13, 3, 0.7, 0.2, 0), (2049, 64, 8, 1.0, 0.0, 40),
+    (1025, 2, 1, 0.5, 0, 0), (700, 16, 4, 0.25, 0.1, 1000)])
+def test_dispatch_token_major_bitexact(abi, oracle_lib, N, E, k, cf, skew, minc):
+    # The walkthrough's dispatch loop order (3.2), with GShard's min_capacity floor (2.1).
+    _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=N + E + k + 1, skew=skew,
+                   order=configs.ORDER_TOKEN_MAJOR, min_capacity=minc)
+
+
+def test_dispatch_min_capacity_slot_major(abi, oracle_lib):
+    d, ref, _ = _dispatch_case(abi, oracle_lib, 3000, 8, 2, 0.25, seed=5, skew=0.2,
+                               min_capacity=500)
+    assert ref["offsets"][-1] <= 8 * 500 and ref["dropped"].any()
 
 
 def test_dispatch_all_records_to_one_expert_set(abi, oracle_lib):
@@ -279,3 +300,33 @@ def test_combine(abi, oracle_lib, N, D, E, k, cf, dtype):
     assert err.max() <= (8e-3 if dtype == configs.DTYPE_BF16 else 1e-6)
     allgone = ref["dropped"].all(1)
     assert (to_f64(out)[allgone] == 0).all()
+
+
+@pytest.mark.parametrize("N,D,E,k,cf,dtype", [
+    (500, 2048, 64, 2, 1.0, configs.DTYPE_BF16), (300, 72, 5, 3, 0.4, configs.DTYPE_BF16),
+    (257, 1024, 8, 4, 0.5, configs.DTYPE_F32), (1000, 4096, 8, 2, 0.6, configs.DTYPE_BF16)])
+def test_combine_case_a_reweight(abi, oracle_lib, N, D, E, k, cf, dtype):
+    # MoE series 2.2 case A: a token that lost some slots gives the whole weight to the kept ones.
+    tdt = inputs.torch_dtype(dtype)
+    d, ref, _ = _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=13, skew=0.2)
+    partial = ref["dropped"].any(1) & ~ref["dropped"].all(1)
+    assert partial.any()
+    R = N * k
+    Y = inputs.randn((R, D), 1.0, tdt, "cuda", 14, 1)
+    rng = np.random.default_rng(5)
+    gate = torch.from_numpy(rng.random((N, k)).astype(np.float32)).cuda()
+    idx = oracle_lib.route(inputs.make_logits(N, E, seed=13).numpy() +
+                           (np.arange(E, dtype=np.float32)[::-1] * 0.2), k=k, renorm=1)["idx"]
+    cfg = _cfg(N, D, 64, E, k, dtype=dtype, cf=cf, drop_policy=configs.DROP_RENORM_KEPT)
+    p = abi.problem(cfg)
+    out = torch.empty((N, D), dtype=tdt, device="cuda")
+    abi.combine(p, Y, torch.from_numpy(idx).cuda(), gate, d["offsets"], d["pos"], d["dropped"],
+                out)
+    torch.cuda.synchronize()
+    rows = ref["offsets"][idx] + ref["pos"]
+    Yrec = to_f64(Y)[np.where(ref["dropped"] == 1, 0, rows)]
+    oref = oracle_lib.combine(gate.cpu().double().numpy(), ref["dropped"], Yrec,
+                              policy=oracle_lib.DROP_RENORM_KEPT)
+    err = normwise_rel_err(to_f64(out), oref)
+    assert err.max() <= (8e-3 if dtype == configs.DTYPE_BF16 else 1e-6)
+    assert (to_f64(out)[ref["dropped"].all(1)] == 0).all()

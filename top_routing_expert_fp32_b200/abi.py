@@ -33,7 +33,8 @@ class moe_problem(ctypes.Structure):
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("renormalize", ctypes.c_int32),
                 ("activation", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("capacity_order", ctypes.c_int32), ("drop_policy", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("min_capacity", ctypes.c_int64)]
 
 
 class MoEError(RuntimeError):
@@ -89,7 +90,9 @@ def _check(status: int):
 def problem(cfg: MoEConfig, N: Optional[int] = None) -> moe_problem:
     return moe_problem(N=cfg.N if N is None else N, D=cfg.D, F=cfg.F, E=cfg.E, k=cfg.k,
                        capacity_factor=float(cfg.capacity_factor), renormalize=cfg.renormalize,
-                       activation=cfg.activation, dtype=cfg.dtype, reserved=0)
+                       activation=cfg.activation, dtype=cfg.dtype,
+                       capacity_order=cfg.capacity_order, drop_policy=cfg.drop_policy,
+                       reserved=0, min_capacity=cfg.min_capacity)
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -15,6 +15,10 @@ described on the pages:
   (MoE formula-to-code walkthrough, section 3).
 * ``decode``     -- decode-sized, expert-weight-bandwidth-bound: N=64, D=4096, F=14336, E=8,
   top-2, SiLU gating, renormalised.
+* ``capacity_gshard`` -- the capacity shape under GShard's policies: token-major positions
+  (the walkthrough's dispatch loop, 3.2), the kept slot of a half-dropped token takes the
+  whole weight (MoE series 2.2, case A), capacity = max(ceil(CF*N*k/E), min_capacity) with
+  CF = 1.0 and min_capacity = 256 (MoE series 2.1).
 
 Only shapes and options live here; no arithmetic of the method.
 """
@@ -28,6 +32,11 @@ DTYPE_BF16 = 1
 ACT_SILU = 0
 ACT_GELU_ERF = 1
 ACT_GELU_TANH = 2
+
+ORDER_SLOT_MAJOR = 0
+ORDER_TOKEN_MAJOR = 1
+DROP_ZERO = 0
+DROP_RENORM_KEPT = 1
 
 
 @dataclass(frozen=True)
@@ -44,6 +53,9 @@ class MoEConfig:
     capacity_factor: float = 0.0  # <= 0: no capacity
     router_bias_var: float = 0.0  # > 0: per-expert logit bias ~ N(0, var)
     seed: int = 0
+    capacity_order: int = ORDER_SLOT_MAJOR
+    drop_policy: int = DROP_ZERO
+    min_capacity: int = 0
 
     @property
     def records(self) -> int:
@@ -68,6 +80,11 @@ CONFIGS = {
                              capacity_factor=1.25, router_bias_var=2.0),
     "decode": MoEConfig("decode", N=64, D=4096, F=14336, E=8, k=2, dtype=DTYPE_BF16,
                         activation=ACT_SILU, renormalize=1),
+    "capacity_gshard": MoEConfig("capacity_gshard", N=16384, D=2048, F=8192, E=64, k=2,
+                                 dtype=DTYPE_BF16, activation=ACT_SILU, renormalize=1,
+                                 capacity_factor=1.0, router_bias_var=2.0,
+                                 capacity_order=ORDER_TOKEN_MAJOR,
+                                 drop_policy=DROP_RENORM_KEPT, min_capacity=256),
 }
 
 # The workload the throughput benchmark times on one GPU.

@@ -63,7 +63,7 @@ size_t elem_size(const moe_problem& p) { return p.dtype == MOE_DTYPE_BF16 ? 2 : 
 
 // Device workspace regions (byte offsets from the workspace base).
 struct Layout {
-  size_t err, colsum_part, wt, zpart, counts, idx, gate, pos, dropped, load, offsets, row_token,
+  size_t err, colsum_part, wt, counts, idx, gate, pos, dropped, load, offsets, row_token,
       xperm, h, y;
   size_t total;       // moe_forward and every other entry point
   size_t xin, xout;   // moe_forward_host only
@@ -83,7 +83,6 @@ Layout make_layout(const moe_problem& p) {
   L.err = take(256);
   L.colsum_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)) * p.E);
   L.wt = take(route_tc_wt_bytes(p));
-  L.zpart = take(route_tc_zpart_bytes(p));
   L.counts = take(sizeof(int32_t) * static_cast<size_t>(dispatch_num_chunks(R)) * p.E);
   L.idx = take(sizeof(int32_t) * R);
   L.gate = take(sizeof(float) * R);
@@ -118,6 +117,11 @@ moe_status check_problem(const moe_problem* p) {
   if (p->renormalize != 0 && p->renormalize != 1)
     return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
   if (std::isnan(p->capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+  if (p->capacity_order != MOE_ORDER_SLOT_MAJOR && p->capacity_order != MOE_ORDER_TOKEN_MAJOR)
+    return fail(MOE_ERR_INVALID_ARG, "unknown capacity_order");
+  if (p->drop_policy != MOE_DROP_ZERO && p->drop_policy != MOE_DROP_RENORM_KEPT)
+    return fail(MOE_ERR_INVALID_ARG, "unknown drop_policy");
+  if (p->min_capacity < 0) return fail(MOE_ERR_INVALID_ARG, "min_capacity < 0");
   if (p->N * static_cast<int64_t>(p->k) > INT32_MAX)
     return fail(MOE_ERR_UNSUPPORTED, "N*k exceeds 2^31-1 records");
   if (p->D > (1 << 24) || p->F > (1 << 24)) return fail(MOE_ERR_UNSUPPORTED, "D or F > 2^24");
@@ -178,9 +182,10 @@ moe_status check_sm100() {
 int64_t capacity_of(const moe_problem& p) {
   const int64_t R = p.N * static_cast<int64_t>(p.k);
   if (p.capacity_factor <= 0.0) return R;
-  return static_cast<int64_t>(
+  const int64_t c = static_cast<int64_t>(
       std::ceil(p.capacity_factor * static_cast<double>(p.N) * static_cast<double>(p.k) /
                 static_cast<double>(p.E)));
+  return c > p.min_capacity ? c : p.min_capacity;
 }
 
 template <typename T>
@@ -244,8 +249,8 @@ moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, c
     return MOE_OK;
   }
   MOE_CUDA(launch_route(p, X, W_r, bias, logits, idx, gate, at<float>(ws, L.colsum_part),
-                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), at<float>(ws, L.zpart), err,
-                        wait_timeout_ns(), stream),
+                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), err, wait_timeout_ns(),
+                        stream),
            "route");
   MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps, dr,
                               row_token, err, stream),
@@ -304,8 +309,8 @@ moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, cons
     return MOE_OK;
   }
   MOE_CUDA(launch_route(*p, X, W_r, bias, logits, topk_idx, topk_gate, at<float>(ws, L.colsum_part),
-                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), at<float>(ws, L.zpart),
-                        at<int>(ws, L.err), wait_timeout_ns(), s),
+                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), at<int>(ws, L.err),
+                        wait_timeout_ns(), s),
            "route");
   return MOE_OK;
 }
@@ -491,7 +496,7 @@ const char* moe_status_string(moe_status s) {
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
-int32_t moe_version(void) { return 100; }
+int32_t moe_version(void) { return 110; }
 
 }  // extern "C"
 

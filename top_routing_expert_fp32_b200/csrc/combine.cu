@@ -1,7 +1,9 @@
 // Combine: out[t] = sum_j [not dropped] * gate[t,j] * Y[offsets[idx[t,j]] + pos[t,j]].
 //   Grok-1 book ch.5, 5.3.5 (gate-weighted sum over the k expert outputs); LLMs-from-scratch
 //   ch.12, 12.2 (a token accumulates its k contributions; never overwrite); MoE series 2.2
-//   (an overflowed slot contributes nothing; a token with every slot dropped gets 0).
+//   (an overflowed slot contributes nothing; a token with every slot dropped gets 0; case A:
+//   with renorm_kept, a token that lost some slots spreads the whole weight over the kept
+//   ones, gate / sum of kept gates).
 //
 // One block per token, each thread owns 16-byte column chunks of the row. The k rows are read
 // with 16-byte loads, accumulated in fp32 in ascending j (fixed order, no atomics), and
@@ -56,7 +58,7 @@ __global__ void __launch_bounds__(kThreads)
                    const float* __restrict__ gate, const int32_t* __restrict__ offsets,
                    const int32_t* __restrict__ pos, const uint8_t* __restrict__ dropped,
                    uint4* __restrict__ out, int64_t N, int k, int E, int64_t chunks_per_row,
-                   int* err) {
+                   bool renorm_kept, int* err) {
   constexpr int V = Vec16<T>::kElems;
   __shared__ int64_t s_row[kMaxK];
   __shared__ float s_g[kMaxK];
@@ -74,6 +76,19 @@ __global__ void __launch_bounds__(kThreads)
     s_g[j] = gate[rec];
   }
   __syncthreads();
+  if (renorm_kept && threadIdx.x == 0) {
+    float kept_sum = 0.f;
+    int kept = 0;
+    for (int j = 0; j < k; ++j)
+      if (s_row[j] >= 0) {
+        kept_sum += s_g[j];
+        ++kept;
+      }
+    if (kept > 0 && kept < k)
+      for (int j = 0; j < k; ++j)
+        if (s_row[j] >= 0) s_g[j] = s_g[j] / kept_sum;
+  }
+  if (renorm_kept) __syncthreads();
   // With BATCH (long rows), kBatch chunks per thread are loaded (all k rows) before any is
   // used, so a thread keeps about 8 16-byte loads in flight instead of one round trip per
   // chunk; short rows keep the register count (and occupancy) of one chunk at a time.
@@ -123,16 +138,17 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
   const uint4* y = static_cast<const uint4*>(Y);
   uint4* o = static_cast<uint4*>(out);
   const bool batch = chunks >= 4 * kThreads;
+  const bool rk = p.drop_policy == MOE_DROP_RENORM_KEPT && dropped != nullptr;
 #define MOE_COMBINE(T, KM)                                                                     \
   do {                                                                                         \
     if (batch)                                                                                 \
       combine_kernel<T, KM, true><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,   \
                                                                  dropped, o, p.N, p.k, p.E,    \
-                                                                 chunks, err);                 \
+                                                                 chunks, rk, err);             \
     else                                                                                       \
       combine_kernel<T, KM, false><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,  \
                                                                   dropped, o, p.N, p.k, p.E,   \
-                                                                  chunks, err);                \
+                                                                  chunks, rk, err);            \
   } while (0)
   if (p.dtype == MOE_DTYPE_BF16) {
     if (p.k <= 1) MOE_COMBINE(__nv_bfloat16, 1);

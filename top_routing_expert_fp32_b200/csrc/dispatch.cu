@@ -4,7 +4,8 @@
 //   (capacity), 3.2 (dispatch with a dropped mask); LLMs-from-scratch ch.12, 12.2 (N*k
 //   dispatch records); MoE series (GShard/Mixtral/Switch) 2.2 (overflow).
 //
-// Record order is slot-major: r = j*N + t (all rank-0 records in token order, then rank 1 ...).
+// Record order: slot-major r = j*N + t (all rank-0 records in token order, then rank 1 ...)
+// or token-major r = t*k + j (the walkthrough's loop, 3.2), per the problem's capacity_order.
 // pos(t,j) = number of earlier records (in that order) routed to the same expert.
 //   pass 1 (count): records are split into chunks of kDispatchChunk; each block counts its
 //                   chunk per expert (integer shared-memory counters: order-free, exact).
@@ -27,9 +28,21 @@ constexpr int kMaxE = 64;
 constexpr int kAssignThreads = 1024;  // 32 warps: one tile = one chunk
 constexpr int kCountThreads = 256;
 
+// Token and rank of the r-th record in the visiting order.
+__device__ __forceinline__ void record_at(int64_t r, int64_t N, int k, bool token_major,
+                                          int64_t& t, int64_t& j) {
+  if (token_major) {
+    t = r / k;
+    j = r - t * k;
+  } else {
+    j = r / N;
+    t = r - j * N;
+  }
+}
+
 __global__ void __launch_bounds__(kCountThreads)
     count_kernel(const int32_t* __restrict__ idx, int64_t N, int k, int E, int64_t R,
-                 int32_t* __restrict__ counts, int* err) {
+                 bool token_major, int32_t* __restrict__ counts, int* err) {
   __shared__ int hist[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -42,7 +55,8 @@ __global__ void __launch_bounds__(kCountThreads)
     const int64_t r = r0 + threadIdx.x + static_cast<int64_t>(u) * kCountThreads;
     ev[u] = -1;
     if (r < r1) {
-      const int64_t j = r / N, t = r - j * N;
+      int64_t t, j;
+      record_at(r, N, k, token_major, t, j);
       ev[u] = idx[t * k + j];
       if (ev[u] < 0 || ev[u] >= E) {
         record_error(err, MOE_DEVERR_BAD_INDEX);
@@ -60,7 +74,7 @@ __global__ void __launch_bounds__(kCountThreads)
 
 __global__ void __launch_bounds__(kAssignThreads)
     assign_kernel(const int32_t* __restrict__ idx, int64_t N, int k, int E, int64_t R,
-                  int64_t C, int nchunks, const int32_t* __restrict__ counts,
+                  bool token_major, int64_t C, int nchunks, const int32_t* __restrict__ counts,
                   int32_t* __restrict__ load, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ pos, uint8_t* __restrict__ dropped,
                   int32_t* __restrict__ row_token) {
@@ -112,8 +126,7 @@ __global__ void __launch_bounds__(kAssignThreads)
     int64_t j = 0, t = 0;
     int e = -1;
     if (valid) {
-      j = r / N;
-      t = r - j * N;
+      record_at(r, N, k, token_major, t, j);
       e = idx[t * k + j];
       if (e < 0 || e >= E) e = -1;  // recorded by the count pass
     }
@@ -271,12 +284,14 @@ cudaError_t launch_slot_assign(const moe_problem& p, int64_t capacity, const int
     return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.E + 1), stream);
   }
   const int nchunks = dispatch_num_chunks(R);
-  count_kernel<<<nchunks, kCountThreads, 0, stream>>>(idx, p.N, p.k, p.E, R, chunk_counts, err);
+  const bool token_major = p.capacity_order == MOE_ORDER_TOKEN_MAJOR;
+  count_kernel<<<nchunks, kCountThreads, 0, stream>>>(idx, p.N, p.k, p.E, R, token_major,
+                                                     chunk_counts, err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  assign_kernel<<<nchunks, kAssignThreads, 0, stream>>>(idx, p.N, p.k, p.E, R, capacity, nchunks,
-                                                       chunk_counts, load, offsets, pos, dropped,
-                                                       row_token);
+  assign_kernel<<<nchunks, kAssignThreads, 0, stream>>>(idx, p.N, p.k, p.E, R, token_major,
+                                                       capacity, nchunks, chunk_counts, load,
+                                                       offsets, pos, dropped, row_token);
   return cudaGetLastError();
 }
 

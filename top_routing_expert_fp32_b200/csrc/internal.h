@@ -19,20 +19,21 @@ int route_num_blocks(int64_t N, int E);
 
 // Router logits + softmax + top-k + gates. X == nullptr: `logits` is an input.
 // colsum_partial: [route_num_blocks][E] floats (or nullptr when prob_colsum is nullptr).
-// wt / zpart: scratch of the tensor-core logits (route_tc_*_bytes), used for bf16 X.
+// wt: scratch of the tensor-core router (route_tc_wt_bytes), used for bf16 X.
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          float* logits, int32_t* idx, float* gate, float* colsum_partial,
-                         float* prob_colsum, __nv_bfloat16* wt, float* zpart, int* err,
-                         uint64_t timeout_ns, cudaStream_t stream);
+                         float* prob_colsum, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
+                         cudaStream_t stream);
 
-// Tensor-core router logits for bf16 X: splits W_r into three bf16 terms (wt), then writes
-// S split-K slices of partial logits zpart[S][N][Ep] (Ep = E rounded up to 8).
+// Tensor-core router for bf16 X (logits from a three-term bf16 split of W_r, then the routing
+// decision in the same kernel). colsum_partial may be nullptr; *grid_out = blocks that wrote a
+// colsum partial row.
 bool route_tc_supported(const moe_problem& p);
 size_t route_tc_wt_bytes(const moe_problem& p);
-size_t route_tc_zpart_bytes(const moe_problem& p);
-cudaError_t launch_route_tc_logits(const moe_problem& p, const void* X, const float* W_r,
-                                   __nv_bfloat16* wt, float* zpart, int* S_out, int* Ep_out,
-                                   int* err, uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
+                            const float* bias, __nv_bfloat16* wt, float* logits_out, int32_t* idx,
+                            float* gate, float* colsum_partial, int* grid_out, int* err,
+                            uint64_t timeout_ns, cudaStream_t stream);
 
 // 2-D bf16 tensor map (cols contiguous, row stride cols * 2 bytes), box box_cols x box_rows,
 // 128-byte swizzle, out-of-range elements read as zero.

@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace moe {
 namespace {
@@ -32,9 +33,7 @@ struct RouteArgs {
   const void* X;
   const float* W_r;
   const float* bias;
-  const float* logits_in;  // selection kernel input: S slices [S][N][in_stride]
-  int S;                   // slices added in order (1 for given logits)
-  int in_stride;           // floats per token row of logits_in (>= E)
+  const float* logits_in;  // X == nullptr: given logits
   float* logits_out;       // may be nullptr
   int32_t* idx;
   float* gate;
@@ -103,39 +102,8 @@ __device__ __forceinline__ void select_tile(const RouteArgs& a, float (*s_z)[kMa
     float* z = s_z[tl];
     if (a.logits_out != nullptr)
       for (int e = 0; e < E; ++e) a.logits_out[t * E + e] = z[e];
-    float zmax = z[0];
-    for (int e = 1; e < E; ++e) zmax = z[e] > zmax ? z[e] : zmax;
-    uint64_t chosen = 0;
-    int sel[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      sel[j] = 0;
-      if (j < a.k) {
-        int best = -1;
-        for (int e = 0; e < E; ++e) {
-          if ((chosen >> e) & 1ull) continue;
-          if (best < 0 || z[e] > z[best]) best = e;  // strict: equal keeps the lower index
-        }
-        chosen |= 1ull << best;
-        sel[j] = best;
-      }
-    }
-    float s_all = 0.f;
-    for (int e = 0; e < E; ++e) s_all += expf(z[e] - zmax);
-    float s_sel = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < a.k) s_sel += expf(z[sel[j]] - zmax);
-    const float denom = a.renorm ? s_sel : s_all;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < a.k) {
-        a.idx[t * a.k + j] = sel[j];
-        a.gate[t * a.k + j] = expf(z[sel[j]] - zmax) / denom;
-      }
-    }
-    if (a.colsum_partial != nullptr)
-      for (int e = 0; e < E; ++e) z[e] = expf(z[e] - zmax) / s_all;
+    select_token(z, E, a.k, a.renorm, a.idx + t * a.k, a.gate + t * a.k,
+                 a.colsum_partial != nullptr);
   }
   __syncthreads();
   if (a.colsum_partial != nullptr && static_cast<int>(threadIdx.x) < E) {
@@ -480,25 +448,16 @@ __global__ void __launch_bounds__(kWideThreads) route_wide_kernel(RouteArgs a) {
 
 constexpr int kSelThreads = 64;
 
-// Logits of a token = sum of its S slices in slice order (+ bias): given logits (S = 1, no
-// bias) or the tensor-core router's split-K partials.
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(RouteArgs a) {
   __shared__ float s_z[kSelThreads][kMaxE + 1];
   float colsum_acc = 0.f;
   const int E = a.E;
-  const int64_t slice = a.N * a.in_stride;
   for (int64_t tile = blockIdx.x; tile * kSelThreads < a.N; tile += gridDim.x) {
     const int64_t t0 = tile * kSelThreads;
     for (int i = threadIdx.x; i < kSelThreads * E; i += kSelThreads) {
       const int tl = i / E;
       const int e = i % E;
-      if (t0 + tl < a.N) {
-        const float* z = a.logits_in + (t0 + tl) * a.in_stride + e;
-        float v = z[0];
-        for (int s = 1; s < a.S; ++s) v += z[s * slice];
-        if (a.bias != nullptr) v += __ldg(a.bias + e);
-        s_z[tl][e] = v;
-      }
+      if (t0 + tl < a.N) s_z[tl][e] = a.logits_in[(t0 + tl) * E + e];
     }
     __syncthreads();
     select_tile(a, s_z, kSelThreads, t0, colsum_acc);
@@ -589,16 +548,14 @@ int route_num_blocks(int64_t N, int E) {
 
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          float* logits, int32_t* idx, float* gate, float* colsum_partial,
-                         float* prob_colsum, __nv_bfloat16* wt, float* zpart, int* err,
-                         uint64_t timeout_ns, cudaStream_t stream) {
+                         float* prob_colsum, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
+                         cudaStream_t stream) {
   if (p.N == 0) return cudaSuccess;
   RouteArgs a;
   a.X = X;
   a.W_r = W_r;
   a.bias = bias;
   a.logits_in = X == nullptr ? logits : nullptr;
-  a.S = 1;
-  a.in_stride = p.E;
   a.logits_out = X != nullptr ? logits : nullptr;
   a.idx = idx;
   a.gate = gate;
@@ -608,23 +565,14 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
   a.E = p.E;
   a.k = p.k;
   a.renorm = p.renormalize;
-  Kind kind = kind_of(X, p.E, a.D);
+  const Kind kind = kind_of(X, p.E, a.D);
   int grid = 1;
   cudaError_t e = cudaSuccess;
   if (X != nullptr && route_tc_supported(p)) {
-    // bf16 activations: logits on the tensor cores (bf16x3 split of W_r), then selection.
-    int S = 1, Ep = p.E;
-    e = launch_route_tc_logits(p, X, W_r, wt, zpart, &S, &Ep, err, timeout_ns, stream);
-    if (e != cudaSuccess) return e;
-    a.X = nullptr;
-    a.logits_in = zpart;
-    a.S = S;
-    a.in_stride = Ep;
-    kind = Kind::kSelect;
-  } else if (X == nullptr) {
-    a.bias = nullptr;  // given logits are used as they are
-  }
-  if (kind == Kind::kSelect) {
+    // bf16 activations: one tensor-core kernel computes the logits and routes.
+    e = launch_route_tc(p, X, W_r, bias, wt, a.logits_out, idx, gate, a.colsum_partial, &grid, err,
+                        timeout_ns, stream);
+  } else if (kind == Kind::kSelect) {
     grid = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>((p.N + kSelThreads - 1) / kSelThreads, kMaxBlocks)));
     route_select_kernel<<<grid, kSelThreads, 0, stream>>>(a);

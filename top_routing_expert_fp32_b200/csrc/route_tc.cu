@@ -1,87 +1,112 @@
-// Router logits on the tensor cores for bf16 activations: z = X W_r (+ bias) with fp32-level
-// accuracy, where X is [N, D] bf16 and W_r is [D, E] fp32.
-//   Grok-1 book ch.5, 5.2 (router logits kept in fp32); MoE formula-to-code walkthrough 1.1.
+// Router for bf16 activations on the tensor cores: logits z = X W_r (+ bias) with fp32-level
+// accuracy, then softmax, top-k and gates, all in one kernel.
+//   Grok-1 book ch.5, 5.2 (router logits kept in fp32, softmax, TopK) and 5.2.3 (gates);
+//   MoE formula-to-code walkthrough 1.1-1.2; LLMs-from-scratch ch.12, 12.1.
 //
-// The fp32 router weights are split into three bf16 terms, w = w0 + w1 + w2 with
+// Precision. The fp32 router weights are split into three bf16 terms, w = w0 + w1 + w2 with
 // w0 = bf16(w), w1 = bf16(w - w0), w2 = bf16(w - w0 - w1) (the "bf16x3" decomposition of
 // Henry, Tang and Heinecke, "Leveraging the bfloat16 Artificial Intelligence Datatype For
-// Higher-Precision Computations", ARITH 2019). The three terms carry 24 significant bits,
-// as many as the fp32 value; what is left over is below 2^-24 |w|. X is bf16 already, so
-// every product x * w_i is exact in fp32 and one bf16 MMA with fp32 accumulation over the
-// concatenated [w0 | w1 | w2] columns gives all three partial dot products. The epilogue adds
-// them smallest first: z = (z2 + z1) + z0.
+// Higher-Precision Computations", ARITH 2019). The three terms carry 24 significant bits, as
+// many as the fp32 value; what is left over is below 2^-24 |w|. X is bf16 already, so every
+// product x * w_i is exact in fp32, and one bf16 MMA with fp32 accumulation over the
+// concatenated [w0 | w1 | w2] columns gives the three partial dot products; they are added
+// smallest first, z = (z2 + z1) + z0.
 //
 // Kernels:
-//   split_wr_kernel  : W_r [D][E] fp32 -> Wt [NB][D] bf16 (K-major B operand), row
-//                      i * Ep + e holding term i of expert e; padding rows are zero.
-//   route_tc_kernel  : persistent, one CTA per SM, 6 warps (TMA producer, MMA issuer, 4
-//                      epilogue warps). A work unit is a 128-token tile and a slice of the
-//                      D range (split-K when there are fewer tiles than SMs). Each unit's
-//                      partial logits go to zpart[slice][token][Ep]; the selection kernel
-//                      adds the slices in slice order (deterministic, no atomics).
+//   split_wr_kernel : W_r [D][E] fp32 -> Wt [NB][D] bf16 (the K-major B operand); row
+//                     i * Ep + e holds term i of expert e, padding rows are zero.
+//   route_tc_kernel : clusters of S CTAs (S = 1, 2, 4 or 8), persistent over 128-token tiles;
+//                     CTA r of a cluster accumulates the r-th slice of D (split-K), so that
+//                     a batch of few tiles still spreads over the SMs. Warp 0 issues the TMA
+//                     loads, warp 1 the tcgen05.mma, warps 2-5 are the epilogue: each CTA puts
+//                     its partial logits in its own shared memory, the cluster synchronises
+//                     through mbarriers, and CTA r adds the S partials of tokens
+//                     [r*128/S, (r+1)*128/S) of the tile in slice order (distributed shared
+//                     memory loads), adds the bias and takes the routing decision. No global
+//                     round trip, no atomics; the result does not depend on timing.
 // Every barrier wait is bounded in time; on a timeout the CTA records MOE_DEVERR_WAIT_TIMEOUT,
-// drains its MMAs and frees its tensor memory.
+// unwinds, drains its MMAs and frees its tensor memory.
 #include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kRows = 128;         // tokens per tile = accumulator lanes
-constexpr int BK = 64;             // k-block: one 128-byte swizzle row of bf16
-constexpr int UK = 16;             // K of one tcgen05.mma kind::f16
+constexpr int kRows = 128;        // tokens per tile = accumulator lanes
+constexpr int BK = 64;            // k-block: one 128-byte swizzle row of bf16
+constexpr int UK = 16;            // K of one tcgen05.mma kind::f16
 constexpr int kThreads = 192;
-constexpr int kMaxNB = 192;        // 3 terms x 64 experts
-constexpr int kABytes = kRows * BK * 2;           // 16 KB
-constexpr int kBBytesMax = kMaxNB * BK * 2;       // 24 KB
-constexpr int kStageBytes = kABytes + kBBytesMax;  // 40 KB
-constexpr int kStages = 5;
-constexpr int kAccStride = 256;    // TMEM columns between the two accumulators
+constexpr int kEpiThreads = 128;  // warps 2-5
+constexpr int kABytes = kRows * BK * 2;  // 16 KB
+constexpr int kMaxStages = 8;
+constexpr int kMaxCluster = 8;
+constexpr int kAccStride = 256;   // TMEM columns between the two accumulators
 constexpr int kTmemCols = 512;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int kUnitTarget = 148;   // work units wanted per launch (one per SM of a B200)
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kUnitTarget = 148;  // CTAs wanted per launch (one per SM of a B200)
+constexpr int kMaxEc = 64;
 
-struct TcParams {
-  float* zpart;       // [S][N][Ep]
+struct TcArgs {
+  const float* bias;       // [E] or nullptr
+  float* logits_out;       // [N][E] or nullptr
+  int32_t* idx;            // [N][k]
+  float* gate;             // [N][k]
+  float* colsum_partial;   // [gridDim.x][E] or nullptr
   int64_t N;
-  int Ep;             // experts padded to a multiple of 8 (TMEM load granularity)
-  int NB;             // MMA N: 3 * Ep padded to a multiple of 16
-  int num_kb;         // k-blocks over D
-  int kps;            // k-blocks per slice
-  int S;              // slices
-  int64_t units;      // tiles * S
+  int64_t tiles;
+  int E, k, renorm;
+  int Ep;                  // E rounded up to 8 (TMEM load granularity)
+  int NB;                  // MMA N: 3 * Ep rounded up to 16
+  int zstride;             // floats per row of the partial-logit buffer (Ep + 4)
+  int num_kb, S, num_clusters, stages;
+  uint32_t stage_bytes, b_off, zbuf_off, sz_off, bar_off;
   int* err;
   uint64_t timeout_ns;
 };
 
+// EB: the experts the epilogue holds in registers per token (8, 16, 32 or 64; >= E).
+template <int EB>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                    const TcParams p) {
+                    const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  float* zbuf = reinterpret_cast<float*>(smem + a.zbuf_off);   // [128][zstride] own partials
+  float* s_z = reinterpret_cast<float*>(smem + a.sz_off);      // [128/S][E+1] summed logits
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.bar_off);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* zready = tempty + 2;  // all S partials of the current tile are in place
+  uint64_t* zfree = zready + 1;   // every CTA has finished reading this CTA's partials
+  uint64_t* drain = zfree + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (static_cast<int64_t>(blockIdx.x) >= p.units) return;  // uniform over the block
+  const int S = a.S;
+  const uint32_t rank = cluster_ctarank();
+  const int64_t first_tile = blockIdx.x / S;  // the cluster index; same for every CTA of it
+  // k-blocks [kb0, kb1) of this CTA: an even share, at least one since S <= num_kb.
+  const int kb0 = static_cast<int>((static_cast<int64_t>(rank) * a.num_kb) / S);
+  const int kb1 = static_cast<int>((static_cast<int64_t>(rank + 1) * a.num_kb) / S);
+  const bool has_k = kb1 > kb0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < a.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
     }
+    mbar_init(zready, 4 * S);  // one arrival per epilogue warp of every CTA of the cluster
+    mbar_init(zfree, 4 * S);
     mbar_init(drain, 1);
     fence_barrier_init();
     prefetch_tensormap(&tmX);
@@ -92,32 +117,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();  // every CTA's barriers exist before any remote arrival
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
-  const uint32_t tx_bytes = static_cast<uint32_t>(kABytes + p.NB * BK * 2);
+  const uint32_t tx_bytes = static_cast<uint32_t>(kABytes + a.NB * BK * 2);
 
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        const int64_t tile = u / p.S;
-        const int s = static_cast<int>(u - tile * p.S);
-        const int kb0 = s * p.kps;
-        const int kb1 = min(kb0 + p.kps, p.num_kb);
+      for (int64_t tile = first_tile; ok && tile < a.tiles; tile += a.num_clusters) {
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns)) {
-            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+          if (!mbar_wait(&empty[stage], phase ^ 1u, a.timeout_ns)) {
+            record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
             ok = false;
             break;
           }
-          uint8_t* a_dst = smem + stage * kStageBytes;
+          uint8_t* dst = smem + stage * a.stage_bytes;
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
-          tma_load_2d(a_dst, &tmX, &full[stage], kb * BK, static_cast<int>(tile * kRows));
-          tma_load_2d(a_dst + kABytes, &tmW, &full[stage], kb * BK, 0);
-          if (++stage == kStages) {
+          tma_load_2d(dst, &tmX, &full[stage], kb * BK, static_cast<int>(tile * kRows));
+          tma_load_2d(dst + a.b_off, &tmW, &full[stage], kb * BK, 0);
+          if (++stage == a.stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -129,35 +151,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       // kind::f16: D fp32 (bit 4), A bf16 (bits 7-9), B bf16 (bits 10-12), both K-major,
       // N >> 3 at bit 17, M >> 4 at bit 24.
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                             (static_cast<uint32_t>(p.NB >> 3) << 17) |
+                             (static_cast<uint32_t>(a.NB >> 3) << 17) |
                              (static_cast<uint32_t>(kRows >> 4) << 24);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int64_t u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++it) {
-        const int64_t tile = u / p.S;
-        const int s = static_cast<int>(u - tile * p.S);
-        const int kb0 = s * p.kps;
-        const int kb1 = min(kb0 + p.kps, p.num_kb);
+      for (int64_t tile = first_tile; ok && tile < a.tiles; tile += a.num_clusters, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
-          record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, a.timeout_ns)) {
+          record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
-            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+          if (!mbar_wait(&full[stage], phase, a.timeout_ns)) {
+            record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint32_t a_addr = smem_u32(smem + stage * a.stage_bytes);
+          const uint32_t b_addr = a_addr + a.b_off;
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
             // Both operands K-major SW128: advance 16 elements = 32 bytes in the swizzle row.
@@ -166,124 +184,240 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16_ss(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
-          if (++stage == kStages) {
+          if (++stage == a.stages) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) umma_commit(&tfull[acc]);
+        if (ok) umma_commit(&tfull[acc]);  // with no k-block this arrives at once
       }
       umma_commit(drain);  // flips once every MMA issued above has completed
-      if (!mbar_wait(drain, 0, p.timeout_ns)) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+      if (!mbar_wait(drain, 0, a.timeout_ns)) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
     }
   } else {  // ------------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // this warp may access TMEM lanes [32q, 32q+32)
+    // Thread row = q*32 + lane reads TMEM lane `row` (tile row = token). With S = 1 it owns
+    // that token outright; with S > 1 every row's partial goes to shared memory and the
+    // thread whose row lies in this CTA's share [rank*T, rank*T + T) adds the S partials.
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127, for the per-expert column sums
+    const int T = kRows / S;
+    const int share0 = static_cast<int>(rank) * T;
+    const bool owner = row >= share0 && row < share0 + T;
+    const int E = a.E;
+    const uint32_t zrow_s = smem_u32(zbuf) + static_cast<uint32_t>(row * a.zstride) * 4u;
+    float colsum_acc = 0.f;
     int it = 0;
-    for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x, ++it) {
-      const int64_t tile = u / p.S;
-      const int s = static_cast<int>(u - tile * p.S);
+    for (int64_t tile = first_tile; tile < a.tiles; tile += a.num_clusters, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, p.timeout_ns);
-      if (__any_sync(0xffffffffu, !ok)) {
-        if (lane == 0) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+      bool ok = mbar_wait(&tfull[acc], acc_phase, a.timeout_ns);
+      // The previous tile's partials must have been read by every CTA before they are
+      // overwritten.
+      if (S > 1 && ok && it > 0)
+        ok = mbar_wait_cluster(zfree, static_cast<uint32_t>(it - 1) & 1u, a.timeout_ns);
+      // Leave together: the four epilogue warps share named barriers below.
+      if (named_bar_any(1, kEpiThreads, !ok)) {
+        if (et == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
         break;
       }
       __syncwarp();
       tc_fence_after_sync();
-      const int64_t t = tile * kRows + q * 32 + lane;
-      const bool valid = t < p.N;
-      float* zrow = p.zpart + (static_cast<int64_t>(s) * p.N + (valid ? t : 0)) * p.Ep;
+      // 1. Accumulator -> registers, the three terms added smallest first.
+      float z[EB];
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * kAccStride);
-#pragma unroll 1
-      for (int g = 0; g < p.Ep; g += 8) {
-        uint32_t r0[8], r1[8], r2[8];
-        tmem_ld_8cols(t_row + g, r0);                // w0 term
-        tmem_ld_8cols(t_row + p.Ep + g, r1);         // w1 term
-        tmem_ld_8cols(t_row + 2 * p.Ep + g, r2);     // w2 term
-        tmem_ld_wait();
-        if (valid) {
-          float z[8];
+#pragma unroll
+      for (int g = 0; g < EB; g += 8) {
+        if (g < a.Ep && has_k) {
+          uint32_t r0[8], r1[8], r2[8];
+          tmem_ld_8cols(t_row + g, r0);
+          tmem_ld_8cols(t_row + a.Ep + g, r1);
+          tmem_ld_8cols(t_row + 2 * a.Ep + g, r2);
+          tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            z[i] = (__uint_as_float(r2[i]) + __uint_as_float(r1[i])) + __uint_as_float(r0[i]);
-          reinterpret_cast<float4*>(zrow + g)[0] = make_float4(z[0], z[1], z[2], z[3]);
-          reinterpret_cast<float4*>(zrow + g)[1] = make_float4(z[4], z[5], z[6], z[7]);
+            z[g + i] = (__uint_as_float(r2[i]) + __uint_as_float(r1[i])) + __uint_as_float(r0[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) z[g + i] = 0.f;
         }
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) mbar_arrive(&tempty[acc]);  // the MMA warp may reuse this accumulator
+      if (S > 1) {
+        // 2. Publish this CTA's partials, then add the S partials of the owned rows in slice
+        //    order (distributed shared memory).
+#pragma unroll
+        for (int c = 0; c < EB; c += 4)
+          if (c < a.Ep)
+            reinterpret_cast<float4*>(zbuf + row * a.zstride)[c / 4] =
+                make_float4(z[c], z[c + 1], z[c + 2], z[c + 3]);
+        fence_cluster();  // this lane's partials before lane 0's release to the peers
+        __syncwarp();
+        if (lane == 0)
+          for (int r = 0; r < S; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(zready), r));
+        ok = mbar_wait_cluster(zready, static_cast<uint32_t>(it) & 1u, a.timeout_ns);
+        if (named_bar_any(1, kEpiThreads, !ok)) {
+          if (et == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
+          break;
+        }
+        if (owner) {
+          float v[EB];
+#pragma unroll
+          for (int c = 0; c < EB; c += 4) {
+            if (c < a.Ep) {
+              float4 acc4 = rank == 0 ? make_float4(z[c], z[c + 1], z[c + 2], z[c + 3])
+                                      : ld_dsmem_f4(mapa_shared(zrow_s + c * 4u, 0));
+#pragma unroll
+              for (int r = 1; r < kMaxCluster; ++r) {
+                if (r < S) {
+                  const float4 w = r == static_cast<int>(rank)
+                                       ? make_float4(z[c], z[c + 1], z[c + 2], z[c + 3])
+                                       : ld_dsmem_f4(mapa_shared(zrow_s + c * 4u, r));
+                  acc4.x += w.x;
+                  acc4.y += w.y;
+                  acc4.z += w.z;
+                  acc4.w += w.w;
+                }
+              }
+              v[c] = acc4.x;
+              v[c + 1] = acc4.y;
+              v[c + 2] = acc4.z;
+              v[c + 3] = acc4.w;
+            } else {
+              v[c] = v[c + 1] = v[c + 2] = v[c + 3] = 0.f;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < EB; ++e) z[e] = v[e];
+        }
+        fence_cluster();  // this lane's reads of the peers' partials before the release below
+        __syncwarp();
+        if (lane == 0)  // done reading every CTA's partials of this tile
+          for (int r = 0; r < S; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(zfree), r));
+      }
+      // 3. Bias and the routing decision for the owned tokens.
+      const int64_t t = tile * kRows + row;
+      if (owner && t < a.N) {
+#pragma unroll
+        for (int e = 0; e < EB; ++e)
+          if (e < E && a.bias != nullptr) z[e] += __ldg(a.bias + e);
+        if (a.logits_out != nullptr)
+#pragma unroll
+          for (int e = 0; e < EB; ++e)
+            if (e < E) a.logits_out[t * E + e] = z[e];
+        select_token_regs<EB>(z, E, a.k, a.renorm, a.idx + t * a.k, a.gate + t * a.k,
+                              a.colsum_partial != nullptr ? s_z + (row - share0) * (E + 1)
+                                                          : nullptr);
+      }
+      if (a.colsum_partial != nullptr) {  // per-expert probability sums in token order
+        named_bar_sync(1, kEpiThreads);
+        if (et < E) {
+          const int64_t left = a.N - (tile * kRows + share0);
+          const int valid = left < T ? static_cast<int>(left > 0 ? left : 0) : T;
+          for (int i = 0; i < valid; ++i) colsum_acc += s_z[i * (E + 1) + et];
+        }
+        named_bar_sync(1, kEpiThreads);
+      }
     }
+    if (a.colsum_partial != nullptr && et < E)
+      a.colsum_partial[static_cast<int64_t>(blockIdx.x) * E + et] = colsum_acc;
   }
 
-  __syncwarp();  // role branches leave warps 0 and 1 divergent; the barrier below is .aligned
+  __syncwarp();  // role branches leave warps 0 and 1 divergent; the barriers below are .aligned
   __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  __syncwarp();
+  cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
 }
 
 // Wt[i * Ep + e][d] = term i of W_r[d][e] (zero for e >= E and for rows >= 3 * Ep).
-// A block converts 64 rows of W_r (contiguous in memory) through shared memory.
-constexpr int kSplitRows = 64;
+// One thread per (row group, 8 consecutive d): rows e, Ep + e and 2 Ep + e for e < Ep, or one
+// padding row past 3 Ep; each row written as one 16-byte store (D % 8 == 0).
 constexpr int kSplitThreads = 256;
 
 __global__ void __launch_bounds__(kSplitThreads)
     split_wr_kernel(const float* __restrict__ W_r, __nv_bfloat16* __restrict__ Wt, int D, int E,
                     int Ep, int NB) {
-  __shared__ float s_w[kSplitRows * 64];
-  const int d0 = blockIdx.x * kSplitRows;
-  const int rows = min(kSplitRows, D - d0);
-  for (int i = threadIdx.x; i < rows * E; i += kSplitThreads)
-    s_w[i] = W_r[static_cast<int64_t>(d0) * E + i];
-  __syncthreads();
-  // Output element (n, d0 + dd): consecutive threads take consecutive dd (coalesced rows).
-  for (int i = threadIdx.x; i < NB * kSplitRows; i += kSplitThreads) {
-    const int n = i / kSplitRows;
-    const int dd = i - n * kSplitRows;
-    if (dd >= rows) continue;
-    const int term = n / Ep;
-    const int e = n - term * Ep;
-    float v = 0.f;
-    if (term < 3 && e < E) {
-      const float w = s_w[dd * E + e];
-      const float w0 = __bfloat162float(__float2bfloat16_rn(w));
-      const float r1 = w - w0;  // exact: w0 holds w's leading 8 significant bits
-      const float w1 = __bfloat162float(__float2bfloat16_rn(r1));
-      const float r2 = r1 - w1;  // exact for the same reason
-      v = term == 0 ? w0 : (term == 1 ? w1 : __bfloat162float(__float2bfloat16_rn(r2)));
-    }
-    Wt[static_cast<int64_t>(n) * D + d0 + dd] = __float2bfloat16_rn(v);
+  const int chunks = D / 8;
+  const int groups = Ep + (NB - 3 * Ep);  // experts, then padding rows
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kSplitThreads + threadIdx.x;
+  if (i >= static_cast<int64_t>(groups) * chunks) return;
+  const int grp = static_cast<int>(i / chunks);
+  const int d0 = static_cast<int>(i - static_cast<int64_t>(grp) * chunks) * 8;
+  if (grp >= Ep) {  // padding row 3 Ep + (grp - Ep)
+    *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(3 * Ep + grp - Ep) * D + d0) =
+        make_uint4(0u, 0u, 0u, 0u);
+    return;
   }
+  const int e = grp;
+  float t0[8], t1[8], t2[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float w = e < E ? __ldg(W_r + static_cast<int64_t>(d0 + j) * E + e) : 0.f;
+    t0[j] = __bfloat162float(__float2bfloat16_rn(w));
+    const float r1 = w - t0[j];  // exact: t0 holds w's leading 8 significant bits
+    t1[j] = __bfloat162float(__float2bfloat16_rn(r1));
+    t2[j] = r1 - t1[j];          // exact for the same reason; rounded to bf16 below
+  }
+  uint4 v0, v1, v2;
+  v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]), pack_bf16x2(t0[4], t0[5]),
+                  pack_bf16x2(t0[6], t0[7]));
+  v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]), pack_bf16x2(t1[4], t1[5]),
+                  pack_bf16x2(t1[6], t1[7]));
+  v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]), pack_bf16x2(t2[4], t2[5]),
+                  pack_bf16x2(t2[6], t2[7]));
+  *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(e) * D + d0) = v0;
+  *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(Ep + e) * D + d0) = v1;
+  *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(2 * Ep + e) * D + d0) = v2;
 }
 
 struct TcShape {
-  int Ep, NB, num_kb, kps, S;
+  int Ep, NB, zstride, num_kb, S, num_clusters, stages;
   int64_t tiles;
+  uint32_t stage_bytes, b_off, zbuf_off, sz_off, bar_off, smem_bytes;
 };
 
 TcShape tc_shape(int64_t N, int D, int E) {
-  TcShape s;
+  TcShape s{};
   s.Ep = (E + 7) / 8 * 8;
   s.NB = (3 * s.Ep + 15) / 16 * 16;
+  s.zstride = s.Ep + 4;  // rows 16 bytes apart in the bank map: conflict-free float4 stores
   s.num_kb = (D + BK - 1) / BK;
   s.tiles = (N + kRows - 1) / kRows;
-  // Slices per tile: as many as keep tiles * S within one unit per SM.
-  const int want = static_cast<int>(
-      std::min<int64_t>(s.num_kb, std::max<int64_t>(1, kUnitTarget / std::max<int64_t>(1, s.tiles))));
-  s.kps = (s.num_kb + want - 1) / want;
-  s.S = (s.num_kb + s.kps - 1) / s.kps;  // no empty slice
+  // Cluster size: the largest power of two <= 8 that keeps tiles * S within one CTA per SM and
+  // leaves every CTA at least one k-block.
+  const int64_t want = std::max<int64_t>(1, kUnitTarget / std::max<int64_t>(1, s.tiles));
+  s.S = 1;
+  while (s.S * 2 <= kMaxCluster && s.S * 2 <= want && s.S * 2 <= s.num_kb) s.S *= 2;
+  s.num_clusters = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(s.tiles, kUnitTarget / s.S)));
+  // Shared memory: [stages][A 16 KB | B] [partials 128 x zstride] [summed logits] [barriers]
+  s.b_off = kABytes;
+  s.stage_bytes = static_cast<uint32_t>(kABytes + (s.NB * BK * 2 + 1023) / 1024 * 1024);
+  // Partials are exchanged only between the CTAs of a cluster (S > 1).
+  const uint32_t zbuf_bytes = s.S > 1 ? static_cast<uint32_t>(kRows * s.zstride * 4) : 0u;
+  const uint32_t sz_bytes = static_cast<uint32_t>(((kRows / s.S) * (E + 1) * 4 + 15) / 16 * 16);
+  const uint32_t fixed = 1024 /*align*/ + 256 /*barriers*/ + zbuf_bytes + sz_bytes;
+  s.stages = static_cast<int>(
+      std::min<uint32_t>(kMaxStages, (kSmemLimit - fixed) / s.stage_bytes));
+  s.zbuf_off = static_cast<uint32_t>(s.stages) * s.stage_bytes;
+  s.sz_off = s.zbuf_off + zbuf_bytes;
+  s.bar_off = s.sz_off + sz_bytes;
+  s.smem_bytes = s.bar_off + 256 + 1024;
   return s;
 }
 
 }  // namespace
 
 bool route_tc_supported(const moe_problem& p) {
-  return p.dtype == MOE_DTYPE_BF16 && p.E <= 64;
+  return p.dtype == MOE_DTYPE_BF16 && p.E <= kMaxEc;
 }
 
 size_t route_tc_wt_bytes(const moe_problem& p) {
@@ -292,45 +426,72 @@ size_t route_tc_wt_bytes(const moe_problem& p) {
   return static_cast<size_t>(s.NB) * static_cast<size_t>(p.D) * 2;
 }
 
-size_t route_tc_zpart_bytes(const moe_problem& p) {
-  if (!route_tc_supported(p)) return 0;
+cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
+                            const float* bias, __nv_bfloat16* wt, float* logits_out, int32_t* idx,
+                            float* gate, float* colsum_partial, int* grid_out, int* err,
+                            uint64_t timeout_ns, cudaStream_t stream) {
   const TcShape s = tc_shape(p.N, static_cast<int>(p.D), p.E);
-  return static_cast<size_t>(s.S) * static_cast<size_t>(p.N) * s.Ep * sizeof(float);
-}
-
-cudaError_t launch_route_tc_logits(const moe_problem& p, const void* X, const float* W_r,
-                                   __nv_bfloat16* Wt, float* zpart, int* S_out, int* Ep_out,
-                                   int* err, uint64_t timeout_ns, cudaStream_t stream) {
-  const TcShape s = tc_shape(p.N, static_cast<int>(p.D), p.E);
-  *S_out = s.S;
-  *Ep_out = s.Ep;
+  *grid_out = 0;
   if (p.N == 0) return cudaSuccess;
+  if (s.stages < 2) return cudaErrorInvalidConfiguration;
   const int D = static_cast<int>(p.D);
-  split_wr_kernel<<<(D + kSplitRows - 1) / kSplitRows, kSplitThreads, 0, stream>>>(
-      W_r, Wt, D, p.E, s.Ep, s.NB);
+  const int64_t split_threads = static_cast<int64_t>(s.Ep + (s.NB - 3 * s.Ep)) * (D / 8);
+  split_wr_kernel<<<static_cast<unsigned>((split_threads + kSplitThreads - 1) / kSplitThreads),
+                    kSplitThreads, 0, stream>>>(W_r, wt, D, p.E, s.Ep, s.NB);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tX, tW;
   if (!make_tensor_map_2d_bf16(&tX, X, static_cast<uint64_t>(D), static_cast<uint64_t>(p.N), 64,
                                kRows) ||
-      !make_tensor_map_2d_bf16(&tW, Wt, static_cast<uint64_t>(D), static_cast<uint64_t>(s.NB), 64,
+      !make_tensor_map_2d_bf16(&tW, wt, static_cast<uint64_t>(D), static_cast<uint64_t>(s.NB), 64,
                                static_cast<uint32_t>(s.NB)))
     return cudaErrorInvalidValue;
-  TcParams tp;
-  tp.zpart = zpart;
-  tp.N = p.N;
-  tp.Ep = s.Ep;
-  tp.NB = s.NB;
-  tp.num_kb = s.num_kb;
-  tp.kps = s.kps;
-  tp.S = s.S;
-  tp.units = s.tiles * s.S;
-  tp.err = err;
-  tp.timeout_ns = timeout_ns;
-  e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  TcArgs a;
+  a.bias = bias;
+  a.logits_out = logits_out;
+  a.idx = idx;
+  a.gate = gate;
+  a.colsum_partial = colsum_partial;
+  a.N = p.N;
+  a.tiles = s.tiles;
+  a.E = p.E;
+  a.k = p.k;
+  a.renorm = p.renormalize;
+  a.Ep = s.Ep;
+  a.NB = s.NB;
+  a.zstride = s.zstride;
+  a.num_kb = s.num_kb;
+  a.S = s.S;
+  a.num_clusters = s.num_clusters;
+  a.stages = s.stages;
+  a.stage_bytes = s.stage_bytes;
+  a.b_off = s.b_off;
+  a.zbuf_off = s.zbuf_off;
+  a.sz_off = s.sz_off;
+  a.bar_off = s.bar_off;
+  a.err = err;
+  a.timeout_ns = timeout_ns;
+  void (*kern)(const CUtensorMap, const CUtensorMap, const TcArgs) =
+      s.Ep <= 8 ? route_tc_kernel<8>
+                : (s.Ep <= 16 ? route_tc_kernel<16> : (s.Ep <= 32 ? route_tc_kernel<32> : route_tc_kernel<64>));
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(s.smem_bytes));
   if (e != cudaSuccess) return e;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), tp.units)));
-  route_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tX, tW, tp);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(s.num_clusters * s.S));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = s.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(s.S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tX, tW, a);
+  if (e != cudaSuccess) return e;
+  *grid_out = s.num_clusters * s.S;
   return cudaGetLastError();
 }
 
