@@ -256,7 +256,10 @@ def run_gpu(args, cfg, world, rank, device):
     stream = torch.cuda.current_stream(device)
 
     names = ["route", "dispatch", "up", "down", "combine"]
-    launches = {"route": 1, "dispatch": 3, "up": 1, "down": 1, "combine": 1}
+    # Kernels per step: route = W_r split + tensor-core router (bf16 X) or one SIMT router
+    # (fp32 X); dispatch = count + assign + gather; one launch each for up, down, combine.
+    launches = {"route": 2 if cfg.dtype == configs.DTYPE_BF16 else 1, "dispatch": 3, "up": 1,
+                "down": 1, "combine": 1}
 
     def step(ev):
         ev[0].record(stream)
