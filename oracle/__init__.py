@@ -70,6 +70,12 @@ def lib():
         L.oracle_forward.argtypes = [i64, i64, i64, i32, i32, f64, i64, i32, i32, i32, i32,
                                      i32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.oracle_forward.restype = ctypes.c_int
+        L.oracle_forward_w8.argtypes = [i64, i64, i64, i32, i32, f64, i64, i32, i32, i32, i32,
+                                        i32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                        P]
+        L.oracle_forward_w8.restype = ctypes.c_int
+        L.oracle_expert_ffn_w8.argtypes = [i64, P, P, i64, i64, P, i32, P, P, P, P, P, P, i32, P]
+        L.oracle_expert_ffn_w8.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
@@ -178,6 +184,24 @@ def expert_ffn(rec_token, rec_expert, X, W1, W2, W3, dtype: int, act: int) -> np
     return Y
 
 
+def expert_ffn_w8(rec_token, rec_expert, X, x_dtype: int, W1q, S1, W2q, S2, W3q, S3,
+                  act: int) -> np.ndarray:
+    """fp64 gated expert output with 8-bit weights: W = q * s, s per expert and output column.
+    W1q, W2q [E,D,F] int8, W3q [E,F,D] int8; S1, S2 [E,F], S3 [E,D] fp32."""
+    rec_token = _c(rec_token, np.int32)
+    rec_expert = _c(rec_expert, np.int32)
+    X = _elems(X, x_dtype)
+    W1q, W2q, W3q = (_c(w, np.int8) for w in (W1q, W2q, W3q))
+    S1, S2, S3 = (_c(s, np.float32) for s in (S1, S2, S3))
+    n = rec_token.shape[0]
+    D = X.shape[1]
+    F = W1q.shape[2]
+    Y = np.empty((n, D), np.float64)
+    lib().oracle_expert_ffn_w8(n, _p(rec_token), _p(rec_expert), D, F, _p(X), x_dtype, _p(W1q),
+                               _p(S1), _p(W2q), _p(S2), _p(W3q), _p(S3), act, _p(Y))
+    return Y
+
+
 def combine(gate, dropped, Yrec, policy: int = DROP_ZERO) -> np.ndarray:
     gate = _c(gate, np.float64)
     N, k = gate.shape
@@ -230,6 +254,39 @@ def forward(X, W_r, bias, W1, W2, W3, *, k: int, cf: float, renorm: int, act: in
                               _p(colsum))
     if rc != 0:
         raise ValueError("oracle_forward: non-finite logits")
+    return dict(out=out, logits32=l32, idx=idx, gate=gate, load=load, offsets=offsets,
+                pos=pos, dropped=dropped, colsum=colsum)
+
+
+def forward_w8(X, W_r, bias, W1q, S1, W2q, S2, W3q, S3, *, k: int, cf: float, renorm: int,
+               act: int, dtype: int, min_capacity: int = 0, order: int = SLOT_MAJOR,
+               drop_policy: int = DROP_ZERO):
+    """Whole layer in fp64 with 8-bit expert weights (W = q * s per expert and output column).
+    Returns the same dict as forward()."""
+    X = _elems(X, dtype)
+    W1q, W2q, W3q = (_c(w, np.int8) for w in (W1q, W2q, W3q))
+    S1, S2, S3 = (_c(s, np.float32) for s in (S1, S2, S3))
+    N, D = X.shape
+    E = W_r.shape[1]
+    F = W1q.shape[2]
+    W_r = _c(W_r, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((N, D), np.float64)
+    l32 = np.empty((N, E), np.float32)
+    idx = np.empty((N, k), np.int32)
+    gate = np.empty((N, k), np.float64)
+    load = np.empty((E,), np.int32)
+    offsets = np.empty((E + 1,), np.int32)
+    pos = np.empty((N, k), np.int32)
+    dropped = np.empty((N, k), np.uint8)
+    colsum = np.empty((E,), np.float64)
+    rc = lib().oracle_forward_w8(N, D, F, E, k, float(cf), int(min_capacity), order, drop_policy,
+                                 renorm, act, dtype, _p(X), _p(W_r), _p(b), _p(W1q), _p(S1),
+                                 _p(W2q), _p(S2), _p(W3q), _p(S3), _p(out), _p(l32), _p(idx),
+                                 _p(gate), _p(load), _p(offsets), _p(pos), _p(dropped),
+                                 _p(colsum))
+    if rc != 0:
+        raise ValueError("oracle_forward_w8: non-finite logits")
     return dict(out=out, logits32=l32, idx=idx, gate=gate, load=load, offsets=offsets,
                 pos=pos, dropped=dropped, colsum=colsum)
 

@@ -278,14 +278,39 @@ static double activation(double a, int32_t act) {
   }
 }
 
+/* Where an expert weight matrix comes from: plain fp32/bf16 values (W, dtype), or 8-bit
+ * weights with one scale per expert and output column (Q, S), dequantized as q * s before the
+ * matmul ([G5] 5.3.3, "weight = weight * scales"; the scales broadcast over the reduction
+ * dimension, the reading that makes the 8-bit copy smaller than the bf16 one). */
+typedef struct {
+  const void* W;
+  int32_t dtype;
+  const int8_t* Q;
+  const float* S;
+} wsrc;
+
+/* Row `row` of expert e's [rows, n] matrix, widened (or dequantized, exactly) to double. */
+static void weight_row(const wsrc* w, int64_t e, int64_t rows, int64_t row, int64_t n,
+                       double* out) {
+  const int64_t first = (e * rows + row) * n;
+  if (w->Q) {
+    const int8_t* q = w->Q + first;
+    const float* sc = w->S + e * n;
+    for (int64_t i = 0; i < n; ++i) out[i] = (double)q[i] * (double)sc[i];
+  } else {
+    widen(w->W, w->dtype, first, n, out);
+  }
+}
+
 /* Gated expert of record r (token t = rec_token[r], expert e = rec_expert[r]):
  *   a = x W1_e, b = x W2_e  (sum over d ascending),  h = act(a) (.) b,
  *   y = h W3_e              (sum over f ascending).
  * W1 (activated branch, Grok "linear"), W2 (linear branch, Grok "linear_v"): [E,D,F];
  * W3 (Grok "linear_1"): [E,F,D]. Y: [n_rec, D] doubles. */
-void oracle_expert_ffn(int64_t n_rec, const int32_t* rec_token, const int32_t* rec_expert,
-                       int64_t D, int64_t F, const void* X, const void* W1, const void* W2,
-                       const void* W3, int32_t dtype, int32_t act, double* Y) {
+static void expert_ffn_core(int64_t n_rec, const int32_t* rec_token, const int32_t* rec_expert,
+                            int64_t D, int64_t F, const void* X, int32_t x_dtype,
+                            const wsrc* W1, const wsrc* W2, const wsrc* W3, int32_t act,
+                            double* Y) {
 #pragma omp parallel
   {
     double* x = (double*)malloc(sizeof(double) * (size_t)D);
@@ -295,19 +320,19 @@ void oracle_expert_ffn(int64_t n_rec, const int32_t* rec_token, const int32_t* r
 #pragma omp for schedule(dynamic, 1)
     for (int64_t r = 0; r < n_rec; ++r) {
       const int64_t t = rec_token[r], e = rec_expert[r];
-      widen(X, dtype, t * D, D, x);
+      widen(X, x_dtype, t * D, D, x);
       for (int64_t f = 0; f < F; ++f) a[f] = b[f] = 0.0;
       for (int64_t d = 0; d < D; ++d) {
-        widen(W1, dtype, (e * D + d) * F, F, w);
+        weight_row(W1, e, D, d, F, w);
         for (int64_t f = 0; f < F; ++f) a[f] += x[d] * w[f];
-        widen(W2, dtype, (e * D + d) * F, F, w);
+        weight_row(W2, e, D, d, F, w);
         for (int64_t f = 0; f < F; ++f) b[f] += x[d] * w[f];
       }
       for (int64_t f = 0; f < F; ++f) a[f] = activation(a[f], act) * b[f]; /* h */
       double* y = Y + r * D;
       for (int64_t d = 0; d < D; ++d) y[d] = 0.0;
       for (int64_t f = 0; f < F; ++f) {
-        widen(W3, dtype, (e * F + f) * D, D, w);
+        weight_row(W3, e, F, f, D, w);
         for (int64_t d = 0; d < D; ++d) y[d] += a[f] * w[d];
       }
     }
@@ -316,6 +341,23 @@ void oracle_expert_ffn(int64_t n_rec, const int32_t* rec_token, const int32_t* r
     free(b);
     free(w);
   }
+}
+
+void oracle_expert_ffn(int64_t n_rec, const int32_t* rec_token, const int32_t* rec_expert,
+                       int64_t D, int64_t F, const void* X, const void* W1, const void* W2,
+                       const void* W3, int32_t dtype, int32_t act, double* Y) {
+  const wsrc w1 = {W1, dtype, NULL, NULL}, w2 = {W2, dtype, NULL, NULL}, w3 = {W3, dtype, NULL, NULL};
+  expert_ffn_core(n_rec, rec_token, rec_expert, D, F, X, dtype, &w1, &w2, &w3, act, Y);
+}
+
+/* The same expert with 8-bit weights: W1q, W2q [E,D,F] and W3q [E,F,D] int8, S1, S2 [E,F] and
+ * S3 [E,D] fp32; X is bf16 (dtype 1) or fp32 (dtype 0). */
+void oracle_expert_ffn_w8(int64_t n_rec, const int32_t* rec_token, const int32_t* rec_expert,
+                          int64_t D, int64_t F, const void* X, int32_t x_dtype,
+                          const int8_t* W1q, const float* S1, const int8_t* W2q, const float* S2,
+                          const int8_t* W3q, const float* S3, int32_t act, double* Y) {
+  const wsrc w1 = {NULL, 0, W1q, S1}, w2 = {NULL, 0, W2q, S2}, w3 = {NULL, 0, W3q, S3};
+  expert_ffn_core(n_rec, rec_token, rec_expert, D, F, X, x_dtype, &w1, &w2, &w3, act, Y);
 }
 
 /* ---------------------------------------------------------------- combine  [G5] 5.3.5 */
@@ -384,13 +426,13 @@ double oracle_drop_rate(int64_t N, int32_t k, const uint8_t* dropped) {
  * record -> gate-weighted combine under the drop policy. out [N,D] doubles (before any
  * rounding to the output dtype). Every other output pointer is optional. Returns 0, or -1 on
  * a non-finite logit. */
-int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double cf,
-                   int64_t min_capacity, int32_t order, int32_t drop_policy,
-                   int32_t renorm, int32_t act, int32_t dtype, const void* X, const float* W_r,
-                   const float* bias, const void* W1, const void* W2, const void* W3,
-                   double* out, float* logits32_out, int32_t* idx_out, double* gate_out,
-                   int32_t* load_out, int32_t* offsets_out, int32_t* pos_out,
-                   uint8_t* dropped_out, double* prob_colsum_out) {
+static int forward_core(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double cf,
+                        int64_t min_capacity, int32_t order, int32_t drop_policy,
+                        int32_t renorm, int32_t act, int32_t dtype, const void* X,
+                        const float* W_r, const float* bias, const wsrc* W1, const wsrc* W2,
+                        const wsrc* W3, double* out, float* logits32_out, int32_t* idx_out,
+                        double* gate_out, int32_t* load_out, int32_t* offsets_out,
+                        int32_t* pos_out, uint8_t* dropped_out, double* prob_colsum_out) {
   const int64_t R = N * k;
   float* l32 = logits32_out ? logits32_out : (float*)malloc(sizeof(float) * (size_t)(N * E + 1));
   int32_t* idx = idx_out ? idx_out : (int32_t*)malloc(sizeof(int32_t) * (size_t)(R + 1));
@@ -420,7 +462,7 @@ int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double
       ++q;
     }
     double* Yk = (double*)malloc(sizeof(double) * (size_t)(nk * D + 1));
-    oracle_expert_ffn(nk, rt, re, D, F, X, W1, W2, W3, dtype, act, Yk);
+    expert_ffn_core(nk, rt, re, D, F, X, dtype, W1, W2, W3, act, Yk);
     double* Yrec = (double*)calloc((size_t)(R * D + 1), sizeof(double));
     q = 0;
     for (int64_t r = 0; r < R; ++r) {
@@ -442,6 +484,34 @@ int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double
   if (!pos_out) free(pos);
   if (!dropped_out) free(drp);
   return rc;
+}
+
+int oracle_forward(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double cf,
+                   int64_t min_capacity, int32_t order, int32_t drop_policy,
+                   int32_t renorm, int32_t act, int32_t dtype, const void* X, const float* W_r,
+                   const float* bias, const void* W1, const void* W2, const void* W3,
+                   double* out, float* logits32_out, int32_t* idx_out, double* gate_out,
+                   int32_t* load_out, int32_t* offsets_out, int32_t* pos_out,
+                   uint8_t* dropped_out, double* prob_colsum_out) {
+  const wsrc w1 = {W1, dtype, NULL, NULL}, w2 = {W2, dtype, NULL, NULL}, w3 = {W3, dtype, NULL, NULL};
+  return forward_core(N, D, F, E, k, cf, min_capacity, order, drop_policy, renorm, act, dtype, X,
+                      W_r, bias, &w1, &w2, &w3, out, logits32_out, idx_out, gate_out, load_out,
+                      offsets_out, pos_out, dropped_out, prob_colsum_out);
+}
+
+/* The forward with 8-bit expert weights (see oracle_expert_ffn_w8). */
+int oracle_forward_w8(int64_t N, int64_t D, int64_t F, int32_t E, int32_t k, double cf,
+                      int64_t min_capacity, int32_t order, int32_t drop_policy,
+                      int32_t renorm, int32_t act, int32_t dtype, const void* X,
+                      const float* W_r, const float* bias, const int8_t* W1q, const float* S1,
+                      const int8_t* W2q, const float* S2, const int8_t* W3q, const float* S3,
+                      double* out, float* logits32_out, int32_t* idx_out, double* gate_out,
+                      int32_t* load_out, int32_t* offsets_out, int32_t* pos_out,
+                      uint8_t* dropped_out, double* prob_colsum_out) {
+  const wsrc w1 = {NULL, 0, W1q, S1}, w2 = {NULL, 0, W2q, S2}, w3 = {NULL, 0, W3q, S3};
+  return forward_core(N, D, F, E, k, cf, min_capacity, order, drop_policy, renorm, act, dtype, X,
+                      W_r, bias, &w1, &w2, &w3, out, logits32_out, idx_out, gate_out, load_out,
+                      offsets_out, pos_out, dropped_out, prob_colsum_out);
 }
 
 int oracle_num_threads(void) {

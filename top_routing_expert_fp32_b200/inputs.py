@@ -96,6 +96,43 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed: Optional[int] = None,
     return MoEInputs(X, W_r, bias, W1, W2, W3)
 
 
+@dataclass
+class MoEWeights8:
+    W1q: torch.Tensor   # [E, D, F] int8 (activated branch)
+    S1: torch.Tensor    # [E, F] fp32, one scale per expert and output column
+    W2q: torch.Tensor   # [E, D, F] int8 (linear branch)
+    S2: torch.Tensor    # [E, F] fp32
+    W3q: torch.Tensor   # [E, F, D] int8 (down projection)
+    S3: torch.Tensor    # [E, D] fp32
+
+
+def _quantize_columns(w: torch.Tensor):
+    """Synthetic 8-bit weights: per output column, scale = max |w| / 127 and q = round(w /
+    scale) in [-127, 127]. Input synthesis only (the layer itself only dequantizes)."""
+    amax = w.abs().amax(dim=0)
+    scale = torch.where(amax > 0, amax / 127.0, torch.ones_like(amax))
+    q = torch.clamp(torch.round(w / scale), -127, 127).to(torch.int8)
+    return q, scale.to(torch.float32)
+
+
+def make_w8_weights(cfg: MoEConfig, device="cpu", seed: Optional[int] = None) -> MoEWeights8:
+    """8-bit expert weights of the same N(0, 1/fan_in) draws as make_inputs (same generators
+    and per-expert chunking), quantized per expert and output column."""
+    s = cfg.seed if seed is None else seed
+    device = torch.device(device)
+    out = []
+    for tid, (rows, cols, fan_in) in ((TID_W1, (cfg.D, cfg.F, cfg.D)), (TID_W2, (cfg.D, cfg.F, cfg.D)),
+                                      (TID_W3, (cfg.F, cfg.D, cfg.F))):
+        g = _gen(device, s, tid)
+        q = torch.empty((cfg.E, rows, cols), dtype=torch.int8, device=device)
+        sc = torch.empty((cfg.E, cols), dtype=torch.float32, device=device)
+        for e in range(cfg.E):
+            w = torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32)
+            q[e], sc[e] = _quantize_columns(w.mul_(1.0 / math.sqrt(fan_in)))
+        out += [q, sc]
+    return MoEWeights8(*out)
+
+
 def make_logits(N: int, E: int, device="cpu", seed: int = 0, std: float = 1.0) -> torch.Tensor:
     """Router logits drawn directly (fp32), for routing tests that start from logits."""
     return randn((N, E), std, torch.float32, device, seed, TID_LOGITS)
