@@ -45,12 +45,20 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_desc(cfg) -> str:
+def workload_desc(cfg, w8: bool = False) -> str:
     act = {0: "SiLU", 1: "GELU(erf)", 2: "GELU(tanh)"}[cfg.activation]
     s = (f"{cfg.name}: N={cfg.N} D={cfg.D} F={cfg.F} E={cfg.E} k={cfg.k} {act} "
          f"{'renormalised' if cfg.renormalize else 'no-renorm'} top-k")
     if cfg.capacity_factor > 0:
         s += f", CF={cfg.capacity_factor}"
+    if cfg.min_capacity > 0:
+        s += f", min_capacity={cfg.min_capacity}"
+    if cfg.capacity_order == 1:
+        s += ", token-major slots"
+    if cfg.drop_policy == 1:
+        s += ", kept gates renormalised on drops"
+    if w8:
+        s += ", 8-bit expert weights (fp32 scale per expert and output column)"
     return s
 
 
@@ -182,7 +190,7 @@ def traffic_from_profile(kernel: str, workload: str):
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def oracle_tokens_per_s(cfg, budget_s: float = 12.0):
+def oracle_tokens_per_s(cfg, budget_s: float = 12.0, w8: bool = False):
     """The oracle (as it stands) on a bounded token sample of the workload. Without capacity the
     tokens are independent, so a prefix of the batch is the same computation per token; with
     capacity the sample is its own batch of n tokens (capacity recomputed for n)."""
@@ -191,19 +199,26 @@ def oracle_tokens_per_s(cfg, budget_s: float = 12.0):
     import oracle
     from top_routing_expert_fp32_b200 import configs, inputs
 
-    inp = inputs.make_inputs(cfg, "cpu")
+    inp = inputs.make_inputs(cfg, "cpu", weights=not w8)
     od = oracle.BF16 if cfg.dtype == configs.DTYPE_BF16 else oracle.F32
     X = oracle.torch_to_numpy(inp.X)
     Wr = inp.W_r.numpy()
     b = None if inp.bias is None else inp.bias.numpy()
-    W1, W2, W3 = (oracle.torch_to_numpy(w) for w in (inp.W1, inp.W2, inp.W3))
+    opts = dict(k=cfg.k, cf=cfg.capacity_factor, renorm=cfg.renormalize, act=cfg.activation,
+                dtype=od, min_capacity=cfg.min_capacity, order=cfg.capacity_order,
+                drop_policy=cfg.drop_policy)
+    if w8:
+        q = inputs.make_w8_weights(cfg, "cpu")
+        qs = [t.numpy() for t in (q.W1q, q.S1, q.W2q, q.S2, q.W3q, q.S3)]
+    else:
+        W1, W2, W3 = (oracle.torch_to_numpy(w) for w in (inp.W1, inp.W2, inp.W3))
 
     def run(n):
         t = time.perf_counter()
-        oracle.forward(X[:n], Wr, b, W1, W2, W3, k=cfg.k, cf=cfg.capacity_factor,
-                       renorm=cfg.renormalize, act=cfg.activation, dtype=od,
-                       min_capacity=cfg.min_capacity, order=cfg.capacity_order,
-                       drop_policy=cfg.drop_policy)
+        if w8:
+            oracle.forward_w8(X[:n], Wr, b, *qs, **opts)
+        else:
+            oracle.forward(X[:n], Wr, b, W1, W2, W3, **opts)
         return time.perf_counter() - t
 
     n = min(cfg.N, max(1, oracle.num_threads()))
@@ -227,7 +242,9 @@ def run_gpu(args, cfg, world, rank, device):
 
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
-    inp = inputs.make_inputs(cfg, device, seed=cfg.seed + rank * 0)
+    w8 = args.weights == "w8"
+    inp = inputs.make_inputs(cfg, device, seed=cfg.seed + rank * 0, weights=not w8)
+    wq = inputs.make_w8_weights(cfg, device) if w8 else None
     N, E, k, D, F = cfg.N, cfg.E, cfg.k, cfg.D, cfg.F
     p = abi.problem(cfg)
     ws = abi.workspace(p, device)
@@ -267,9 +284,15 @@ def run_gpu(args, cfg, world, rank, device):
         ev[1].record(stream)
         abi.dispatch(p, inp.X, idx, load, offsets, pos, dropped, row_token, X_perm, ws)
         ev[2].record(stream)
-        abi.expert_up(p, X_perm, offsets, inp.W1, inp.W2, H, ws)
+        if w8:
+            abi.expert_up_w8(p, X_perm, offsets, wq.W1q, wq.S1, wq.W2q, wq.S2, H, ws)
+        else:
+            abi.expert_up(p, X_perm, offsets, inp.W1, inp.W2, H, ws)
         ev[3].record(stream)
-        abi.expert_down(p, H, offsets, inp.W3, Y, ws)
+        if w8:
+            abi.expert_down_w8(p, H, offsets, wq.W3q, wq.S3, Y, ws)
+        else:
+            abi.expert_down(p, H, offsets, inp.W3, Y, ws)
         ev[4].record(stream)
         abi.combine(p, Y, idx, gate, offsets, pos, dropped, out)
         ev[5].record(stream)
@@ -337,37 +360,55 @@ def run_gpu(args, cfg, world, rank, device):
     # algorithmic bytes at the HBM peak (A rows read once, the weights of every expert that
     # keeps a row read once, H written once).
     used = int((offsets[1:] - offsets[:-1] > 0).sum().item())
-    bytes_up = kept * D * es + used * 2.0 * D * F * es + kept * F * es
+    # 8-bit weights: one byte per weight plus the fp32 column scales.
+    ew = 1 if w8 else es
+    bytes_up = kept * D * es + used * 2.0 * (D * F * ew + (F * 4 if w8 else 0)) + kept * F * es
     t_tensor = flops_up / (tc * 1e12) if cfg.dtype == configs.DTYPE_BF16 else 0.0
     t_hbm = bytes_up / (hbm * 1e9)
     dom = "up"
     psrc = (f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback")
     if t_tensor >= t_hbm:
-        roof = {"kernel": "grouped_gemm_sm100<dual> (expert up-projection + gating)",
+        roof = {"kernel": ("grouped_gemm_w8<dual>" if w8 else "grouped_gemm_sm100<dual>")
+                + " (expert up-projection + gating)",
                 "bound": "tensor", "achieved": kern["up"]["TFLOP/s"], "peak": tc,
                 "unit": "TFLOP/s", "frac": kern["up"]["TFLOP/s"] / tc,
                 "peak_source": psrc + ", bf16 burst", "flops_per_launch": flops_up}
     else:
         gbs = bytes_up / mean["up"] / 1e6
-        roof = {"kernel": "expert up-projection (bound by streaming the used experts' weights)",
+        roof = {"kernel": ("grouped_gemm_w8<dual>" if w8 else "grouped_gemm_sm100<dual>")
+                + " (expert up-projection; bound by streaming the used experts' weights)",
                 "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                 "frac": gbs / hbm, "peak_source": psrc, "bytes_per_launch": bytes_up}
     roof["min_us"] = {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6}
     roof["experts_used"] = used
     # Same two-sided bound for both GEMMs: frac_roofline = bound time / measured time.
-    bytes_down = kept * F * es + used * 1.0 * D * F * es + kept * D * es
+    bytes_down = kept * F * es + used * (D * F * ew + (D * 4 if w8 else 0)) + kept * D * es
     for n, fl, by in (("up", flops_up, bytes_up), ("down", flops_down, bytes_down)):
         t_min = max(fl / (tc * 1e12) if cfg.dtype == configs.DTYPE_BF16 else 0.0,
                     by / (hbm * 1e9))
         kern[n]["frac_roofline"] = t_min * 1e3 / mean[n]
-    roof["traffic"] = traffic_from_profile("up", cfg.name)
+    roof["traffic"] = traffic_from_profile("up_w8" if w8 else "up", cfg.name)
 
-    # end-to-end through the public host-buffer entry point
+    # end-to-end through the public entry points, host X in and host out inside the timed
+    # region: moe_forward_host (bf16 weights; it copies and synchronises itself) or, for 8-bit
+    # weights, pinned-host copies around moe_forward_w8.
     ws_h = abi.workspace(p, device, host=True)
     xh = inp.X.cpu().pin_memory()
     oh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(inp.X)
+    od = torch.empty_like(inp.X)
+
+    def e2e_call():
+        if w8:
+            xd.copy_(xh, non_blocking=True)
+            abi.forward_w8(p, xd, inp.W_r, inp.bias, wq, od, ws)
+            oh.copy_(od, non_blocking=True)
+        else:
+            abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
+
     for _ in range(2):
-        abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
+        e2e_call()
+    torch.cuda.synchronize(device)
     barrier(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -375,7 +416,7 @@ def run_gpu(args, cfg, world, rank, device):
     for _ in range(args.steps):
         flush_l2()
         e0.record(stream)
-        abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
+        e2e_call()
         e1.record(stream)
         e1.synchronize()
         e_total += e0.elapsed_time(e1)
@@ -392,7 +433,9 @@ def run_gpu(args, cfg, world, rank, device):
         "dtype": dtype_name(cfg),
         "data": "synthetic, seeded: X~N(0,1), W_r/W1/W2~N(0,1/D), W3~N(0,1/F)"
                 + (", bias~N(0,2)" if cfg.router_bias_var > 0 else ""),
-        "config": {"workload": workload_desc(cfg), "tokens_per_gpu": N,
+        "config": {"workload": workload_desc(cfg, w8), "tokens_per_gpu": N,
+                   "expert_weights": "int8 + fp32 scale per expert and output column" if w8
+                   else dtype_name(cfg),
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "flushed between steps (512 MiB write + read-back, outside the step events)",
                    "kept_records": kept,
@@ -402,7 +445,9 @@ def run_gpu(args, cfg, world, rank, device):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "api": "moe_forward_host (pinned host X in, host out; copies in the timed region)"},
+                "api": ("moe_forward_w8 between pinned-host copies of X and out" if w8 else
+                        "moe_forward_host (pinned host X in, host out)")
+                       + "; copies in the timed region"},
         "gpu_launches": sum(launches.values()) * args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
@@ -422,6 +467,8 @@ def main():
                     help="override N (smaller cases for profiling)")
     ap.add_argument("--ffn", type=int, default=None,
                     help="override F (smaller weight footprint for profiling)")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "w8"],
+                    help="expert weights: bf16, or int8 with per-column fp32 scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -437,13 +484,14 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = oracle_tokens_per_s(cfg, budget_s=min(20.0, 6.0 * args.steps))
+        cb = oracle_tokens_per_s(cfg, budget_s=min(20.0, 6.0 * args.steps),
+                                 w8=args.weights == "w8")
         line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * cfg.N / cb["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic, seeded (same inputs as the GPU arm)",
-                "config": {"workload": workload_desc(cfg)},
+                "config": {"workload": workload_desc(cfg, args.weights == "w8")},
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -460,7 +508,7 @@ def main():
     line = run_gpu(args, cfg, world, rank, device)
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = oracle_tokens_per_s(cfg)
+            line["cpu_baseline"] = oracle_tokens_per_s(cfg, w8=args.weights == "w8")
         else:
             line["cpu_baseline"] = None
         print(json.dumps(line))

@@ -229,6 +229,29 @@ moe_status moe_forward(const moe_problem* p, const void* X, const float* W_r, co
                        int32_t* pos, uint8_t* dropped, float* prob_colsum, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* ---- 8-bit expert weights (Grok-1 book 5.3.3 and 5.3.5: weight = weight * scales before
+ * each expert matmul). Layouts as the bf16 weights, stored as int8: W1q, W2q [E,D,F], W3q
+ * [E,F,D]; one fp32 scale per expert and output column: S1, S2 [E,F], S3 [E,D]; the expert
+ * uses W[e][k][n] = Wq[e][k][n] * S[e][n]. Activations (X, X_perm, H, Y, out) are bf16
+ * (p->dtype must be MOE_DTYPE_BF16) and D, F must be multiples of 16, else
+ * MOE_ERR_UNSUPPORTED. The tensor cores multiply bf16 activations by the exact bf16 value of q
+ * with fp32 accumulation and the scale is applied to the fp32 sum (x.(q s) = s (x.q) for a
+ * per-column s), so the weights cross HBM as int8. Pointers: device memory, 16-byte aligned.
+ * Same results rules, workspace and error behaviour as the bf16 entry points. */
+moe_status moe_expert_up_w8(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                            const int8_t* W1q, const float* S1, const int8_t* W2q,
+                            const float* S2, void* H, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_expert_down_w8(const moe_problem* p, const void* H, const int32_t* offsets,
+                              const int8_t* W3q, const float* S3, void* Y, void* ws,
+                              size_t ws_bytes, void* stream);
+/* moe_forward with 8-bit expert weights (router, dispatch and combine unchanged). */
+moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
+                          const float* bias, const int8_t* W1q, const float* S1,
+                          const int8_t* W2q, const float* S2, const int8_t* W3q, const float* S3,
+                          void* out, float* logits, int32_t* topk_idx, float* topk_gate,
+                          int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                          float* prob_colsum, void* ws, size_t ws_bytes, void* stream);
+
 /* moe_forward with HOST activations: X_host [N,D] and out_host [N,D] are host pointers
  * (page-locked memory gives asynchronous copies), the weights and W_r/bias are device
  * pointers. Enqueues the host->device copy of X, the forward, and the device->host copy

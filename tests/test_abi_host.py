@@ -153,3 +153,19 @@ def test_null_and_misaligned_pointers_rejected(abi):
     st = abi.lib.moe_forward(ctypes.byref(p), 4096, 4096, None, None, 4096, 4096, 4096,
                              *([None] * 8), 4096, need, None)
     assert st == abi.MOE_ERR_INVALID_ARG and b"W1" in abi.lib.moe_last_error()
+
+
+def test_w8_entry_points_reject_unsupported_shapes_on_host(abi):
+    # 8-bit expert weights need bf16 activations and D, F multiples of 16; the check runs on
+    # the host before anything is enqueued.
+    from top_routing_expert_fp32_b200 import configs
+    for dtype, D in ((configs.DTYPE_F32, 64), (configs.DTYPE_BF16, 24)):
+        cfg = configs.MoEConfig("w8", N=8, D=D, F=64, E=4, k=1, dtype=dtype, activation=0,
+                                renormalize=1)
+        p = abi.problem(cfg)
+        st = abi.lib.moe_expert_up_w8(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, 256, 1 << 20,
+                                      None)
+        assert st == 2, abi.lib.moe_last_error()
+        st = abi.lib.moe_forward_w8(ctypes.byref(p), *([16] * 10), *([None] * 8), 256, 1 << 20,
+                                    None)
+        assert st == 2

@@ -1,0 +1,156 @@
+"""GPU parity of the 8-bit expert-weight path (moe_expert_up_w8 / moe_expert_down_w8 /
+moe_forward_w8) against the oracle's fp64 dequantized experts (W = q * s per expert and output
+column; Grok-1 book 5.3.3, 5.3.5)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from top_routing_expert_fp32_b200 import configs, inputs
+from gpu_helpers import NEAR_TIE, TOL_BF16, normwise_rel_err, np_host, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from top_routing_expert_fp32_b200 import abi as a
+    return a
+
+
+def _cfg(N, D, F, E, k=1, act=configs.ACT_SILU, **kw):
+    return configs.MoEConfig("w8", N=N, D=D, F=F, E=E, k=k, dtype=configs.DTYPE_BF16,
+                             activation=act, renormalize=1, **kw)
+
+
+def _ffn_w8(abi, counts, D, F, act, seed=0):
+    E = len(counts)
+    R = int(sum(counts))
+    cfg = _cfg(max(R, 1), D, F, E, act=act)
+    Xp = inputs.randn((max(R, 1), D), 1.0, torch.bfloat16, "cuda", seed, 1)
+    w = inputs.make_w8_weights(cfg, "cuda", seed)
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32,
+                           device="cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    H = torch.full((max(R, 1), F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Y = torch.full((max(R, 1), D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    abi.expert_up_w8(p, Xp, offsets, w.W1q, w.S1, w.W2q, w.S2, H, ws)
+    abi.expert_down_w8(p, H, offsets, w.W3q, w.S3, Y, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    return cfg, Xp, w, offsets, H, Y, R
+
+
+@pytest.mark.parametrize("counts,D,F,act", [
+    ([128], 64, 256, configs.ACT_SILU),
+    ([0, 1, 300], 128, 256, configs.ACT_SILU),
+    ([129, 127, 128, 0, 5, 256, 1, 64], 256, 384, configs.ACT_GELU_ERF),
+    ([70, 0, 33], 80, 208, configs.ACT_GELU_TANH),
+    ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
+    ([700, 0, 257, 1100], 512, 400, configs.ACT_GELU_ERF),
+])
+def test_expert_ffn_w8_matches_oracle(abi, counts, D, F, act):
+    cfg, Xp, w, offsets, H, Y, R = _ffn_w8(abi, counts, D, F, act)
+    rec_e = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
+    ref = oracle.expert_ffn_w8(np.arange(R, dtype=np.int32), rec_e, np_host(Xp), oracle.BF16,
+                               w.W1q.cpu().numpy(), w.S1.cpu().numpy(), w.W2q.cpu().numpy(),
+                               w.S2.cpu().numpy(), w.W3q.cpu().numpy(), w.S3.cpu().numpy(), act)
+    err = normwise_rel_err(to_f64(Y[:R]), ref)
+    assert err.max() <= TOL_BF16, f"max normwise rel err {err.max():.3g}"
+
+
+def test_unit_scales_reproduce_bf16_kernel_bit_for_bit(abi, monkeypatch):
+    # int8 -> bf16 is exact and a unit scale is exact, so with the same 128-row tiles the 8-bit
+    # path must give the bf16 path's bits on W = q.
+    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", "128")
+    counts, D, F = [129, 3, 200, 64], 256, 384
+    cfg, Xp, w, offsets, H8, Y8, R = _ffn_w8(abi, counts, D, F, configs.ACT_SILU, seed=4)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    one = lambda s: torch.ones_like(s)
+    H1 = torch.empty_like(H8)
+    Y1 = torch.empty_like(Y8)
+    abi.expert_up_w8(p, Xp, offsets, w.W1q, one(w.S1), w.W2q, one(w.S2), H1, ws)
+    abi.expert_down_w8(p, H1, offsets, w.W3q, one(w.S3), Y1, ws)
+    W1, W2, W3 = (q.to(torch.bfloat16) for q in (w.W1q, w.W2q, w.W3q))
+    Hb = torch.empty_like(H8)
+    Yb = torch.empty_like(Y8)
+    abi.expert_up(p, Xp, offsets, W1, W2, Hb, ws)
+    abi.expert_down(p, Hb, offsets, W3, Yb, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(H1[:R].view(torch.int16), Hb[:R].view(torch.int16))
+    assert torch.equal(Y1[:R].view(torch.int16), Yb[:R].view(torch.int16))
+
+
+def test_w8_rejected_without_bf16_or_16_multiples(abi):
+    from top_routing_expert_fp32_b200.abi import MoEError
+    cfg = _cfg(64, 24, 64, 4)           # D % 16 != 0
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    t = torch.zeros(16, dtype=torch.int8, device="cuda")
+    f = torch.zeros(16, dtype=torch.float32, device="cuda")
+    with pytest.raises(MoEError):
+        abi.expert_up_w8(p, f, t, t, f, t, f, f, ws)
+
+
+def _forward_w8_check(abi, cfg, sample=None):
+    inp = inputs.make_inputs(cfg, "cuda", weights=False)
+    w = inputs.make_w8_weights(cfg, "cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    N, E, k = cfg.N, cfg.E, cfg.k
+    idx = torch.empty((N, k), dtype=torch.int32, device="cuda")
+    dropped = torch.empty((N, k), dtype=torch.uint8, device="cuda")
+    out = torch.empty((N, cfg.D), dtype=torch.bfloat16, device="cuda")
+    abi.forward_w8(p, inp.X, inp.W_r, inp.bias, w, out, ws, topk_idx=idx, dropped=dropped)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    Xn = np_host(inp.X)
+    l64, l32 = oracle.router_logits(Xn, oracle.BF16, inp.W_r.cpu().numpy(),
+                                    None if inp.bias is None else inp.bias.cpu().numpy())
+    ro = oracle.route(l32, k=k, renorm=cfg.renormalize)
+    flips = (idx.cpu().numpy() != ro["idx"]).any(1)
+    assert (oracle.topk_margin(l64, k)[flips] < NEAR_TIE).all()
+    C = oracle.capacity(N, k, E, cfg.capacity_factor, cfg.min_capacity)
+    do = oracle.dispatch(ro["idx"], E, C, order=cfg.capacity_order)
+    toks = np.arange(N) if sample is None else np.asarray(sample)
+    toks = toks[~flips[toks] & (dropped.cpu().numpy()[toks] == do["dropped"][toks]).all(1)]
+    rec_t, rec_e, slot = [], [], []
+    for t in toks:
+        for j in range(k):
+            if not do["dropped"][t, j]:
+                rec_t.append(t)
+                rec_e.append(ro["idx"][t, j])
+                slot.append((t, j))
+    Y = oracle.expert_ffn_w8(np.array(rec_t, np.int32), np.array(rec_e, np.int32), Xn,
+                             oracle.BF16, w.W1q.cpu().numpy(), w.S1.cpu().numpy(),
+                             w.W2q.cpu().numpy(), w.S2.cpu().numpy(), w.W3q.cpu().numpy(),
+                             w.S3.cpu().numpy(), cfg.activation)
+    ref = np.zeros((len(toks), cfg.D))
+    row = {t: i for i, t in enumerate(toks)}
+    for (t, j), y in zip(slot, Y):
+        ref[row[t]] += ro["gate"][t, j] * y
+    err = normwise_rel_err(to_f64(out)[toks], ref)
+    assert err.max() <= TOL_BF16, f"max normwise rel err {err.max():.3g}"
+    return len(toks), int(flips.sum())
+
+
+@pytest.mark.parametrize("cfg", [
+    _cfg(300, 256, 512, 8, k=2),
+    _cfg(500, 128, 256, 16, k=2, capacity_factor=1.0, router_bias_var=2.0),
+    _cfg(257, 384, 640, 8, k=2, act=configs.ACT_GELU_ERF).with_(renormalize=0),
+], ids=["silu_e8", "capacity_e16", "gelu_norenorm"])
+def test_forward_w8_small_all_tokens(abi, cfg):
+    n, flips = _forward_w8_check(abi, cfg)
+    assert n >= cfg.N - 2 * flips - 8
+
+
+@pytest.mark.parametrize("name", ["decode", "mixtral"])
+def test_forward_w8_full_size_sampled(abi, name):
+    cfg = configs.CONFIGS[name]
+    sample = sorted(set(np.linspace(0, cfg.N - 1, 12).astype(int).tolist()))
+    _forward_w8_check(abi, cfg, sample)
+    torch.cuda.empty_cache()

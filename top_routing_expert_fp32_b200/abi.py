@@ -63,6 +63,9 @@ def _load() -> ctypes.CDLL:
         "moe_combine": [PP, P, P, P, P, P, P, P, P],
         "moe_forward": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "moe_forward_host": [PP, P, P, P, P, P, P, P, P, S, P],
+        "moe_expert_up_w8": [PP, P, P, P, P, P, P, P, P, S, P],
+        "moe_expert_down_w8": [PP, P, P, P, P, P, P, S, P],
+        "moe_forward_w8": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "moe_workspace_init": [P, S, P],
         "moe_get_device_error": [P, P, ctypes.POINTER(ctypes.c_int32)],
     }
@@ -176,6 +179,27 @@ def forward(p, X, W_r, bias, W1, W2, W3, out, ws, *, logits=None, topk_idx=None,
                            _ptr(W3), _ptr(out), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
                            _ptr(load), _ptr(offsets), _ptr(pos), _ptr(dropped),
                            _ptr(prob_colsum), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def expert_up_w8(p, X_perm, offsets, W1q, S1, W2q, S2, H, ws, stream=None):
+    _check(lib.moe_expert_up_w8(ctypes.byref(p), _ptr(X_perm), _ptr(offsets), _ptr(W1q), _ptr(S1),
+                                _ptr(W2q), _ptr(S2), _ptr(H), _ptr(ws), ws.numel(),
+                                _stream(stream)))
+
+
+def expert_down_w8(p, H, offsets, W3q, S3, Y, ws, stream=None):
+    _check(lib.moe_expert_down_w8(ctypes.byref(p), _ptr(H), _ptr(offsets), _ptr(W3q), _ptr(S3),
+                                  _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def forward_w8(p, X, W_r, bias, w8, out, ws, *, logits=None, topk_idx=None, topk_gate=None,
+               load=None, offsets=None, pos=None, dropped=None, prob_colsum=None, stream=None):
+    """w8: an object with W1q, S1, W2q, S2, W3q, S3 (e.g. inputs.MoEWeights8)."""
+    _check(lib.moe_forward_w8(ctypes.byref(p), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(w8.W1q),
+                              _ptr(w8.S1), _ptr(w8.W2q), _ptr(w8.S2), _ptr(w8.W3q), _ptr(w8.S3),
+                              _ptr(out), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
+                              _ptr(load), _ptr(offsets), _ptr(pos), _ptr(dropped),
+                              _ptr(prob_colsum), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def forward_host(p, X_host: torch.Tensor, W_r, bias, W1, W2, W3, out_host: torch.Tensor, ws,

@@ -217,15 +217,47 @@ moe_status run_down(const moe_problem& p, const void* H, const int32_t* offsets,
   return MOE_OK;
 }
 
+// Expert weights: bf16/fp32 (W1..W3) or 8-bit with per-column scales (Q1..Q3, S1..S3).
+struct Experts {
+  const void* W1 = nullptr;
+  const void* W2 = nullptr;
+  const void* W3 = nullptr;
+  const int8_t* Q1 = nullptr;
+  const int8_t* Q2 = nullptr;
+  const int8_t* Q3 = nullptr;
+  const float* S1 = nullptr;
+  const float* S2 = nullptr;
+  const float* S3 = nullptr;
+  bool w8() const { return Q1 != nullptr; }
+};
+
 moe_status run_ffn(const moe_problem& p, const void* X_perm, const int32_t* offsets,
-                   const void* W1, const void* W2, const void* W3, void* H, void* Y, int* err,
-                   cudaStream_t stream) {
-  MOE_TRY(run_up(p, X_perm, offsets, W1, W2, H, err, stream));
-  return run_down(p, H, offsets, W3, Y, err, stream);
+                   const Experts& w, void* H, void* Y, int* err, cudaStream_t stream) {
+  if (!w.w8()) {
+    MOE_TRY(run_up(p, X_perm, offsets, w.W1, w.W2, H, err, stream));
+    return run_down(p, H, offsets, w.W3, Y, err, stream);
+  }
+  MOE_TRY(check_sm100());
+  MOE_CUDA(launch_ffn_up_w8(p, X_perm, offsets, w.Q1, w.S1, w.Q2, w.S2, H, err,
+                            wait_timeout_ns(), stream),
+           "expert up-projection, 8-bit weights (tcgen05)");
+  MOE_CUDA(launch_ffn_down_w8(p, H, offsets, w.Q3, w.S3, Y, err, wait_timeout_ns(), stream),
+           "expert down-projection, 8-bit weights (tcgen05)");
+  return MOE_OK;
+}
+
+// Extra shape rule of the 8-bit expert path: bf16 activations, and D, F multiples of 16
+// (16-byte rows of int8 weights for the tensor-memory copies).
+moe_status check_w8(const moe_problem& p) {
+  if (p.dtype != MOE_DTYPE_BF16)
+    return fail(MOE_ERR_UNSUPPORTED, "8-bit expert weights need bf16 activations");
+  if (p.D % 16 != 0 || p.F % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "8-bit expert weights need D and F multiples of 16");
+  return MOE_OK;
 }
 
 moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, const float* bias,
-                        const void* W1, const void* W2, const void* W3, void* out, float* logits,
+                        const Experts& w, void* out, float* logits,
                         int32_t* topk_idx, float* topk_gate, int32_t* load, int32_t* offsets,
                         int32_t* pos, uint8_t* dropped, float* prob_colsum, void* ws,
                         cudaStream_t stream) {
@@ -256,7 +288,7 @@ moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, c
                               row_token, err, stream),
            "slot assign");
   MOE_CUDA(launch_gather(p, X, row_token, off, xperm, err, stream), "gather");
-  MOE_TRY(run_ffn(p, xperm, off, W1, W2, W3, h, y, err, stream));
+  MOE_TRY(run_ffn(p, xperm, off, w, h, y, err, stream));
   MOE_CUDA(launch_combine(p, y, idx, gate, off, ps, dr, out, err, stream), "combine");
   return MOE_OK;
 }
@@ -359,7 +391,11 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* X_perm, const int32_
   MOE_TRY(need(Y, "Y"));
   if (p->N == 0) return MOE_OK;
   const Layout L = make_layout(*p);
-  return run_ffn(*p, X_perm, offsets, W1, W2, W3, H, Y, at<int>(ws, L.err),
+  Experts w;
+  w.W1 = W1;
+  w.W2 = W2;
+  w.W3 = W3;
+  return run_ffn(*p, X_perm, offsets, w, H, Y, at<int>(ws, L.err),
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -431,7 +467,11 @@ moe_status moe_forward(const moe_problem* p, const void* X, const float* W_r, co
   MOE_TRY(opt(pos, "pos", 4));
   MOE_TRY(opt(dropped, "dropped", 1));
   MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
-  return forward_impl(*p, X, W_r, bias, W1, W2, W3, out, logits, topk_idx, topk_gate, load,
+  Experts w;
+  w.W1 = W1;
+  w.W2 = W2;
+  w.W3 = W3;
+  return forward_impl(*p, X, W_r, bias, w, out, logits, topk_idx, topk_gate, load,
                       offsets, pos, dropped, prob_colsum, ws, static_cast<cudaStream_t>(stream));
 }
 
@@ -455,11 +495,95 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
   void* xin = at<void>(ws, L.xin);
   void* xout = at<void>(ws, L.xout);
   if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(xin, X_host, bytes, cudaMemcpyHostToDevice, s), "H2D");
-  MOE_TRY(forward_impl(*p, xin, W_r, bias, W1, W2, W3, xout, nullptr, nullptr, nullptr, nullptr,
+  Experts w;
+  w.W1 = W1;
+  w.W2 = W2;
+  w.W3 = W3;
+  MOE_TRY(forward_impl(*p, xin, W_r, bias, w, xout, nullptr, nullptr, nullptr, nullptr,
                        nullptr, nullptr, nullptr, nullptr, ws, s));
   if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, s), "D2H");
   MOE_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   return MOE_OK;
+}
+
+moe_status moe_expert_up_w8(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                            const int8_t* W1q, const float* S1, const int8_t* W2q,
+                            const float* S2, void* H, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_w8(*p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X_perm, "X_perm"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W1q, "W1q"));
+  MOE_TRY(need(S1, "S1"));
+  MOE_TRY(need(W2q, "W2q"));
+  MOE_TRY(need(S2, "S2"));
+  MOE_TRY(need(H, "H"));
+  if (p->N == 0) return MOE_OK;
+  MOE_TRY(check_sm100());
+  const Layout L = make_layout(*p);
+  MOE_CUDA(launch_ffn_up_w8(*p, X_perm, offsets, W1q, S1, W2q, S2, H, at<int>(ws, L.err),
+                            wait_timeout_ns(), static_cast<cudaStream_t>(stream)),
+           "expert up-projection, 8-bit weights (tcgen05)");
+  return MOE_OK;
+}
+
+moe_status moe_expert_down_w8(const moe_problem* p, const void* H, const int32_t* offsets,
+                              const int8_t* W3q, const float* S3, void* Y, void* ws,
+                              size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_w8(*p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(H, "H"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W3q, "W3q"));
+  MOE_TRY(need(S3, "S3"));
+  MOE_TRY(need(Y, "Y"));
+  if (p->N == 0) return MOE_OK;
+  MOE_TRY(check_sm100());
+  const Layout L = make_layout(*p);
+  MOE_CUDA(launch_ffn_down_w8(*p, H, offsets, W3q, S3, Y, at<int>(ws, L.err), wait_timeout_ns(),
+                              static_cast<cudaStream_t>(stream)),
+           "expert down-projection, 8-bit weights (tcgen05)");
+  return MOE_OK;
+}
+
+moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
+                          const float* bias, const int8_t* W1q, const float* S1,
+                          const int8_t* W2q, const float* S2, const int8_t* W3q, const float* S3,
+                          void* out, float* logits, int32_t* topk_idx, float* topk_gate,
+                          int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                          float* prob_colsum, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_w8(*p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X, "X"));
+  MOE_TRY(need(W_r, "W_r"));
+  MOE_TRY(opt(bias, "bias", 4));
+  MOE_TRY(need(W1q, "W1q"));
+  MOE_TRY(need(S1, "S1"));
+  MOE_TRY(need(W2q, "W2q"));
+  MOE_TRY(need(S2, "S2"));
+  MOE_TRY(need(W3q, "W3q"));
+  MOE_TRY(need(S3, "S3"));
+  MOE_TRY(need(out, "out"));
+  MOE_TRY(opt(logits, "logits", 4));
+  MOE_TRY(opt(topk_idx, "topk_idx", 4));
+  MOE_TRY(opt(topk_gate, "topk_gate", 4));
+  MOE_TRY(opt(load, "load", 4));
+  MOE_TRY(opt(offsets, "offsets", 4));
+  MOE_TRY(opt(pos, "pos", 4));
+  MOE_TRY(opt(dropped, "dropped", 1));
+  MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
+  Experts w;
+  w.Q1 = W1q;
+  w.Q2 = W2q;
+  w.Q3 = W3q;
+  w.S1 = S1;
+  w.S2 = S2;
+  w.S3 = S3;
+  return forward_impl(*p, X, W_r, bias, w, out, logits, topk_idx, topk_gate, load, offsets, pos,
+                      dropped, prob_colsum, ws, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {

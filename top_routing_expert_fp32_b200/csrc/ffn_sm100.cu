@@ -539,6 +539,19 @@ bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t cols, uin
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tensor_map_3d_u8(CUtensorMap* m, const void* ptr, uint64_t n, uint64_t k, uint64_t E,
+                           uint32_t box_n, uint32_t box_k) {
+  if (encode_fn() == nullptr) return false;
+  const cuuint64_t dims[3] = {n, k, E};
+  const cuuint64_t strides[2] = {n, n * k};
+  const cuuint32_t box[3] = {box_n, box_k, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
                                 const void* W1, const void* W2, void* H, int* err,
                                 uint64_t timeout_ns, cudaStream_t stream) {

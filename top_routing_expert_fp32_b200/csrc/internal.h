@@ -40,6 +40,21 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
 bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
                              uint32_t box_cols, uint32_t box_rows);
 
+// 3-D uint8 tensor map over stacked [E][k][n] bytes (n contiguous), box box_n x box_k x 1,
+// 128-byte swizzle (box_n must be 128).
+bool make_tensor_map_3d_u8(CUtensorMap* m, const void* ptr, uint64_t n, uint64_t k, uint64_t E,
+                           uint32_t box_n, uint32_t box_k);
+
+// Grouped expert GEMMs with 8-bit weights (W = q * s, s per expert and output column),
+// bf16 activations, tcgen05 tensor cores; 128-row tiles on single CTAs.
+cudaError_t launch_ffn_up_w8(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                             const int8_t* W1q, const float* S1, const int8_t* W2q,
+                             const float* S2, void* H, int* err, uint64_t timeout_ns,
+                             cudaStream_t stream);
+cudaError_t launch_ffn_down_w8(const moe_problem& p, const void* H, const int32_t* offsets,
+                               const int8_t* W3q, const float* S3, void* Y, int* err,
+                               uint64_t timeout_ns, cudaStream_t stream);
+
 // Records are processed in chunks of this many for the slot assignment.
 constexpr int kDispatchChunk = 1024;
 
