@@ -55,6 +55,8 @@ def lib():
         L.oracle_router_logits.restype = None
         L.oracle_route.argtypes = [i64, i32, i32, i32, P, P, P, P, P]
         L.oracle_route.restype = ctypes.c_int
+        L.oracle_route_ex.argtypes = [i64, i32, i32, i32, i32, P, P, P, P, P, P, P]
+        L.oracle_route_ex.restype = ctypes.c_int
         L.oracle_topk_margin.argtypes = [i64, i32, i32, P, P]
         L.oracle_topk_margin.restype = None
         L.oracle_dispatch.argtypes = [i64, i32, i32, i64, P, P, P, P, P, P]
@@ -144,6 +146,29 @@ def route(logits32: np.ndarray, k: int, renorm: int, want_probs: bool = False):
     if rc != 0:
         raise ValueError("oracle_route: non-finite logits")
     return dict(idx=idx, gate=gate, colsum=colsum, probs=probs)
+
+
+# Routing modes (training-time variants of the selection).
+ROUTE_TOPK, ROUTE_NOISY_TOPK, ROUTE_GSHARD_RANDOM = 0, 1, 2
+
+
+def route_ex(logits32: np.ndarray, k: int, renorm: int, mode: int = ROUTE_TOPK, noise=None,
+             want_probs: bool = False):
+    """route() with the training-time variants and the z-loss. Returns dict(idx, gate, colsum,
+    probs, zloss) where zloss = mean over tokens of (log sum exp logits)^2."""
+    logits32 = _c(logits32, np.float32)
+    N, E = logits32.shape
+    nz = None if noise is None else _c(noise, np.float32)
+    idx = np.empty((N, k), np.int32)
+    gate = np.empty((N, k), np.float64)
+    colsum = np.empty((E,), np.float64)
+    probs = np.empty((N, E), np.float64) if want_probs else None
+    z = np.zeros((1,), np.float64)
+    rc = lib().oracle_route_ex(N, E, k, renorm, mode, _p(logits32), _p(nz), _p(idx), _p(gate),
+                               _p(probs), _p(colsum), _p(z))
+    if rc != 0:
+        raise ValueError("oracle_route_ex: non-finite logits or noise, or missing noise")
+    return dict(idx=idx, gate=gate, colsum=colsum, probs=probs, zloss=float(z[0]))
 
 
 def topk_margin(logits64: np.ndarray, k: int) -> np.ndarray:

@@ -182,6 +182,87 @@ int oracle_route(int64_t N, int32_t E, int32_t k, int32_t renorm, const float* l
   return 0;
 }
 
+/* Training-time routing variants ([G5] 5.2.2, [GS] 3) and the z-loss ([G5] 5.2.2).
+ *   mode 0: plain top-k (oracle_route).
+ *   mode 1, noisy top-k (Switch): z' = z + noise, formed in fp32 (the precision the kernel adds
+ *           in, so both sides decide on the same values); top-k of z' and gates from
+ *           softmax(z') (renormalised over the selected set when renorm).
+ *   mode 2, GShard random routing: the first expert is the largest unperturbed logit; every
+ *           later one is the largest z' = z + noise (fp32) among the experts not yet chosen;
+ *           gates from the unperturbed softmax(z) (renormalised over the selected set when
+ *           renorm: w_i = P_i / (P_0 + P_1) for top-2, [GS] 3).
+ * Ties keep the lower expert index. probs / prob_colsum report the softmax the gates come
+ * from. zloss (optional): mean over tokens of (log sum_e exp z_e)^2 on the unperturbed logits
+ * (the penalty alpha * (log Z)^2 of [G5] 5.2.2 without alpha). noise may be NULL for mode 0. */
+static int32_t argmax_excluding(const float* v, int32_t E, const uint8_t* taken) {
+  int32_t best = -1;
+  for (int32_t e = 0; e < E; ++e) {
+    if (taken[e]) continue;
+    if (best < 0 || v[e] > v[best]) best = e;
+  }
+  return best;
+}
+
+int oracle_route_ex(int64_t N, int32_t E, int32_t k, int32_t renorm, int32_t mode,
+                    const float* logits32, const float* noise32, int32_t* idx, double* gate,
+                    double* probs, double* prob_colsum, double* zloss) {
+  if (mode == 0) {
+    if (oracle_route(N, E, k, renorm, logits32, idx, gate, probs, prob_colsum) != 0) return -1;
+  } else {
+    if (!all_finite_f32(logits32, N * E) || noise32 == NULL || !all_finite_f32(noise32, N * E))
+      return -1;
+    double* P = probs ? probs : (double*)malloc(sizeof(double) * (size_t)(N * E + 1));
+#pragma omp parallel
+    {
+      float* zn = (float*)malloc(sizeof(float) * (size_t)E);
+      uint8_t* taken = (uint8_t*)malloc((size_t)E);
+#pragma omp for schedule(static)
+      for (int64_t t = 0; t < N; ++t) {
+        const float* z = logits32 + t * E;
+        for (int32_t e = 0; e < E; ++e) {
+          volatile float sum = z[e] + noise32[t * E + e]; /* one fp32 rounding */
+          zn[e] = sum;
+          taken[e] = 0;
+        }
+        double* p = P + t * E;
+        softmax_row(mode == 1 ? zn : z, E, p);
+        for (int32_t j = 0; j < k; ++j) {
+          const int32_t c = argmax_excluding((mode == 2 && j == 0) ? z : zn, E, taken);
+          taken[c] = 1;
+          idx[t * k + j] = c;
+        }
+        double sel = 0.0;
+        for (int32_t j = 0; j < k; ++j) sel += p[idx[t * k + j]];
+        for (int32_t j = 0; j < k; ++j)
+          gate[t * k + j] = renorm ? p[idx[t * k + j]] / sel : p[idx[t * k + j]];
+      }
+      free(zn);
+      free(taken);
+    }
+    if (prob_colsum) {
+      for (int32_t e = 0; e < E; ++e) prob_colsum[e] = 0.0;
+      for (int64_t t = 0; t < N; ++t)
+        for (int32_t e = 0; e < E; ++e) prob_colsum[e] += P[t * E + e];
+    }
+    if (!probs) free(P);
+  }
+  if (zloss) {
+    double acc = 0.0;
+    for (int64_t t = 0; t < N; ++t) {
+      const float* z = logits32 + t * E;
+      double m = (double)z[0];
+      for (int32_t e = 1; e < E; ++e)
+        if ((double)z[e] > m) m = (double)z[e];
+      double sum = 0.0;
+      for (int32_t e = 0; e < E; ++e) sum += exp((double)z[e] - m);
+      const double lz = m + log(sum);
+      acc += lz * lz;
+    }
+    *zloss = N > 0 ? acc / (double)N : 0.0;
+  }
+  return 0;
+}
+
 /* Near-tie margin of each token: with the fp64 logits sorted descending s_0 >= s_1 >= ...,
  * margin = min over the gaps that decide the selected set and its order:
  * s_i - s_{i+1} for i = 0 .. min(k, E-1) - 1. (+inf when E == 1.) */
