@@ -74,6 +74,15 @@ enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_ERF = 1, MOE_ACT_GELU_TANH = 2 };
 enum { MOE_ORDER_SLOT_MAJOR = 0, MOE_ORDER_TOKEN_MAJOR = 1 };
 /* Weights of a token's kept slots when another of its slots was dropped (MoE series 2.2). */
 enum { MOE_DROP_ZERO = 0, MOE_DROP_RENORM_KEPT = 1 };
+/* Expert selection (moe_route_ex / moe_forward_ex; the other entry points need TOPK):
+ *   TOPK           the k largest logits.
+ *   NOISY_TOPK     Grok-1 book 5.2.2 (Switch's noisy top-k): z' = z + noise (fp32); the k
+ *                  largest z' are selected and the gates come from softmax(z').
+ *   GSHARD_RANDOM  MoE series 3: the first expert is the largest z; each later one is the
+ *                  largest z' = z + noise (fp32) among the experts not chosen yet; the gates
+ *                  come from softmax(z) (over the selected set when renormalize = 1, which is
+ *                  GShard's w_i = P_i / (P_0 + P_1) for top-2). */
+enum { MOE_ROUTE_TOPK = 0, MOE_ROUTE_NOISY_TOPK = 1, MOE_ROUTE_GSHARD_RANDOM = 2 };
 
 /* Device error codes written to the workspace error word. */
 enum {
@@ -100,6 +109,7 @@ enum {
  *                   their gates; MOE_DROP_RENORM_KEPT: when a token has dropped and kept
  *                   slots, the kept gates are divided by their sum (GShard case A, MoE series
  *                   2.2: (w1, w2) -> (1, 0) when the second expert overflows)
+ *   routing_mode    MOE_ROUTE_* (selection variant; needs a noise array unless TOPK)
  *   min_capacity    >= 0; the capacity is max(ceil(CF*N*k/E), min_capacity) (MoE series 2.1)
  * bf16 problems need D and F to be multiples of 8 (16-byte rows for the tensor-memory
  * copies); fp32 problems need D and F to be multiples of 4. */
@@ -115,8 +125,9 @@ typedef struct {
   int32_t dtype;
   int32_t capacity_order;
   int32_t drop_policy;
-  int32_t reserved; /* must be 0 */
+  int32_t routing_mode;
   int64_t min_capacity;
+  int32_t reserved; /* must be 0 */
 } moe_problem;
 
 /* Host only. C = max(ceil(CF * N * k / E), min_capacity), the first term evaluated in double
@@ -146,6 +157,20 @@ moe_status moe_workspace_size(const moe_problem* p, size_t* bytes);
 moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, const float* bias,
                      float* logits, int32_t* topk_idx, float* topk_gate, float* prob_colsum,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* moe_route with the training-time selection variants (p->routing_mode) and the z-loss.
+ *   noise   [N,E] fp32, device; the caller's random draws (e.g. N(0, sigma^2) for noisy
+ *           top-k, Grok-1 book 5.2.2; GShard's perturbation, MoE series 3). Required unless
+ *           routing_mode is MOE_ROUTE_TOPK (then ignored).
+ *   z_loss  optional [1] fp32, device: mean over tokens of (log sum_e exp(logits_te))^2 on the
+ *           unperturbed logits (the z-loss of Grok-1 book 5.2.2 before its coefficient);
+ *           summed in a fixed order.
+ *   prob_colsum reports the softmax the gates come from (of z' under NOISY_TOPK).
+ * Everything else as moe_route. */
+moe_status moe_route_ex(const moe_problem* p, const void* X, const float* W_r, const float* bias,
+                        const float* noise, float* logits, int32_t* topk_idx, float* topk_gate,
+                        float* prob_colsum, float* z_loss, void* ws, size_t ws_bytes,
+                        void* stream);
 
 /* Load histogram, capacity, slot assignment and permutation (walkthrough 1.3, 3.1, 3.2;
  * LLMs-from-scratch 12.2; MoE series 2.2).
@@ -251,6 +276,15 @@ moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
                           void* out, float* logits, int32_t* topk_idx, float* topk_gate,
                           int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
                           float* prob_colsum, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward with the training-time selection variants (p->routing_mode, noise as in
+ * moe_route_ex) and the optional z_loss output. */
+moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,
+                          const float* bias, const float* noise, const void* W1, const void* W2,
+                          const void* W3, void* out, float* logits, int32_t* topk_idx,
+                          float* topk_gate, int32_t* load, int32_t* offsets, int32_t* pos,
+                          uint8_t* dropped, float* prob_colsum, float* z_loss, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /* moe_forward with HOST activations: X_host [N,D] and out_host [N,D] are host pointers
  * (page-locked memory gives asynchronous copies), the weights and W_r/bias are device

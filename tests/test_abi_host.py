@@ -23,7 +23,7 @@ def _header_functions():
     with open(os.path.join(ROOT, "include", "moe.h")) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_symbols_exported(abi):
@@ -31,7 +31,7 @@ def test_header_symbols_exported(abi):
     assert set(declared) == set(abi.EXPORTS)
     out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\s[TW]\s(moe_[a-z_]+)$", out, flags=re.M))
+    exported = set(re.findall(r"\s[TW]\s(moe_[a-z0-9_]+)$", out, flags=re.M))
     missing = set(declared) - exported
     assert not missing, f"declared but not exported: {missing}"
     for name in declared:
@@ -169,3 +169,23 @@ def test_w8_entry_points_reject_unsupported_shapes_on_host(abi):
         st = abi.lib.moe_forward_w8(ctypes.byref(p), *([16] * 10), *([None] * 8), 256, 1 << 20,
                                     None)
         assert st == 2
+
+
+def test_routing_mode_checks_on_host(abi):
+    # Unknown modes are invalid; the entry points without a noise argument take plain top-k
+    # only; moe_route_ex needs the noise for the noisy modes.
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("r", N=8, D=64, F=64, E=4, k=2, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1)
+    p = abi.problem(cfg)
+    b = ctypes.c_size_t()
+    p.routing_mode = 3
+    assert abi.lib.moe_workspace_size(ctypes.byref(p), ctypes.byref(b)) == 1
+    p.routing_mode = configs.ROUTE_GSHARD_RANDOM
+    assert abi.lib.moe_workspace_size(ctypes.byref(p), ctypes.byref(b)) == 0
+    ws_bytes = b.value
+    st = abi.lib.moe_route(ctypes.byref(p), 16, 16, None, None, 16, 16, None, 256, ws_bytes, None)
+    assert st == 1 and b"noise" in abi.lib.moe_last_error()
+    st = abi.lib.moe_route_ex(ctypes.byref(p), 16, 16, None, None, None, 16, 16, None, None, 256,
+                              ws_bytes, None)
+    assert st == 1 and b"noise" in abi.lib.moe_last_error()

@@ -23,7 +23,9 @@ DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_INDEX = range(3)
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_workspace_size_host", "moe_route",
-           "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_host",
+           "moe_route_ex", "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn",
+           "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_ex",
+           "moe_forward_host", "moe_expert_up_w8", "moe_expert_down_w8", "moe_forward_w8",
            "moe_workspace_init", "moe_get_device_error", "moe_status_string", "moe_last_error",
            "moe_version")
 
@@ -34,7 +36,8 @@ class moe_problem(ctypes.Structure):
                 ("capacity_factor", ctypes.c_double), ("renormalize", ctypes.c_int32),
                 ("activation", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("capacity_order", ctypes.c_int32), ("drop_policy", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("min_capacity", ctypes.c_int64)]
+                ("routing_mode", ctypes.c_int32), ("min_capacity", ctypes.c_int64),
+                ("reserved", ctypes.c_int32)]
 
 
 class MoEError(RuntimeError):
@@ -63,6 +66,8 @@ def _load() -> ctypes.CDLL:
         "moe_combine": [PP, P, P, P, P, P, P, P, P],
         "moe_forward": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "moe_forward_host": [PP, P, P, P, P, P, P, P, P, S, P],
+        "moe_route_ex": [PP, P, P, P, P, P, P, P, P, P, P, S, P],
+        "moe_forward_ex": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_up_w8": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_down_w8": [PP, P, P, P, P, P, P, S, P],
         "moe_forward_w8": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
@@ -95,7 +100,7 @@ def problem(cfg: MoEConfig, N: Optional[int] = None) -> moe_problem:
                        capacity_factor=float(cfg.capacity_factor), renormalize=cfg.renormalize,
                        activation=cfg.activation, dtype=cfg.dtype,
                        capacity_order=cfg.capacity_order, drop_policy=cfg.drop_policy,
-                       reserved=0, min_capacity=cfg.min_capacity)
+                       routing_mode=cfg.routing_mode, min_capacity=cfg.min_capacity, reserved=0)
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -139,6 +144,13 @@ def route(p, X, W_r, bias, logits, topk_idx, topk_gate, prob_colsum, ws, stream=
                          ws.numel(), _stream(stream)))
 
 
+def route_ex(p, X, W_r, bias, noise, logits, topk_idx, topk_gate, prob_colsum, z_loss, ws,
+             stream=None):
+    _check(lib.moe_route_ex(ctypes.byref(p), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(noise),
+                            _ptr(logits), _ptr(topk_idx), _ptr(topk_gate), _ptr(prob_colsum),
+                            _ptr(z_loss), _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def dispatch(p, X, topk_idx, load, offsets, pos, dropped, row_token, X_perm, ws, stream=None):
     _check(lib.moe_dispatch(ctypes.byref(p), _ptr(X), _ptr(topk_idx), _ptr(load), _ptr(offsets),
                             _ptr(pos), _ptr(dropped), _ptr(row_token), _ptr(X_perm), _ptr(ws),
@@ -179,6 +191,16 @@ def forward(p, X, W_r, bias, W1, W2, W3, out, ws, *, logits=None, topk_idx=None,
                            _ptr(W3), _ptr(out), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
                            _ptr(load), _ptr(offsets), _ptr(pos), _ptr(dropped),
                            _ptr(prob_colsum), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def forward_ex(p, X, W_r, bias, noise, W1, W2, W3, out, ws, *, logits=None, topk_idx=None,
+               topk_gate=None, load=None, offsets=None, pos=None, dropped=None, prob_colsum=None,
+               z_loss=None, stream=None):
+    _check(lib.moe_forward_ex(ctypes.byref(p), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(noise),
+                              _ptr(W1), _ptr(W2), _ptr(W3), _ptr(out), _ptr(logits),
+                              _ptr(topk_idx), _ptr(topk_gate), _ptr(load), _ptr(offsets),
+                              _ptr(pos), _ptr(dropped), _ptr(prob_colsum), _ptr(z_loss),
+                              _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def expert_up_w8(p, X_perm, offsets, W1q, S1, W2q, S2, H, ws, stream=None):

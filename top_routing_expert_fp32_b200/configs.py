@@ -38,6 +38,10 @@ ORDER_TOKEN_MAJOR = 1
 DROP_ZERO = 0
 DROP_RENORM_KEPT = 1
 
+ROUTE_TOPK = 0
+ROUTE_NOISY_TOPK = 1
+ROUTE_GSHARD_RANDOM = 2
+
 
 @dataclass(frozen=True)
 class MoEConfig:
@@ -56,6 +60,8 @@ class MoEConfig:
     capacity_order: int = ORDER_SLOT_MAJOR
     drop_policy: int = DROP_ZERO
     min_capacity: int = 0
+    routing_mode: int = ROUTE_TOPK
+    noise_std: float = 0.0          # std of the routing noise (routing_mode != ROUTE_TOPK)
 
     @property
     def records(self) -> int:

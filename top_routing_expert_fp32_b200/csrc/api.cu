@@ -63,7 +63,7 @@ size_t elem_size(const moe_problem& p) { return p.dtype == MOE_DTYPE_BF16 ? 2 : 
 
 // Device workspace regions (byte offsets from the workspace base).
 struct Layout {
-  size_t err, colsum_part, wt, counts, idx, gate, pos, dropped, load, offsets, row_token,
+  size_t err, colsum_part, zl_part, wt, counts, idx, gate, pos, dropped, load, offsets, row_token,
       xperm, h, y;
   size_t total;       // moe_forward and every other entry point
   size_t xin, xout;   // moe_forward_host only
@@ -82,6 +82,7 @@ Layout make_layout(const moe_problem& p) {
   const size_t es = elem_size(p);
   L.err = take(256);
   L.colsum_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)) * p.E);
+  L.zl_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)));
   L.wt = take(route_tc_wt_bytes(p));
   L.counts = take(sizeof(int32_t) * static_cast<size_t>(dispatch_num_chunks(R)) * p.E);
   L.idx = take(sizeof(int32_t) * R);
@@ -122,6 +123,8 @@ moe_status check_problem(const moe_problem* p) {
   if (p->drop_policy != MOE_DROP_ZERO && p->drop_policy != MOE_DROP_RENORM_KEPT)
     return fail(MOE_ERR_INVALID_ARG, "unknown drop_policy");
   if (p->min_capacity < 0) return fail(MOE_ERR_INVALID_ARG, "min_capacity < 0");
+  if (p->routing_mode < MOE_ROUTE_TOPK || p->routing_mode > MOE_ROUTE_GSHARD_RANDOM)
+    return fail(MOE_ERR_INVALID_ARG, "unknown routing_mode");
   if (p->N * static_cast<int64_t>(p->k) > INT32_MAX)
     return fail(MOE_ERR_UNSUPPORTED, "N*k exceeds 2^31-1 records");
   if (p->D > (1 << 24) || p->F > (1 << 24)) return fail(MOE_ERR_UNSUPPORTED, "D or F > 2^24");
@@ -256,11 +259,35 @@ moe_status check_w8(const moe_problem& p) {
   return MOE_OK;
 }
 
+// Entry points without a noise argument: only plain top-k selection.
+moe_status need_topk(const moe_problem& p) {
+  if (p.routing_mode != MOE_ROUTE_TOPK)
+    return fail(MOE_ERR_INVALID_ARG,
+                "routing_mode needs a noise array: use moe_route_ex / moe_forward_ex");
+  return MOE_OK;
+}
+
+moe_status route_impl(const moe_problem& p, const void* X, const float* W_r, const float* bias,
+                      const float* noise, float* logits, int32_t* topk_idx, float* topk_gate,
+                      float* prob_colsum, float* z_loss, void* ws, cudaStream_t s) {
+  const Layout L = make_layout(p);
+  if (p.N == 0) {
+    if (prob_colsum) MOE_CUDA(cudaMemsetAsync(prob_colsum, 0, sizeof(float) * p.E, s), "memset");
+    if (z_loss) MOE_CUDA(cudaMemsetAsync(z_loss, 0, sizeof(float), s), "memset");
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_route(p, X, W_r, bias, noise, logits, topk_idx, topk_gate,
+                        at<float>(ws, L.colsum_part), prob_colsum, at<float>(ws, L.zl_part), z_loss,
+                        at<__nv_bfloat16>(ws, L.wt), at<int>(ws, L.err), wait_timeout_ns(), s),
+           "route");
+  return MOE_OK;
+}
+
 moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, const float* bias,
-                        const Experts& w, void* out, float* logits,
+                        const float* noise, const Experts& w, void* out, float* logits,
                         int32_t* topk_idx, float* topk_gate, int32_t* load, int32_t* offsets,
-                        int32_t* pos, uint8_t* dropped, float* prob_colsum, void* ws,
-                        cudaStream_t stream) {
+                        int32_t* pos, uint8_t* dropped, float* prob_colsum, float* z_loss,
+                        void* ws, cudaStream_t stream) {
   const Layout L = make_layout(p);
   int* err = at<int>(ws, L.err);
   int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
@@ -278,12 +305,10 @@ moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, c
                                 err, stream),
              "dispatch");
     if (prob_colsum) MOE_CUDA(cudaMemsetAsync(prob_colsum, 0, sizeof(float) * p.E, stream), "memset");
+    if (z_loss) MOE_CUDA(cudaMemsetAsync(z_loss, 0, sizeof(float), stream), "memset");
     return MOE_OK;
   }
-  MOE_CUDA(launch_route(p, X, W_r, bias, logits, idx, gate, at<float>(ws, L.colsum_part),
-                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), err, wait_timeout_ns(),
-                        stream),
-           "route");
+  MOE_TRY(route_impl(p, X, W_r, bias, noise, logits, idx, gate, prob_colsum, z_loss, ws, stream));
   MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps, dr,
                               row_token, err, stream),
            "slot assign");
@@ -334,17 +359,32 @@ moe_status moe_route(const moe_problem* p, const void* X, const float* W_r, cons
   MOE_TRY(need(topk_idx, "topk_idx", 4));
   MOE_TRY(need(topk_gate, "topk_gate", 4));
   MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
-  const Layout L = make_layout(*p);
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p->N == 0) {
-    if (prob_colsum) MOE_CUDA(cudaMemsetAsync(prob_colsum, 0, sizeof(float) * p->E, s), "memset");
-    return MOE_OK;
+  MOE_TRY(need_topk(*p));
+  return route_impl(*p, X, W_r, bias, nullptr, logits, topk_idx, topk_gate, prob_colsum, nullptr,
+                    ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_route_ex(const moe_problem* p, const void* X, const float* W_r, const float* bias,
+                        const float* noise, float* logits, int32_t* topk_idx, float* topk_gate,
+                        float* prob_colsum, float* z_loss, void* ws, size_t ws_bytes,
+                        void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  if (X != nullptr) {
+    MOE_TRY(need(X, "X"));
+    MOE_TRY(need(W_r, "W_r"));
+    MOE_TRY(opt(logits, "logits", 4));
+  } else {
+    MOE_TRY(need(logits, "logits (input when X is NULL)", 4));
   }
-  MOE_CUDA(launch_route(*p, X, W_r, bias, logits, topk_idx, topk_gate, at<float>(ws, L.colsum_part),
-                        prob_colsum, at<__nv_bfloat16>(ws, L.wt), at<int>(ws, L.err),
-                        wait_timeout_ns(), s),
-           "route");
-  return MOE_OK;
+  MOE_TRY(opt(bias, "bias", 4));
+  if (p->routing_mode != MOE_ROUTE_TOPK && p->N > 0) MOE_TRY(need(noise, "noise", 4));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(topk_gate, "topk_gate", 4));
+  MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
+  MOE_TRY(opt(z_loss, "z_loss", 4));
+  return route_impl(*p, X, W_r, bias, noise, logits, topk_idx, topk_gate, prob_colsum, z_loss,
+                    ws, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk_idx,
@@ -471,8 +511,44 @@ moe_status moe_forward(const moe_problem* p, const void* X, const float* W_r, co
   w.W1 = W1;
   w.W2 = W2;
   w.W3 = W3;
-  return forward_impl(*p, X, W_r, bias, w, out, logits, topk_idx, topk_gate, load,
-                      offsets, pos, dropped, prob_colsum, ws, static_cast<cudaStream_t>(stream));
+  MOE_TRY(need_topk(*p));
+  return forward_impl(*p, X, W_r, bias, nullptr, w, out, logits, topk_idx, topk_gate, load,
+                      offsets, pos, dropped, prob_colsum, nullptr, ws,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,
+                          const float* bias, const float* noise, const void* W1, const void* W2,
+                          const void* W3, void* out, float* logits, int32_t* topk_idx,
+                          float* topk_gate, int32_t* load, int32_t* offsets, int32_t* pos,
+                          uint8_t* dropped, float* prob_colsum, float* z_loss, void* ws,
+                          size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X, "X"));
+  MOE_TRY(need(W_r, "W_r"));
+  MOE_TRY(opt(bias, "bias", 4));
+  if (p->routing_mode != MOE_ROUTE_TOPK && p->N > 0) MOE_TRY(need(noise, "noise", 4));
+  MOE_TRY(need(W1, "W1"));
+  MOE_TRY(need(W2, "W2"));
+  MOE_TRY(need(W3, "W3"));
+  MOE_TRY(need(out, "out"));
+  MOE_TRY(opt(logits, "logits", 4));
+  MOE_TRY(opt(topk_idx, "topk_idx", 4));
+  MOE_TRY(opt(topk_gate, "topk_gate", 4));
+  MOE_TRY(opt(load, "load", 4));
+  MOE_TRY(opt(offsets, "offsets", 4));
+  MOE_TRY(opt(pos, "pos", 4));
+  MOE_TRY(opt(dropped, "dropped", 1));
+  MOE_TRY(opt(prob_colsum, "prob_colsum", 4));
+  MOE_TRY(opt(z_loss, "z_loss", 4));
+  Experts w;
+  w.W1 = W1;
+  w.W2 = W2;
+  w.W3 = W3;
+  return forward_impl(*p, X, W_r, bias, noise, w, out, logits, topk_idx, topk_gate, load,
+                      offsets, pos, dropped, prob_colsum, z_loss, ws,
+                      static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_forward_host(const moe_problem* p, const void* X_host, const float* W_r,
@@ -480,6 +556,7 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
                             void* out_host, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(check_problem(p));
   MOE_TRY(check_ws(*p, ws, ws_bytes, true));
+  MOE_TRY(need_topk(*p));
   if (p->N > 0) {
     MOE_TRY(need(X_host, "X_host", 1));
     MOE_TRY(need(out_host, "out_host", 1));
@@ -499,8 +576,8 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
   w.W1 = W1;
   w.W2 = W2;
   w.W3 = W3;
-  MOE_TRY(forward_impl(*p, xin, W_r, bias, w, xout, nullptr, nullptr, nullptr, nullptr,
-                       nullptr, nullptr, nullptr, nullptr, ws, s));
+  MOE_TRY(forward_impl(*p, xin, W_r, bias, nullptr, w, xout, nullptr, nullptr, nullptr,
+                       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, ws, s));
   if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, s), "D2H");
   MOE_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   return MOE_OK;
@@ -582,8 +659,10 @@ moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
   w.S1 = S1;
   w.S2 = S2;
   w.S3 = S3;
-  return forward_impl(*p, X, W_r, bias, w, out, logits, topk_idx, topk_gate, load, offsets, pos,
-                      dropped, prob_colsum, ws, static_cast<cudaStream_t>(stream));
+  MOE_TRY(need_topk(*p));
+  return forward_impl(*p, X, W_r, bias, nullptr, w, out, logits, topk_idx, topk_gate, load,
+                      offsets, pos, dropped, prob_colsum, nullptr, ws,
+                      static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -620,7 +699,7 @@ const char* moe_status_string(moe_status s) {
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
-int32_t moe_version(void) { return 110; }
+int32_t moe_version(void) { return 120; }
 
 }  // extern "C"
 

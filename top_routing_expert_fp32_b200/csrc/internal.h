@@ -20,9 +20,12 @@ int route_num_blocks(int64_t N, int E);
 // Router logits + softmax + top-k + gates. X == nullptr: `logits` is an input.
 // colsum_partial: [route_num_blocks][E] floats (or nullptr when prob_colsum is nullptr).
 // wt: scratch of the tensor-core router (route_tc_wt_bytes), used for bf16 X.
+// noise: [N][E] (p.routing_mode != TOPK). zl_partial: [route_num_blocks] floats, used when
+// z_loss (device scalar) is requested.
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
-                         float* logits, int32_t* idx, float* gate, float* colsum_partial,
-                         float* prob_colsum, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
+                         const float* noise, float* logits, int32_t* idx, float* gate,
+                         float* colsum_partial, float* prob_colsum, float* zl_partial,
+                         float* z_loss, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
                          cudaStream_t stream);
 
 // Tensor-core router for bf16 X (logits from a three-term bf16 split of W_r, then the routing
@@ -31,9 +34,10 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
 bool route_tc_supported(const moe_problem& p);
 size_t route_tc_wt_bytes(const moe_problem& p);
 cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
-                            const float* bias, __nv_bfloat16* wt, float* logits_out, int32_t* idx,
-                            float* gate, float* colsum_partial, int* grid_out, int* err,
-                            uint64_t timeout_ns, cudaStream_t stream);
+                            const float* bias, const float* noise, __nv_bfloat16* wt,
+                            float* logits_out, int32_t* idx, float* gate, float* colsum_partial,
+                            float* zl_partial, int* grid_out, int* err, uint64_t timeout_ns,
+                            cudaStream_t stream);
 
 // 2-D bf16 tensor map (cols contiguous, row stride cols * 2 bytes), box box_cols x box_rows,
 // 128-byte swizzle, out-of-range elements read as zero.

@@ -38,6 +38,9 @@ struct RouteArgs {
   int32_t* idx;
   float* gate;
   float* colsum_partial;  // [gridDim.x][E] or nullptr
+  const float* noise;     // [N][E] (routing_mode != TOPK) or nullptr
+  int mode;               // MOE_ROUTE_*
+  float* zl_partial;      // [gridDim.x]: per-block sum of (log Z)^2, or nullptr
   int64_t N;
   int D;
   int E;
@@ -93,8 +96,10 @@ __device__ __forceinline__ void load_w(const float* __restrict__ W_r, int d, int
 // kMaxE + 1). One thread per token; afterwards s_z holds the probabilities if colsum is
 // wanted. `colsum_acc` (thread e < E) accumulates this block's per-expert probability sum in
 // token order.
+// (log Z)^2 of token row i is parked in the row's spare column kMaxE (E <= kMaxE).
 __device__ __forceinline__ void select_tile(const RouteArgs& a, float (*s_z)[kMaxE + 1],
-                                            int tpc, int64_t t_tile, float& colsum_acc) {
+                                            int tpc, int64_t t_tile, float& colsum_acc,
+                                            float& zl_acc) {
   const int E = a.E;
   const int tl = threadIdx.x;
   const int64_t t = t_tile + tl;
@@ -102,21 +107,26 @@ __device__ __forceinline__ void select_tile(const RouteArgs& a, float (*s_z)[kMa
     float* z = s_z[tl];
     if (a.logits_out != nullptr)
       for (int e = 0; e < E; ++e) a.logits_out[t * E + e] = z[e];
-    select_token(z, E, a.k, a.renorm, a.idx + t * a.k, a.gate + t * a.k,
-                 a.colsum_partial != nullptr);
+    float lse = 0.f;
+    select_token(z, E, a.k, a.renorm, a.mode, a.noise != nullptr ? a.noise + t * E : nullptr,
+                 a.idx + t * a.k, a.gate + t * a.k, a.colsum_partial != nullptr,
+                 a.zl_partial != nullptr ? &lse : nullptr);
+    z[kMaxE] = lse * lse;
   }
   __syncthreads();
-  if (a.colsum_partial != nullptr && static_cast<int>(threadIdx.x) < E) {
-    const int64_t valid64 = a.N - t_tile;
-    const int valid = valid64 < tpc ? static_cast<int>(valid64) : tpc;
+  const int64_t valid64 = a.N - t_tile;
+  const int valid = valid64 < tpc ? static_cast<int>(valid64) : tpc;
+  if (a.colsum_partial != nullptr && static_cast<int>(threadIdx.x) < E)
     for (int i = 0; i < valid; ++i) colsum_acc += s_z[i][threadIdx.x];
-  }
+  if (a.zl_partial != nullptr && threadIdx.x == 0)
+    for (int i = 0; i < valid; ++i) zl_acc += s_z[i][kMaxE];
   __syncthreads();
 }
 
-__device__ __forceinline__ void write_colsum(const RouteArgs& a, float colsum_acc) {
+__device__ __forceinline__ void write_colsum(const RouteArgs& a, float colsum_acc, float zl_acc) {
   if (a.colsum_partial != nullptr && static_cast<int>(threadIdx.x) < a.E)
     a.colsum_partial[static_cast<int64_t>(blockIdx.x) * a.E + threadIdx.x] = colsum_acc;
+  if (a.zl_partial != nullptr && threadIdx.x == 0) a.zl_partial[blockIdx.x] = zl_acc;
 }
 
 // ------------------------------------------------------------------ narrow: E <= 16
@@ -204,6 +214,7 @@ __global__ void __launch_bounds__(kNarrowThreads, 1) route_narrow_kernel(RouteAr
   const int ks = warp % KS;                          // this warp's K slice
   const int tpb = groups_per_block * G;              // tokens per block step
   float colsum_acc = 0.f;
+  float zl_acc = 0.f;
   const int nvec = D / V;  // 16-byte chunks of an X row
 
   for (int64_t step = blockIdx.x; step * tpb < a.N; step += gridDim.x) {
@@ -299,9 +310,9 @@ __global__ void __launch_bounds__(kNarrowThreads, 1) route_narrow_kernel(RouteAr
       if (e < E) s_z[tg * G + g][e] = z + (a.bias != nullptr ? __ldg(a.bias + e) : 0.f);
     }
     __syncthreads();
-    select_tile(a, s_z, tpb, step * tpb, colsum_acc);
+    select_tile(a, s_z, tpb, step * tpb, colsum_acc, zl_acc);
   }
-  write_colsum(a, colsum_acc);
+  write_colsum(a, colsum_acc, zl_acc);
 }
 
 // ------------------------------------------------------------------ wide: 16 < E <= 64
@@ -333,6 +344,7 @@ __global__ void __launch_bounds__(kWideThreads) route_wide_kernel(RouteArgs a) {
   const int D = a.D;
   const int E = a.E;
   float colsum_acc = 0.f;
+  float zl_acc = 0.f;
   constexpr int kChunks = kWBK / V;                      // 16-byte chunks per token per slice
   constexpr int kXLoads = kWT * kChunks / kWideThreads;  // 2 (bf16) or 4 (fp32)
   const int nslices = (D + kWBK - 1) / kWBK;
@@ -439,9 +451,9 @@ __global__ void __launch_bounds__(kWideThreads) route_wide_kernel(RouteArgs a) {
         }
     }
     __syncthreads();
-    select_tile(a, s_z, kWT, t0, colsum_acc);
+    select_tile(a, s_z, kWT, t0, colsum_acc, zl_acc);
   }
-  write_colsum(a, colsum_acc);
+  write_colsum(a, colsum_acc, zl_acc);
 }
 
 // ------------------------------------------------------------------ routing from given logits
@@ -451,6 +463,7 @@ constexpr int kSelThreads = 64;
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(RouteArgs a) {
   __shared__ float s_z[kSelThreads][kMaxE + 1];
   float colsum_acc = 0.f;
+  float zl_acc = 0.f;
   const int E = a.E;
   for (int64_t tile = blockIdx.x; tile * kSelThreads < a.N; tile += gridDim.x) {
     const int64_t t0 = tile * kSelThreads;
@@ -460,9 +473,18 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(RouteArgs a) 
       if (t0 + tl < a.N) s_z[tl][e] = a.logits_in[(t0 + tl) * E + e];
     }
     __syncthreads();
-    select_tile(a, s_z, kSelThreads, t0, colsum_acc);
+    select_tile(a, s_z, kSelThreads, t0, colsum_acc, zl_acc);
   }
-  write_colsum(a, colsum_acc);
+  write_colsum(a, colsum_acc, zl_acc);
+}
+
+// z_loss = (sum over blocks, in block order, of the per-block sums of (log Z)^2) / N.
+__global__ void zloss_reduce_kernel(const float* __restrict__ partial, int nblocks, int64_t N,
+                                    float* __restrict__ out) {
+  if (threadIdx.x != 0) return;
+  float s = 0.f;
+  for (int b = 0; b < nblocks; ++b) s += partial[b];
+  out[0] = N > 0 ? s / static_cast<float>(N) : 0.f;
 }
 
 // prob_colsum[e] = sum over blocks, in block order, of the per-block partials.
@@ -547,11 +569,15 @@ int route_num_blocks(int64_t N, int E) {
 }
 
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
-                         float* logits, int32_t* idx, float* gate, float* colsum_partial,
-                         float* prob_colsum, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
+                         const float* noise, float* logits, int32_t* idx, float* gate,
+                         float* colsum_partial, float* prob_colsum, float* zl_partial,
+                         float* z_loss, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
                          cudaStream_t stream) {
   if (p.N == 0) return cudaSuccess;
   RouteArgs a;
+  a.noise = p.routing_mode != MOE_ROUTE_TOPK ? noise : nullptr;
+  a.mode = p.routing_mode;
+  a.zl_partial = z_loss != nullptr ? zl_partial : nullptr;
   a.X = X;
   a.W_r = W_r;
   a.bias = bias;
@@ -570,8 +596,8 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
   cudaError_t e = cudaSuccess;
   if (X != nullptr && route_tc_supported(p)) {
     // bf16 activations: one tensor-core kernel computes the logits and routes.
-    e = launch_route_tc(p, X, W_r, bias, wt, a.logits_out, idx, gate, a.colsum_partial, &grid, err,
-                        timeout_ns, stream);
+    e = launch_route_tc(p, X, W_r, bias, a.noise, wt, a.logits_out, idx, gate, a.colsum_partial,
+                        a.zl_partial, &grid, err, timeout_ns, stream);
   } else if (kind == Kind::kSelect) {
     grid = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>((p.N + kSelThreads - 1) / kSelThreads, kMaxBlocks)));
@@ -593,6 +619,11 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
   if (e != cudaSuccess) return e;
   if (prob_colsum != nullptr) {
     colsum_reduce_kernel<<<1, kMaxE, 0, stream>>>(colsum_partial, grid, p.E, prob_colsum);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (z_loss != nullptr) {
+    zloss_reduce_kernel<<<1, 32, 0, stream>>>(zl_partial, grid, p.N, z_loss);
     e = cudaGetLastError();
   }
   return e;

@@ -55,6 +55,9 @@ struct TcArgs {
   int32_t* idx;            // [N][k]
   float* gate;             // [N][k]
   float* colsum_partial;   // [gridDim.x][E] or nullptr
+  const float* noise;      // [N][E] (mode != TOPK) or nullptr
+  float* zl_partial;       // [gridDim.x] sums of (log Z)^2, or nullptr
+  int mode;                // MOE_ROUTE_*
   int64_t N;
   int64_t tiles;
   int E, k, renorm;
@@ -207,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int E = a.E;
     const uint32_t zrow_s = smem_u32(zbuf) + static_cast<uint32_t>(row * a.zstride) * 4u;
     float colsum_acc = 0.f;
+    float zl_acc = 0.f;
     int it = 0;
     for (int64_t tile = first_tile; tile < a.tiles; tile += a.num_clusters, ++it) {
       const int acc = it & 1;
@@ -308,22 +312,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < EB; ++e)
             if (e < E) a.logits_out[t * E + e] = z[e];
-        select_token_regs<EB>(z, E, a.k, a.renorm, a.idx + t * a.k, a.gate + t * a.k,
-                              a.colsum_partial != nullptr ? s_z + (row - share0) * (E + 1)
-                                                          : nullptr);
+        float* zt = s_z + (row - share0) * (E + 1);  // column E: (log Z)^2 of the token
+        float lse = 0.f;
+        select_token_regs<EB>(z, E, a.k, a.renorm, a.mode,
+                              a.noise != nullptr ? a.noise + t * E : nullptr, a.idx + t * a.k,
+                              a.gate + t * a.k, a.colsum_partial != nullptr ? zt : nullptr,
+                              a.zl_partial != nullptr ? &lse : nullptr);
+        zt[E] = lse * lse;
       }
-      if (a.colsum_partial != nullptr) {  // per-expert probability sums in token order
+      if (a.colsum_partial != nullptr || a.zl_partial != nullptr) {  // sums in token order
         named_bar_sync(1, kEpiThreads);
-        if (et < E) {
-          const int64_t left = a.N - (tile * kRows + share0);
-          const int valid = left < T ? static_cast<int>(left > 0 ? left : 0) : T;
+        const int64_t left = a.N - (tile * kRows + share0);
+        const int valid = left < T ? static_cast<int>(left > 0 ? left : 0) : T;
+        if (a.colsum_partial != nullptr && et < E)
           for (int i = 0; i < valid; ++i) colsum_acc += s_z[i * (E + 1) + et];
-        }
+        if (a.zl_partial != nullptr && et == 0)
+          for (int i = 0; i < valid; ++i) zl_acc += s_z[i * (E + 1) + E];
         named_bar_sync(1, kEpiThreads);
       }
     }
     if (a.colsum_partial != nullptr && et < E)
       a.colsum_partial[static_cast<int64_t>(blockIdx.x) * E + et] = colsum_acc;
+    if (a.zl_partial != nullptr && et == 0) a.zl_partial[blockIdx.x] = zl_acc;
   }
 
   __syncwarp();  // role branches leave warps 0 and 1 divergent; the barriers below are .aligned
@@ -427,9 +437,10 @@ size_t route_tc_wt_bytes(const moe_problem& p) {
 }
 
 cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
-                            const float* bias, __nv_bfloat16* wt, float* logits_out, int32_t* idx,
-                            float* gate, float* colsum_partial, int* grid_out, int* err,
-                            uint64_t timeout_ns, cudaStream_t stream) {
+                            const float* bias, const float* noise, __nv_bfloat16* wt,
+                            float* logits_out, int32_t* idx, float* gate, float* colsum_partial,
+                            float* zl_partial, int* grid_out, int* err, uint64_t timeout_ns,
+                            cudaStream_t stream) {
   const TcShape s = tc_shape(p.N, static_cast<int>(p.D), p.E);
   *grid_out = 0;
   if (p.N == 0) return cudaSuccess;
@@ -452,6 +463,9 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   a.idx = idx;
   a.gate = gate;
   a.colsum_partial = colsum_partial;
+  a.noise = noise;
+  a.zl_partial = zl_partial;
+  a.mode = p.routing_mode;
   a.N = p.N;
   a.tiles = s.tiles;
   a.E = p.E;

@@ -1,8 +1,15 @@
 // Per-token routing decision from fp32 logits, shared by every router kernel:
-// softmax over the E experts, the k largest logits in descending order (equal logits keep the
-// lower expert index first), and the gates.
+// softmax over the E experts, the k selected experts in order (equal values keep the lower
+// expert index first), and the gates.
 //   Grok-1 book ch.5, 5.2 (softmax, TopK) and 5.2.3 (gates with and without renormalisation);
 //   MoE formula-to-code walkthrough 1.1-1.2; LLMs-from-scratch ch.12, 12.1.
+// Training-time variants (mode), with the caller's noise row n:
+//   MOE_ROUTE_NOISY_TOPK (Grok-1 book 5.2.2, Switch's noisy top-k): z' = z + n in fp32; the
+//     selection and the gates use z'.
+//   MOE_ROUTE_GSHARD_RANDOM (MoE series 3): the first expert is the largest z; every later one
+//     the largest z' = z + n (fp32) among the experts not chosen yet; the gates use z.
+// lse (optional) receives log sum_e exp(z_e) of the unperturbed logits (the z-loss term of
+// Grok-1 book 5.2.2).
 #pragma once
 
 #include "common.cuh"
@@ -10,12 +17,22 @@
 namespace moe {
 
 // z: the token's E logits (shared memory). Writes idx[0..k) and gate[0..k) (global). With
-// `probs`, z is overwritten with the full softmax probabilities (for the balance statistic).
-//   renorm = 0: gate_j = softmax(z)[idx_j];  renorm = 1: softmax over the selected logits.
+// `probs`, z is overwritten with the softmax the gates come from (for the balance statistic).
+//   renorm = 0: gate_j = softmax[idx_j];  renorm = 1: softmax over the selected set.
 // Selection compares logits, never probabilities: softmax is increasing, so the set is the
 // same, and the decision is taken in fp32 on the values the caller holds.
-__device__ __forceinline__ void select_token(float* z, int E, int k, int renorm, int32_t* idx,
-                                             float* gate, bool probs) {
+__device__ __forceinline__ void select_token(float* z, int E, int k, int renorm, int mode,
+                                             const float* noise, int32_t* idx, float* gate,
+                                             bool probs, float* lse) {
+  if (lse != nullptr) {
+    float m = z[0];
+    for (int e = 1; e < E; ++e) m = z[e] > m ? z[e] : m;
+    float s = 0.f;
+    for (int e = 0; e < E; ++e) s += expf(z[e] - m);
+    *lse = m + logf(s);
+  }
+  if (mode == MOE_ROUTE_NOISY_TOPK)
+    for (int e = 0; e < E; ++e) z[e] = z[e] + noise[e];
   float zmax = z[0];
   for (int e = 1; e < E; ++e) zmax = z[e] > zmax ? z[e] : zmax;
   uint64_t chosen = 0;
@@ -24,10 +41,16 @@ __device__ __forceinline__ void select_token(float* z, int E, int k, int renorm,
   for (int j = 0; j < 8; ++j) {
     sel[j] = 0;
     if (j < k) {
+      const bool perturbed = mode == MOE_ROUTE_GSHARD_RANDOM && j > 0;
       int best = -1;
+      float vb = 0.f;
       for (int e = 0; e < E; ++e) {
         if ((chosen >> e) & 1ull) continue;
-        if (best < 0 || z[e] > z[best]) best = e;  // strict: equal keeps the lower index
+        const float v = perturbed ? z[e] + noise[e] : z[e];
+        if (best < 0 || v > vb) {  // strict: equal keeps the lower index
+          best = e;
+          vb = v;
+        }
       }
       chosen |= 1ull << best;
       sel[j] = best;
@@ -54,10 +77,29 @@ __device__ __forceinline__ void select_token(float* z, int E, int k, int renorm,
 // The same decision with the logits in registers (EB >= E, entries past E ignored): every
 // loop is unrolled, so nothing waits on shared memory. Sums run in the same order as
 // select_token, so both give the same bits for the same logits. probs (shared memory,
-// optional) receives the full softmax.
+// optional) receives the softmax the gates come from.
 template <int EB>
-__device__ __forceinline__ void select_token_regs(const float (&z)[EB], int E, int k, int renorm,
-                                                  int32_t* idx, float* gate, float* probs) {
+__device__ __forceinline__ void select_token_regs(float (&z)[EB], int E, int k, int renorm,
+                                                  int mode, const float* noise, int32_t* idx,
+                                                  float* gate, float* probs, float* lse) {
+  if (lse != nullptr) {
+    float m = z[0];
+#pragma unroll
+    for (int e = 1; e < EB; ++e)
+      if (e < E) m = z[e] > m ? z[e] : m;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < EB; ++e)
+      if (e < E) s += expf(z[e] - m);
+    *lse = m + logf(s);
+  }
+  float n[EB];
+#pragma unroll
+  for (int e = 0; e < EB; ++e) n[e] = (mode != MOE_ROUTE_TOPK && e < E) ? noise[e] : 0.f;
+  if (mode == MOE_ROUTE_NOISY_TOPK) {
+#pragma unroll
+    for (int e = 0; e < EB; ++e) z[e] = z[e] + n[e];
+  }
   float zmax = z[0];
 #pragma unroll
   for (int e = 1; e < EB; ++e)
@@ -70,17 +112,22 @@ __device__ __forceinline__ void select_token_regs(const float (&z)[EB], int E, i
     sel[j] = 0;
     selz[j] = 0.f;
     if (j < k) {
+      const bool perturbed = mode == MOE_ROUTE_GSHARD_RANDOM && j > 0;
       int best = -1;
-      float zb = 0.f;
+      float vb = 0.f;
 #pragma unroll
       for (int e = 0; e < EB; ++e) {
-        const bool take = e < E && !((chosen >> e) & 1ull) && (best < 0 || z[e] > zb);
+        const float v = perturbed ? z[e] + n[e] : z[e];
+        const bool take = e < E && !((chosen >> e) & 1ull) && (best < 0 || v > vb);
         best = take ? e : best;  // strict: equal keeps the lower index
-        zb = take ? z[e] : zb;
+        vb = take ? v : vb;
       }
       chosen |= 1ull << best;
       sel[j] = best;
-      selz[j] = zb;
+      float zs = 0.f;  // the gate uses the (unperturbed, or mode-1 perturbed) z of the choice
+#pragma unroll
+      for (int e = 0; e < EB; ++e) zs = e == best ? z[e] : zs;
+      selz[j] = zs;
     }
   }
   float s_all = 0.f;

@@ -7,7 +7,7 @@ of the same values), so the two sides never disagree about their inputs.
 Recipe (every config; seed 0 unless a test says otherwise):
 
 * every tensor has its own ``torch.Generator`` seeded with ``seed * 1000 + tensor_id``
-  (X=1, W_r=2, W1=3, W2=4, W3=5, bias=6, logits=7);
+  (X=1, W_r=2, W1=3, W2=4, W3=5, bias=6, logits=7, routing noise=8);
 * values are drawn in fp32 with ``torch.randn``, scaled by the standard deviation, then
   cast to the config dtype (bf16 or fp32); W_r and the bias always stay fp32;
 * X ~ N(0, 1); W_r, W1, W2 ~ N(0, 1/D); W3 ~ N(0, 1/F) (variance = 1/fan_in);
@@ -27,7 +27,7 @@ import torch
 
 from .configs import DTYPE_BF16, DTYPE_F32, MoEConfig
 
-TID_X, TID_WR, TID_W1, TID_W2, TID_W3, TID_BIAS, TID_LOGITS = 1, 2, 3, 4, 5, 6, 7
+TID_X, TID_WR, TID_W1, TID_W2, TID_W3, TID_BIAS, TID_LOGITS, TID_NOISE = 1, 2, 3, 4, 5, 6, 7, 8
 
 
 def torch_dtype(code: int) -> torch.dtype:
@@ -131,6 +131,12 @@ def make_w8_weights(cfg: MoEConfig, device="cpu", seed: Optional[int] = None) ->
             q[e], sc[e] = _quantize_columns(w.mul_(1.0 / math.sqrt(fan_in)))
         out += [q, sc]
     return MoEWeights8(*out)
+
+
+def make_noise(N: int, E: int, std: float, device="cpu", seed: int = 0) -> torch.Tensor:
+    """The random draws of the training-time routing variants, N(0, std^2) fp32 [N, E]: the
+    layer takes them as an input so that every consumer sees the same numbers."""
+    return randn((N, E), std, torch.float32, device, seed, TID_NOISE)
 
 
 def make_logits(N: int, E: int, device="cpu", seed: int = 0, std: float = 1.0) -> torch.Tensor:
