@@ -291,7 +291,10 @@ moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,
  * pointers. Enqueues the host->device copy of X, the forward, and the device->host copy
  * of out on `stream`, then waits for the stream, so out_host is valid on return. Uses
  * the workspace (moe_workspace_size + N*D*2*sizeof(element) bytes, see
- * moe_workspace_size_host). */
+ * moe_workspace_size_host). Without capacity (capacity_factor <= 0) and with N >= 1024 the
+ * batch runs as two halves, the copies of one half overlapping the other half's layer on an
+ * internal copy stream; each token's output is then the layer on its own half-batch (the same
+ * result up to the rounding of the router's split of D). Needs routing_mode = TOPK. */
 moe_status moe_forward_host(const moe_problem* p, const void* X_host, const float* W_r,
                             const float* bias, const void* W1, const void* W2, const void* W3,
                             void* out_host, void* ws, size_t ws_bytes, void* stream);

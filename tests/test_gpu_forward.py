@@ -177,3 +177,24 @@ def test_forward_named_workload_full_size(abi, name):
     print(f"\n{name}: {s}")
     del inp
     torch.cuda.empty_cache()
+
+
+def test_forward_host_two_halves_equal_forward_on_each_half(abi):
+    # Without capacity moe_forward_host runs the batch as two pipelined halves; each half's
+    # output must be exactly moe_forward on that half alone.
+    cfg = configs.MoEConfig("split", N=1501, D=256, F=512, E=8, k=2, dtype=configs.DTYPE_BF16,
+                            activation=configs.ACT_SILU, renormalize=1)
+    inp = inputs.make_inputs(cfg, "cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p, host=True)
+    xh = inp.X.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws)
+    n0 = cfg.N // 2
+    for lo, hi in ((0, n0), (n0, cfg.N)):
+        ph = abi.problem(cfg, N=hi - lo)
+        wsh = abi.workspace(ph)
+        o = torch.empty((hi - lo, cfg.D), dtype=torch.bfloat16, device="cuda")
+        abi.forward(ph, inp.X[lo:hi].contiguous(), inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, o, wsh)
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu().view(torch.int16), oh[lo:hi].view(torch.int16))

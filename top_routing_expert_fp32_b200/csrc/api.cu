@@ -551,6 +551,27 @@ moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,
                       static_cast<cudaStream_t>(stream));
 }
 
+// A non-blocking stream per device for the host copies of moe_forward_host (created on first
+// use, kept for the life of the process).
+cudaError_t copy_stream(cudaStream_t* out) {
+  static cudaStream_t streams[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (streams[dev] == nullptr) {
+    e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+  }
+  *out = streams[dev];
+  return cudaSuccess;
+}
+
+// Tokens per half below which moe_forward_host does not split the batch.
+constexpr int64_t kMinHalfTokens = 512;
+
 moe_status moe_forward_host(const moe_problem* p, const void* X_host, const float* W_r,
                             const float* bias, const void* W1, const void* W2, const void* W3,
                             void* out_host, void* ws, size_t ws_bytes, void* stream) {
@@ -571,16 +592,69 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
   const size_t bytes = elem_size(*p) * static_cast<size_t>(p->N) * static_cast<size_t>(p->D);
   void* xin = at<void>(ws, L.xin);
   void* xout = at<void>(ws, L.xout);
-  if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(xin, X_host, bytes, cudaMemcpyHostToDevice, s), "H2D");
   Experts w;
   w.W1 = W1;
   w.W2 = W2;
   w.W3 = W3;
-  MOE_TRY(forward_impl(*p, xin, W_r, bias, nullptr, w, xout, nullptr, nullptr, nullptr,
-                       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, ws, s));
-  if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, s), "D2H");
-  MOE_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
-  return MOE_OK;
+  // Without capacity every token's output depends on that token alone, so the batch runs as
+  // two halves: the copy of the second half's X overlaps the first half's layer, and the copy
+  // of the first half's output overlaps the second half's layer. With capacity the positions
+  // depend on the whole batch, which then runs as one.
+  const bool split = p->capacity_factor <= 0.0 && p->N >= 2 * kMinHalfTokens;
+  if (!split) {
+    if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(xin, X_host, bytes, cudaMemcpyHostToDevice, s), "H2D");
+    MOE_TRY(forward_impl(*p, xin, W_r, bias, nullptr, w, xout, nullptr, nullptr, nullptr,
+                         nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, ws, s));
+    if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, s), "D2H");
+    MOE_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    return MOE_OK;
+  }
+  cudaStream_t cs = nullptr;
+  MOE_CUDA(copy_stream(&cs), "copy stream");
+  const size_t row = elem_size(*p) * static_cast<size_t>(p->D);
+  const int64_t n_half[2] = {p->N / 2, p->N - p->N / 2};
+  const int64_t t_first[2] = {0, p->N / 2};
+  cudaEvent_t ev[6] = {};  // start, in0, in1, done0, done1, out
+  moe_status st = MOE_OK;
+  for (int i = 0; i < 6 && st == MOE_OK; ++i)
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess)
+      st = fail(MOE_ERR_CUDA, "cudaEventCreateWithFlags");
+  auto step = [&](cudaError_t e, const char* what) {
+    if (st == MOE_OK && e != cudaSuccess) st = cuda_fail(e, what);
+  };
+  if (st == MOE_OK) {
+    // The copies follow whatever the caller's stream has queued before this call.
+    step(cudaEventRecord(ev[0], s), "event");
+    step(cudaStreamWaitEvent(cs, ev[0], 0), "wait");
+    for (int h = 0; h < 2; ++h) {
+      step(cudaMemcpyAsync(static_cast<uint8_t*>(xin) + t_first[h] * row,
+                           static_cast<const uint8_t*>(X_host) + t_first[h] * row,
+                           n_half[h] * row, cudaMemcpyHostToDevice, cs),
+           "H2D");
+      step(cudaEventRecord(ev[1 + h], cs), "event");
+    }
+    for (int h = 0; h < 2 && st == MOE_OK; ++h) {
+      moe_problem ph = *p;
+      ph.N = n_half[h];
+      step(cudaStreamWaitEvent(s, ev[1 + h], 0), "wait");
+      if (st == MOE_OK)
+        st = forward_impl(ph, static_cast<uint8_t*>(xin) + t_first[h] * row, W_r, bias, nullptr,
+                          w, static_cast<uint8_t*>(xout) + t_first[h] * row, nullptr, nullptr,
+                          nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, ws, s);
+      step(cudaEventRecord(ev[3 + h], s), "event");
+      step(cudaStreamWaitEvent(cs, ev[3 + h], 0), "wait");
+      step(cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + t_first[h] * row,
+                           static_cast<const uint8_t*>(xout) + t_first[h] * row, n_half[h] * row,
+                           cudaMemcpyDeviceToHost, cs),
+           "D2H");
+    }
+    step(cudaEventRecord(ev[5], cs), "event");
+    step(cudaStreamWaitEvent(s, ev[5], 0), "wait");
+    step(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  }
+  for (int i = 0; i < 6; ++i)
+    if (ev[i] != nullptr) cudaEventDestroy(ev[i]);
+  return st;
 }
 
 moe_status moe_expert_up_w8(const moe_problem* p, const void* X_perm, const int32_t* offsets,

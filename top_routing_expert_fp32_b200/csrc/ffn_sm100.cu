@@ -480,7 +480,9 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 }
 
 // Tile shape: CTA pairs (256-row tiles) pay off when experts hold many rows; 128-row tiles
-// waste less on small or capacity-limited experts. MOE_GEMM_TILE_ROWS=128|256 overrides.
+// waste less on small or skewed experts. Without capacity the routing of a large batch is
+// close to balanced, so R/E >= 384 rows already fill pair tiles; under a capacity the per-expert
+// counts are skewed below the cap, and pairs need 768. MOE_GEMM_TILE_ROWS=128|256 overrides.
 bool use_pairs(const moe_problem& p) {
   if (const char* env = std::getenv("MOE_GEMM_TILE_ROWS")) {
     if (std::strcmp(env, "256") == 0) return true;
@@ -493,7 +495,7 @@ bool use_pairs(const moe_problem& p) {
                                                      static_cast<double>(p.k) / static_cast<double>(p.E)));
     per_expert = std::min(per_expert, C);
   }
-  return per_expert >= 768;
+  return per_expert >= (p.capacity_factor > 0.0 ? 768 : 384);
 }
 
 // Column blocks per tile group. Experts that hold many rows (CTA-pair tiles) keep the
