@@ -45,7 +45,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_desc(cfg, w8: bool = False) -> str:
+def workload_desc(cfg, w8: bool = False, packed: bool = False) -> str:
     act = {0: "SiLU", 1: "GELU(erf)", 2: "GELU(tanh)"}[cfg.activation]
     s = (f"{cfg.name}: N={cfg.N} D={cfg.D} F={cfg.F} E={cfg.E} k={cfg.k} {act} "
          f"{'renormalised' if cfg.renormalize else 'no-renorm'} top-k")
@@ -59,6 +59,8 @@ def workload_desc(cfg, w8: bool = False) -> str:
         s += ", kept gates renormalised on drops"
     if w8:
         s += ", 8-bit expert weights (fp32 scale per expert and output column)"
+        if packed:
+            s += ", repacked K-contiguous at load time"
     return s
 
 
@@ -242,12 +244,26 @@ def run_gpu(args, cfg, world, rank, device):
 
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
-    w8 = args.weights == "w8"
+    w8 = args.weights in ("w8", "w8p")
+    packed = args.weights == "w8p"
     inp = inputs.make_inputs(cfg, device, seed=cfg.seed + rank * 0, weights=not w8)
     wq = inputs.make_w8_weights(cfg, device) if w8 else None
     N, E, k, D, F = cfg.N, cfg.E, cfg.k, cfg.D, cfg.F
     p = abi.problem(cfg)
     ws = abi.workspace(p, device)
+    if packed:
+        # Load-time repacking (outside every timed region): K-contiguous copies, scales shared.
+        W1p = torch.empty((E, F, D), dtype=torch.int8, device=device)
+        W2p = torch.empty_like(W1p)
+        W3p = torch.empty((E, D, F), dtype=torch.int8, device=device)
+        abi.pack_w8(p, wq.W1q, wq.W2q, wq.W3q, W1p, W2p, W3p)
+        wq = inputs.MoEWeights8(W1p, wq.S1, W2p, wq.S2, W3p, wq.S3)
+        torch.cuda.synchronize(device)
+    # 8-bit weights: the transposed tensor-memory-operand kernel when packed or when the
+    # experts hold few rows (N k <= 64 E), else the shared-memory one.
+    w8_kernel = ("grouped_gemm_w8t" if packed or N * k <= 64 * E else "grouped_gemm_w8")
+    up_kernel = (f"{w8_kernel}<dual{', K-contiguous' if packed else ''}>" if w8
+                 else "grouped_gemm_sm100<dual>")
     tdt = inp.X.dtype
     R = N * k
     logits = None
@@ -284,12 +300,16 @@ def run_gpu(args, cfg, world, rank, device):
         ev[1].record(stream)
         abi.dispatch(p, inp.X, idx, load, offsets, pos, dropped, row_token, X_perm, ws)
         ev[2].record(stream)
-        if w8:
+        if packed:
+            abi.expert_up_w8p(p, X_perm, offsets, wq.W1q, wq.S1, wq.W2q, wq.S2, H, ws)
+        elif w8:
             abi.expert_up_w8(p, X_perm, offsets, wq.W1q, wq.S1, wq.W2q, wq.S2, H, ws)
         else:
             abi.expert_up(p, X_perm, offsets, inp.W1, inp.W2, H, ws)
         ev[3].record(stream)
-        if w8:
+        if packed:
+            abi.expert_down_w8p(p, H, offsets, wq.W3q, wq.S3, Y, ws)
+        elif w8:
             abi.expert_down_w8(p, H, offsets, wq.W3q, wq.S3, Y, ws)
         else:
             abi.expert_down(p, H, offsets, inp.W3, Y, ws)
@@ -368,14 +388,13 @@ def run_gpu(args, cfg, world, rank, device):
     dom = "up"
     psrc = (f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback")
     if t_tensor >= t_hbm:
-        roof = {"kernel": ("grouped_gemm_w8<dual>" if w8 else "grouped_gemm_sm100<dual>")
-                + " (expert up-projection + gating)",
+        roof = {"kernel": up_kernel + " (expert up-projection + gating)",
                 "bound": "tensor", "achieved": kern["up"]["TFLOP/s"], "peak": tc,
                 "unit": "TFLOP/s", "frac": kern["up"]["TFLOP/s"] / tc,
                 "peak_source": psrc + ", bf16 burst", "flops_per_launch": flops_up}
     else:
         gbs = bytes_up / mean["up"] / 1e6
-        roof = {"kernel": ("grouped_gemm_w8<dual>" if w8 else "grouped_gemm_sm100<dual>")
+        roof = {"kernel": up_kernel
                 + " (expert up-projection; bound by streaming the used experts' weights)",
                 "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                 "frac": gbs / hbm, "peak_source": psrc, "bytes_per_launch": bytes_up}
@@ -387,7 +406,8 @@ def run_gpu(args, cfg, world, rank, device):
         t_min = max(fl / (tc * 1e12) if cfg.dtype == configs.DTYPE_BF16 else 0.0,
                     by / (hbm * 1e9))
         kern[n]["frac_roofline"] = t_min * 1e3 / mean[n]
-    roof["traffic"] = traffic_from_profile("up_w8" if w8 else "up", cfg.name)
+    roof["traffic"] = traffic_from_profile(
+        ("up_w8p" if packed else "up_w8" if w8 else "up"), cfg.name)
 
     # end-to-end through the public entry points, host X in and host out inside the timed
     # region: moe_forward_host (bf16 weights; it copies and synchronises itself) or, for 8-bit
@@ -401,7 +421,7 @@ def run_gpu(args, cfg, world, rank, device):
     def e2e_call():
         if w8:
             xd.copy_(xh, non_blocking=True)
-            abi.forward_w8(p, xd, inp.W_r, inp.bias, wq, od, ws)
+            abi.forward_w8(p, xd, inp.W_r, inp.bias, wq, od, ws, packed=packed)
             oh.copy_(od, non_blocking=True)
         else:
             abi.forward_host(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws_h)
@@ -433,7 +453,7 @@ def run_gpu(args, cfg, world, rank, device):
         "dtype": dtype_name(cfg),
         "data": "synthetic, seeded: X~N(0,1), W_r/W1/W2~N(0,1/D), W3~N(0,1/F)"
                 + (", bias~N(0,2)" if cfg.router_bias_var > 0 else ""),
-        "config": {"workload": workload_desc(cfg, w8), "tokens_per_gpu": N,
+        "config": {"workload": workload_desc(cfg, w8, packed), "tokens_per_gpu": N,
                    "expert_weights": "int8 + fp32 scale per expert and output column" if w8
                    else dtype_name(cfg),
                    "parallelism": f"replicas x{world} (no data-path collective)",
@@ -445,7 +465,8 @@ def run_gpu(args, cfg, world, rank, device):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "api": ("moe_forward_w8 between pinned-host copies of X and out" if w8 else
+                "api": (f"moe_forward_w8{'p' if packed else ''} between pinned-host copies of"
+                        " X and out" if w8 else
                         "moe_forward_host (pinned host X in, host out)")
                        + "; copies in the timed region"},
         "gpu_launches": sum(launches.values()) * args.steps,
@@ -467,7 +488,7 @@ def main():
                     help="override N (smaller cases for profiling)")
     ap.add_argument("--ffn", type=int, default=None,
                     help="override F (smaller weight footprint for profiling)")
-    ap.add_argument("--weights", default="bf16", choices=["bf16", "w8"],
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "w8", "w8p"],
                     help="expert weights: bf16, or int8 with per-column fp32 scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -485,13 +506,14 @@ def main():
         if rank != 0:
             return 0
         cb = oracle_tokens_per_s(cfg, budget_s=min(20.0, 6.0 * args.steps),
-                                 w8=args.weights == "w8")
+                                 w8=args.weights != "bf16")
         line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * cfg.N / cb["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic, seeded (same inputs as the GPU arm)",
-                "config": {"workload": workload_desc(cfg, args.weights == "w8")},
+                "config": {"workload": workload_desc(cfg, args.weights != "bf16",
+                                                     args.weights == "w8p")},
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -508,7 +530,7 @@ def main():
     line = run_gpu(args, cfg, world, rank, device)
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = oracle_tokens_per_s(cfg, w8=args.weights == "w8")
+            line["cpu_baseline"] = oracle_tokens_per_s(cfg, w8=args.weights != "bf16")
         else:
             line["cpu_baseline"] = None
         print(json.dumps(line))

@@ -277,6 +277,32 @@ moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
                           int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
                           float* prob_colsum, void* ws, size_t ws_bytes, void* stream);
 
+/* Load-time repacking of the 8-bit expert weights with the reduction dimension contiguous:
+ * W1p, W2p [E,F,D] from W1q, W2q [E,D,F]; W3p [E,D,F] from W3q [E,F,D] (an exact byte
+ * transpose of each expert's matrix, Wp[e][n][k] = Wq[e][k][n]). Same shape rules as
+ * moe_expert_up_w8; the caller owns all six device buffers (16-byte aligned, no overlap).
+ * Enqueued on `stream`; returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_CUDA. */
+moe_status moe_pack_w8(const moe_problem* p, const int8_t* W1q, const int8_t* W2q,
+                       const int8_t* W3q, int8_t* W1p, int8_t* W2p, int8_t* W3p, void* stream);
+/* moe_expert_up_w8 / moe_expert_down_w8 / moe_forward_w8 on weights repacked by moe_pack_w8
+ * (scales unchanged). Same results: each output element is the same fp32 sum of the same
+ * products, taken by the kernel that computes each expert transposed (weights as the
+ * tensor-memory operand), which is also the one the unpacked entry points pick for
+ * decode-sized batches. */
+moe_status moe_expert_up_w8p(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                             const int8_t* W1p, const float* S1, const int8_t* W2p,
+                             const float* S2, void* H, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_expert_down_w8p(const moe_problem* p, const void* H, const int32_t* offsets,
+                               const int8_t* W3p, const float* S3, void* Y, void* ws,
+                               size_t ws_bytes, void* stream);
+moe_status moe_forward_w8p(const moe_problem* p, const void* X, const float* W_r,
+                           const float* bias, const int8_t* W1p, const float* S1,
+                           const int8_t* W2p, const float* S2, const int8_t* W3p,
+                           const float* S3, void* out, float* logits, int32_t* topk_idx,
+                           float* topk_gate, int32_t* load, int32_t* offsets, int32_t* pos,
+                           uint8_t* dropped, float* prob_colsum, void* ws, size_t ws_bytes,
+                           void* stream);
+
 /* moe_forward with the training-time selection variants (p->routing_mode, noise as in
  * moe_route_ex) and the optional z_loss output. */
 moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,

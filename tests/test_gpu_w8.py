@@ -1,6 +1,6 @@
 """GPU parity of the 8-bit expert-weight path (moe_expert_up_w8 / moe_expert_down_w8 /
-moe_forward_w8) against the oracle's fp64 dequantized experts (W = q * s per expert and output
-column; Grok-1 book 5.3.3, 5.3.5)."""
+moe_forward_w8, and their K-contiguous variants after moe_pack_w8) against the oracle's fp64
+dequantized experts (W = q * s per expert and output column; Grok-1 book 5.3.3, 5.3.5)."""
 import math
 
 import numpy as np
@@ -25,7 +25,18 @@ def _cfg(N, D, F, E, k=1, act=configs.ACT_SILU, **kw):
                              activation=act, renormalize=1, **kw)
 
 
-def _ffn_w8(abi, counts, D, F, act, seed=0):
+def _packed(abi, p, w):
+    """The K-contiguous copies of w's 8-bit matrices (moe_pack_w8), scales shared."""
+    W1p = torch.empty(w.W1q.shape[0], w.W1q.shape[2], w.W1q.shape[1], dtype=torch.int8,
+                      device="cuda")
+    W2p = torch.empty_like(W1p)
+    W3p = torch.empty(w.W3q.shape[0], w.W3q.shape[2], w.W3q.shape[1], dtype=torch.int8,
+                      device="cuda")
+    abi.pack_w8(p, w.W1q, w.W2q, w.W3q, W1p, W2p, W3p)
+    return inputs.MoEWeights8(W1p, w.S1, W2p, w.S2, W3p, w.S3)
+
+
+def _ffn_w8(abi, counts, D, F, act, seed=0, packed=False):
     E = len(counts)
     R = int(sum(counts))
     cfg = _cfg(max(R, 1), D, F, E, act=act)
@@ -37,8 +48,13 @@ def _ffn_w8(abi, counts, D, F, act, seed=0):
     ws = abi.workspace(p)
     H = torch.full((max(R, 1), F), float("nan"), dtype=torch.bfloat16, device="cuda")
     Y = torch.full((max(R, 1), D), float("nan"), dtype=torch.bfloat16, device="cuda")
-    abi.expert_up_w8(p, Xp, offsets, w.W1q, w.S1, w.W2q, w.S2, H, ws)
-    abi.expert_down_w8(p, H, offsets, w.W3q, w.S3, Y, ws)
+    if packed:
+        wp = _packed(abi, p, w)
+        abi.expert_up_w8p(p, Xp, offsets, wp.W1q, wp.S1, wp.W2q, wp.S2, H, ws)
+        abi.expert_down_w8p(p, H, offsets, wp.W3q, wp.S3, Y, ws)
+    else:
+        abi.expert_up_w8(p, Xp, offsets, w.W1q, w.S1, w.W2q, w.S2, H, ws)
+        abi.expert_down_w8(p, H, offsets, w.W3q, w.S3, Y, ws)
     torch.cuda.synchronize()
     assert abi.device_error(ws) == 0
     return cfg, Xp, w, offsets, H, Y, R
@@ -52,8 +68,13 @@ def _ffn_w8(abi, counts, D, F, act, seed=0):
     ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
     ([700, 0, 257, 1100], 512, 400, configs.ACT_GELU_ERF),
 ])
-def test_expert_ffn_w8_matches_oracle(abi, counts, D, F, act):
-    cfg, Xp, w, offsets, H, Y, R = _ffn_w8(abi, counts, D, F, act)
+@pytest.mark.parametrize("kernel", ["smem", "tmem", "packed"])
+def test_expert_ffn_w8_matches_oracle(abi, monkeypatch, counts, D, F, act, kernel):
+    # smem: converted weights in shared memory (larger batches); tmem: transposed product with
+    # the converted weights as the tensor-memory operand (few rows per expert); packed: the
+    # tmem kernel on K-contiguous weights from moe_pack_w8.
+    monkeypatch.setenv("MOE_W8_KERNEL", "tmem" if kernel == "packed" else kernel)
+    cfg, Xp, w, offsets, H, Y, R = _ffn_w8(abi, counts, D, F, act, packed=kernel == "packed")
     rec_e = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
     ref = oracle.expert_ffn_w8(np.arange(R, dtype=np.int32), rec_e, np_host(Xp), oracle.BF16,
                                w.W1q.cpu().numpy(), w.S1.cpu().numpy(), w.W2q.cpu().numpy(),
@@ -66,6 +87,7 @@ def test_unit_scales_reproduce_bf16_kernel_bit_for_bit(abi, monkeypatch):
     # int8 -> bf16 is exact and a unit scale is exact, so with the same 128-row tiles the 8-bit
     # path must give the bf16 path's bits on W = q.
     monkeypatch.setenv("MOE_GEMM_TILE_ROWS", "128")
+    monkeypatch.setenv("MOE_W8_KERNEL", "smem")
     counts, D, F = [129, 3, 200, 64], 256, 384
     cfg, Xp, w, offsets, H8, Y8, R = _ffn_w8(abi, counts, D, F, configs.ACT_SILU, seed=4)
     p = abi.problem(cfg)
@@ -85,6 +107,35 @@ def test_unit_scales_reproduce_bf16_kernel_bit_for_bit(abi, monkeypatch):
     assert torch.equal(Y1[:R].view(torch.int16), Yb[:R].view(torch.int16))
 
 
+@pytest.mark.parametrize("E,k,n", [(1, 16, 16), (3, 80, 208), (2, 4096, 48), (5, 1040, 336)])
+def test_pack_w8_is_exact_transpose(abi, E, k, n):
+    # W1q/W2q are [E, D, F] (k = D rows), W3q is [E, F, D]: moe_pack_w8 transposes each
+    # expert's matrix, ragged 32 x 32 tiles included, byte for byte.
+    cfg = _cfg(16, k, n, E)
+    p = abi.problem(cfg)
+    g = torch.Generator(device="cuda").manual_seed(E * 7 + k + n)
+    rnd = lambda *sh: torch.randint(-128, 128, sh, generator=g, device="cuda",
+                                    dtype=torch.int32).to(torch.int8)
+    w = inputs.MoEWeights8(rnd(E, k, n), None, rnd(E, k, n), None, rnd(E, n, k), None)
+    wp = _packed(abi, p, w)
+    torch.cuda.synchronize()
+    assert torch.equal(wp.W1q, w.W1q.transpose(1, 2))
+    assert torch.equal(wp.W2q, w.W2q.transpose(1, 2))
+    assert torch.equal(wp.W3q, w.W3q.transpose(1, 2))
+
+
+def test_packed_reproduces_tmem_kernel_bit_for_bit(abi, monkeypatch):
+    # The same bf16 values of q enter the same MMAs in the same order, only the staging layout
+    # differs, so H and Y match the unpacked tensor-memory kernel bit for bit.
+    monkeypatch.setenv("MOE_W8_KERNEL", "tmem")
+    counts, D, F = [0, 65, 3, 130, 64, 1], 336, 208
+    _, _, _, _, Hu, Yu, R = _ffn_w8(abi, counts, D, F, configs.ACT_GELU_TANH, seed=9)
+    _, _, _, _, Hp, Yp, _ = _ffn_w8(abi, counts, D, F, configs.ACT_GELU_TANH, seed=9,
+                                    packed=True)
+    assert torch.equal(Hu[:R].view(torch.int16), Hp[:R].view(torch.int16))
+    assert torch.equal(Yu[:R].view(torch.int16), Yp[:R].view(torch.int16))
+
+
 def test_w8_rejected_without_bf16_or_16_multiples(abi):
     from top_routing_expert_fp32_b200.abi import MoEError
     cfg = _cfg(64, 24, 64, 4)           # D % 16 != 0
@@ -96,16 +147,18 @@ def test_w8_rejected_without_bf16_or_16_multiples(abi):
         abi.expert_up_w8(p, f, t, t, f, t, f, f, ws)
 
 
-def _forward_w8_check(abi, cfg, sample=None):
+def _forward_w8_check(abi, cfg, sample=None, packed=False):
     inp = inputs.make_inputs(cfg, "cuda", weights=False)
     w = inputs.make_w8_weights(cfg, "cuda")
     p = abi.problem(cfg)
     ws = abi.workspace(p)
+    wk = _packed(abi, p, w) if packed else w
     N, E, k = cfg.N, cfg.E, cfg.k
     idx = torch.empty((N, k), dtype=torch.int32, device="cuda")
     dropped = torch.empty((N, k), dtype=torch.uint8, device="cuda")
     out = torch.empty((N, cfg.D), dtype=torch.bfloat16, device="cuda")
-    abi.forward_w8(p, inp.X, inp.W_r, inp.bias, w, out, ws, topk_idx=idx, dropped=dropped)
+    abi.forward_w8(p, inp.X, inp.W_r, inp.bias, wk, out, ws, topk_idx=idx, dropped=dropped,
+                   packed=packed)
     torch.cuda.synchronize()
     assert abi.device_error(ws) == 0
     Xn = np_host(inp.X)
@@ -143,14 +196,16 @@ def _forward_w8_check(abi, cfg, sample=None):
     _cfg(500, 128, 256, 16, k=2, capacity_factor=1.0, router_bias_var=2.0),
     _cfg(257, 384, 640, 8, k=2, act=configs.ACT_GELU_ERF).with_(renormalize=0),
 ], ids=["silu_e8", "capacity_e16", "gelu_norenorm"])
-def test_forward_w8_small_all_tokens(abi, cfg):
-    n, flips = _forward_w8_check(abi, cfg)
+@pytest.mark.parametrize("packed", [False, True], ids=["kn", "packed"])
+def test_forward_w8_small_all_tokens(abi, cfg, packed):
+    n, flips = _forward_w8_check(abi, cfg, packed=packed)
     assert n >= cfg.N - 2 * flips - 8
 
 
-@pytest.mark.parametrize("name", ["decode", "mixtral"])
-def test_forward_w8_full_size_sampled(abi, name):
+@pytest.mark.parametrize("name,packed", [("decode", False), ("mixtral", False),
+                                         ("decode", True)])
+def test_forward_w8_full_size_sampled(abi, name, packed):
     cfg = configs.CONFIGS[name]
     sample = sorted(set(np.linspace(0, cfg.N - 1, 12).astype(int).tolist()))
-    _forward_w8_check(abi, cfg, sample)
+    _forward_w8_check(abi, cfg, sample, packed=packed)
     torch.cuda.empty_cache()

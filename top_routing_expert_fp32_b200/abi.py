@@ -26,6 +26,7 @@ EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_workspace_size_host", "moe
            "moe_route_ex", "moe_dispatch", "moe_dispatch_noalloc", "moe_expert_ffn",
            "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_ex",
            "moe_forward_host", "moe_expert_up_w8", "moe_expert_down_w8", "moe_forward_w8",
+           "moe_pack_w8", "moe_expert_up_w8p", "moe_expert_down_w8p", "moe_forward_w8p",
            "moe_workspace_init", "moe_get_device_error", "moe_status_string", "moe_last_error",
            "moe_version")
 
@@ -71,6 +72,10 @@ def _load() -> ctypes.CDLL:
         "moe_expert_up_w8": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_down_w8": [PP, P, P, P, P, P, P, S, P],
         "moe_forward_w8": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
+        "moe_pack_w8": [PP, P, P, P, P, P, P, P],
+        "moe_expert_up_w8p": [PP, P, P, P, P, P, P, P, P, S, P],
+        "moe_expert_down_w8p": [PP, P, P, P, P, P, P, S, P],
+        "moe_forward_w8p": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "moe_workspace_init": [P, S, P],
         "moe_get_device_error": [P, P, ctypes.POINTER(ctypes.c_int32)],
     }
@@ -214,10 +219,29 @@ def expert_down_w8(p, H, offsets, W3q, S3, Y, ws, stream=None):
                                   _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def pack_w8(p, W1q, W2q, W3q, W1p, W2p, W3p, stream=None):
+    _check(lib.moe_pack_w8(ctypes.byref(p), _ptr(W1q), _ptr(W2q), _ptr(W3q), _ptr(W1p),
+                           _ptr(W2p), _ptr(W3p), _stream(stream)))
+
+
+def expert_up_w8p(p, X_perm, offsets, W1p, S1, W2p, S2, H, ws, stream=None):
+    _check(lib.moe_expert_up_w8p(ctypes.byref(p), _ptr(X_perm), _ptr(offsets), _ptr(W1p),
+                                 _ptr(S1), _ptr(W2p), _ptr(S2), _ptr(H), _ptr(ws), ws.numel(),
+                                 _stream(stream)))
+
+
+def expert_down_w8p(p, H, offsets, W3p, S3, Y, ws, stream=None):
+    _check(lib.moe_expert_down_w8p(ctypes.byref(p), _ptr(H), _ptr(offsets), _ptr(W3p), _ptr(S3),
+                                   _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def forward_w8(p, X, W_r, bias, w8, out, ws, *, logits=None, topk_idx=None, topk_gate=None,
-               load=None, offsets=None, pos=None, dropped=None, prob_colsum=None, stream=None):
-    """w8: an object with W1q, S1, W2q, S2, W3q, S3 (e.g. inputs.MoEWeights8)."""
-    _check(lib.moe_forward_w8(ctypes.byref(p), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(w8.W1q),
+               load=None, offsets=None, pos=None, dropped=None, prob_colsum=None, packed=False,
+               stream=None):
+    """w8: an object with W1q, S1, W2q, S2, W3q, S3 (e.g. inputs.MoEWeights8); packed=True:
+    its W1q, W2q, W3q are the K-contiguous copies written by pack_w8 (moe_forward_w8p)."""
+    fn = lib.moe_forward_w8p if packed else lib.moe_forward_w8
+    _check(fn(ctypes.byref(p), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(w8.W1q),
                               _ptr(w8.S1), _ptr(w8.W2q), _ptr(w8.S2), _ptr(w8.W3q), _ptr(w8.S3),
                               _ptr(out), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
                               _ptr(load), _ptr(offsets), _ptr(pos), _ptr(dropped),

@@ -231,8 +231,49 @@ struct Experts {
   const float* S1 = nullptr;
   const float* S2 = nullptr;
   const float* S3 = nullptr;
+  bool packed = false;  // 8-bit weights K-contiguous (moe_pack_w8)
   bool w8() const { return Q1 != nullptr; }
 };
+
+// 8-bit experts: the tensor-memory-operand kernel for experts with few rows (decode-sized
+// batches, R/E <= 64), the shared-memory kernel otherwise. MOE_W8_KERNEL=tmem|smem overrides.
+bool use_w8t(const moe_problem& p) {
+  if (const char* env = std::getenv("MOE_W8_KERNEL")) {
+    if (std::strcmp(env, "tmem") == 0) return true;
+    if (std::strcmp(env, "smem") == 0) return false;
+  }
+  return p.N * p.k <= 64 * static_cast<int64_t>(p.E);
+}
+
+// packed: K-contiguous weights from moe_pack_w8 (always the tensor-memory-operand kernel).
+moe_status run_up_w8(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                     const int8_t* Q1, const float* S1, const int8_t* Q2, const float* S2,
+                     void* H, bool packed, int* err, cudaStream_t stream) {
+  MOE_TRY(check_sm100());
+  if (packed || use_w8t(p))
+    MOE_CUDA(launch_ffn_up_w8t(p, X_perm, offsets, Q1, S1, Q2, S2, H, packed, err,
+                               wait_timeout_ns(), stream),
+             "expert up-projection, 8-bit weights (tcgen05, TMEM operand)");
+  else
+    MOE_CUDA(launch_ffn_up_w8(p, X_perm, offsets, Q1, S1, Q2, S2, H, err, wait_timeout_ns(),
+                              stream),
+             "expert up-projection, 8-bit weights (tcgen05)");
+  return MOE_OK;
+}
+
+moe_status run_down_w8(const moe_problem& p, const void* H, const int32_t* offsets,
+                       const int8_t* Q3, const float* S3, void* Y, bool packed, int* err,
+                       cudaStream_t stream) {
+  MOE_TRY(check_sm100());
+  if (packed || use_w8t(p))
+    MOE_CUDA(launch_ffn_down_w8t(p, H, offsets, Q3, S3, Y, packed, err, wait_timeout_ns(),
+                                 stream),
+             "expert down-projection, 8-bit weights (tcgen05, TMEM operand)");
+  else
+    MOE_CUDA(launch_ffn_down_w8(p, H, offsets, Q3, S3, Y, err, wait_timeout_ns(), stream),
+             "expert down-projection, 8-bit weights (tcgen05)");
+  return MOE_OK;
+}
 
 moe_status run_ffn(const moe_problem& p, const void* X_perm, const int32_t* offsets,
                    const Experts& w, void* H, void* Y, int* err, cudaStream_t stream) {
@@ -240,13 +281,8 @@ moe_status run_ffn(const moe_problem& p, const void* X_perm, const int32_t* offs
     MOE_TRY(run_up(p, X_perm, offsets, w.W1, w.W2, H, err, stream));
     return run_down(p, H, offsets, w.W3, Y, err, stream);
   }
-  MOE_TRY(check_sm100());
-  MOE_CUDA(launch_ffn_up_w8(p, X_perm, offsets, w.Q1, w.S1, w.Q2, w.S2, H, err,
-                            wait_timeout_ns(), stream),
-           "expert up-projection, 8-bit weights (tcgen05)");
-  MOE_CUDA(launch_ffn_down_w8(p, H, offsets, w.Q3, w.S3, Y, err, wait_timeout_ns(), stream),
-           "expert down-projection, 8-bit weights (tcgen05)");
-  return MOE_OK;
+  MOE_TRY(run_up_w8(p, X_perm, offsets, w.Q1, w.S1, w.Q2, w.S2, H, w.packed, err, stream));
+  return run_down_w8(p, H, offsets, w.Q3, w.S3, Y, w.packed, err, stream);
 }
 
 // Extra shape rule of the 8-bit expert path: bf16 activations, and D, F multiples of 16
@@ -671,12 +707,9 @@ moe_status moe_expert_up_w8(const moe_problem* p, const void* X_perm, const int3
   MOE_TRY(need(S2, "S2"));
   MOE_TRY(need(H, "H"));
   if (p->N == 0) return MOE_OK;
-  MOE_TRY(check_sm100());
   const Layout L = make_layout(*p);
-  MOE_CUDA(launch_ffn_up_w8(*p, X_perm, offsets, W1q, S1, W2q, S2, H, at<int>(ws, L.err),
-                            wait_timeout_ns(), static_cast<cudaStream_t>(stream)),
-           "expert up-projection, 8-bit weights (tcgen05)");
-  return MOE_OK;
+  return run_up_w8(*p, X_perm, offsets, W1q, S1, W2q, S2, H, false, at<int>(ws, L.err),
+                   static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_expert_down_w8(const moe_problem* p, const void* H, const int32_t* offsets,
@@ -691,20 +724,22 @@ moe_status moe_expert_down_w8(const moe_problem* p, const void* H, const int32_t
   MOE_TRY(need(S3, "S3"));
   MOE_TRY(need(Y, "Y"));
   if (p->N == 0) return MOE_OK;
-  MOE_TRY(check_sm100());
   const Layout L = make_layout(*p);
-  MOE_CUDA(launch_ffn_down_w8(*p, H, offsets, W3q, S3, Y, at<int>(ws, L.err), wait_timeout_ns(),
-                              static_cast<cudaStream_t>(stream)),
-           "expert down-projection, 8-bit weights (tcgen05)");
-  return MOE_OK;
+  return run_down_w8(*p, H, offsets, W3q, S3, Y, false, at<int>(ws, L.err),
+                     static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
-                          const float* bias, const int8_t* W1q, const float* S1,
-                          const int8_t* W2q, const float* S2, const int8_t* W3q, const float* S3,
-                          void* out, float* logits, int32_t* topk_idx, float* topk_gate,
-                          int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
-                          float* prob_colsum, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+moe_status forward_w8_impl(const moe_problem* p, const void* X, const float* W_r,
+                           const float* bias, const int8_t* W1q, const float* S1,
+                           const int8_t* W2q, const float* S2, const int8_t* W3q,
+                           const float* S3, void* out, float* logits, int32_t* topk_idx,
+                           float* topk_gate, int32_t* load, int32_t* offsets, int32_t* pos,
+                           uint8_t* dropped, float* prob_colsum, void* ws, size_t ws_bytes,
+                           void* stream, bool packed) {
   MOE_TRY(check_problem(p));
   MOE_TRY(check_w8(*p));
   MOE_TRY(check_ws(*p, ws, ws_bytes, false));
@@ -733,10 +768,92 @@ moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
   w.S1 = S1;
   w.S2 = S2;
   w.S3 = S3;
+  w.packed = packed;
   MOE_TRY(need_topk(*p));
   return forward_impl(*p, X, W_r, bias, nullptr, w, out, logits, topk_idx, topk_gate, load,
                       offsets, pos, dropped, prob_colsum, nullptr, ws,
                       static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward_w8(const moe_problem* p, const void* X, const float* W_r,
+                          const float* bias, const int8_t* W1q, const float* S1,
+                          const int8_t* W2q, const float* S2, const int8_t* W3q, const float* S3,
+                          void* out, float* logits, int32_t* topk_idx, float* topk_gate,
+                          int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
+                          float* prob_colsum, void* ws, size_t ws_bytes, void* stream) {
+  return forward_w8_impl(p, X, W_r, bias, W1q, S1, W2q, S2, W3q, S3, out, logits, topk_idx,
+                         topk_gate, load, offsets, pos, dropped, prob_colsum, ws, ws_bytes,
+                         stream, false);
+}
+
+moe_status moe_forward_w8p(const moe_problem* p, const void* X, const float* W_r,
+                           const float* bias, const int8_t* W1p, const float* S1,
+                           const int8_t* W2p, const float* S2, const int8_t* W3p,
+                           const float* S3, void* out, float* logits, int32_t* topk_idx,
+                           float* topk_gate, int32_t* load, int32_t* offsets, int32_t* pos,
+                           uint8_t* dropped, float* prob_colsum, void* ws, size_t ws_bytes,
+                           void* stream) {
+  return forward_w8_impl(p, X, W_r, bias, W1p, S1, W2p, S2, W3p, S3, out, logits, topk_idx,
+                         topk_gate, load, offsets, pos, dropped, prob_colsum, ws, ws_bytes,
+                         stream, true);
+}
+
+moe_status moe_pack_w8(const moe_problem* p, const int8_t* W1q, const int8_t* W2q,
+                       const int8_t* W3q, int8_t* W1p, int8_t* W2p, int8_t* W3p, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_w8(*p));
+  MOE_TRY(need(W1q, "W1q"));
+  MOE_TRY(need(W2q, "W2q"));
+  MOE_TRY(need(W3q, "W3q"));
+  MOE_TRY(need(W1p, "W1p"));
+  MOE_TRY(need(W2p, "W2p"));
+  MOE_TRY(need(W3p, "W3p"));
+  MOE_TRY(check_sm100());
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(launch_pack_w8(W1q, W1p, p->E, p->D, p->F, s), "pack W1");
+  MOE_CUDA(launch_pack_w8(W2q, W2p, p->E, p->D, p->F, s), "pack W2");
+  MOE_CUDA(launch_pack_w8(W3q, W3p, p->E, p->F, p->D, s), "pack W3");
+  return MOE_OK;
+}
+
+moe_status moe_expert_up_w8p(const moe_problem* p, const void* X_perm, const int32_t* offsets,
+                             const int8_t* W1p, const float* S1, const int8_t* W2p,
+                             const float* S2, void* H, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_w8(*p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(X_perm, "X_perm"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W1p, "W1p"));
+  MOE_TRY(need(S1, "S1"));
+  MOE_TRY(need(W2p, "W2p"));
+  MOE_TRY(need(S2, "S2"));
+  MOE_TRY(need(H, "H"));
+  if (p->N == 0) return MOE_OK;
+  const Layout L = make_layout(*p);
+  return run_up_w8(*p, X_perm, offsets, W1p, S1, W2p, S2, H, true, at<int>(ws, L.err),
+                   static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_down_w8p(const moe_problem* p, const void* H, const int32_t* offsets,
+                               const int8_t* W3p, const float* S3, void* Y, void* ws,
+                               size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  MOE_TRY(check_w8(*p));
+  MOE_TRY(check_ws(*p, ws, ws_bytes, false));
+  MOE_TRY(need(H, "H"));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(W3p, "W3p"));
+  MOE_TRY(need(S3, "S3"));
+  MOE_TRY(need(Y, "Y"));
+  if (p->N == 0) return MOE_OK;
+  const Layout L = make_layout(*p);
+  return run_down_w8(*p, H, offsets, W3p, S3, Y, true, at<int>(ws, L.err),
+                     static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {

@@ -554,6 +554,19 @@ bool make_tensor_map_3d_u8(CUtensorMap* m, const void* ptr, uint64_t n, uint64_t
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tensor_map_3d_u8_sw64(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                                uint64_t E, uint32_t box_inner, uint32_t box_rows) {
+  if (encode_fn() == nullptr) return false;
+  const cuuint64_t dims[3] = {inner, rows, E};
+  const cuuint64_t strides[2] = {inner, inner * rows};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
                                 const void* W1, const void* W2, void* H, int* err,
                                 uint64_t timeout_ns, cudaStream_t stream) {

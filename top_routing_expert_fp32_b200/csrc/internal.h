@@ -49,6 +49,15 @@ bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t cols, uin
 bool make_tensor_map_3d_u8(CUtensorMap* m, const void* ptr, uint64_t n, uint64_t k, uint64_t E,
                            uint32_t box_n, uint32_t box_k);
 
+// 3-D uint8 tensor map over stacked [E][rows][inner] bytes with a 64-byte swizzle (box_inner
+// must be 64): the K-contiguous (packed) 8-bit expert weights.
+bool make_tensor_map_3d_u8_sw64(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                                uint64_t E, uint32_t box_inner, uint32_t box_rows);
+
+// Repack 8-bit expert weights [E][k][n] (n contiguous) into [E][n][k] (k contiguous).
+cudaError_t launch_pack_w8(const int8_t* src, int8_t* dst, int64_t E, int64_t k, int64_t n,
+                           cudaStream_t stream);
+
 // Grouped expert GEMMs with 8-bit weights (W = q * s, s per expert and output column),
 // bf16 activations, tcgen05 tensor cores; 128-row tiles on single CTAs.
 cudaError_t launch_ffn_up_w8(const moe_problem& p, const void* X_perm, const int32_t* offsets,
@@ -58,6 +67,16 @@ cudaError_t launch_ffn_up_w8(const moe_problem& p, const void* X_perm, const int
 cudaError_t launch_ffn_down_w8(const moe_problem& p, const void* H, const int32_t* offsets,
                                const int8_t* W3q, const float* S3, void* Y, int* err,
                                uint64_t timeout_ns, cudaStream_t stream);
+// The same two GEMMs for experts holding few rows: computed transposed with the converted
+// weights as the tensor-memory operand (64-row tiles).
+// `packed`: the weights are K-contiguous ([E][n][k], from launch_pack_w8).
+cudaError_t launch_ffn_up_w8t(const moe_problem& p, const void* X_perm, const int32_t* offsets,
+                              const int8_t* W1q, const float* S1, const int8_t* W2q,
+                              const float* S2, void* H, bool packed, int* err,
+                              uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_ffn_down_w8t(const moe_problem& p, const void* H, const int32_t* offsets,
+                                const int8_t* W3q, const float* S3, void* Y, bool packed,
+                                int* err, uint64_t timeout_ns, cudaStream_t stream);
 
 // Records are processed in chunks of this many for the slot assignment.
 constexpr int kDispatchChunk = 1024;
