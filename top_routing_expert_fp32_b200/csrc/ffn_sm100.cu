@@ -28,6 +28,7 @@
 // MOE_DEVERR_WAIT_TIMEOUT, unwinds, drains its MMAs and frees its TMEM.
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -79,6 +80,8 @@ struct GemmParams {
   int K;                   // reduction length (D for GEMM1, F for GEMM2)
   int n_out;               // output columns (F for GEMM1, D for GEMM2)
   int n_group;             // column blocks per tile group (>= 1)
+  int l2_a;                // L2 eviction priority of the A rows (+1 last, 0 normal, -1 first)
+  int l2_b;                // and of the expert weights
   int* err;
   uint64_t timeout_ns;
 };
@@ -182,6 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const uint64_t pol_a = l2_policy(p.l2_a);
+      const uint64_t pol_b = l2_policy(p.l2_b);
       for (int tile = first_tile; ok && tile < total_tiles; tile += tile_stride) {
         int e, m_blk, n_blk;
         decode(tile, e, m_blk, n_blk);
@@ -200,28 +205,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Both CTAs' bytes are counted on the MMA CTA's barrier.
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (mma_cta) mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
-            tma_load_2d_pair(a_dst, &tmA, bar, k0, row0);
+            tma_load_2d_pair_hint(a_dst, &tmA, bar, k0, row0, pol_a);
             if (DUAL) {  // CTA 0 holds the W1 columns, CTA 1 the W2 columns
               const CUtensorMap* m = rank == 0 ? &tmB0 : &tmB1;
-              tma_load_3d_pair(b_dst, m, bar, n0, k0, e);
-              tma_load_3d_pair(b_dst + kBoxBytes, m, bar, n0 + 64, k0, e);
+              tma_load_3d_pair_hint(b_dst, m, bar, n0, k0, e, pol_b);
+              tma_load_3d_pair_hint(b_dst + kBoxBytes, m, bar, n0 + 64, k0, e, pol_b);
             } else {     // CTA r holds columns [n0 + 128r, n0 + 128r + 128)
               const int nc = n0 + static_cast<int>(rank) * 128;
-              tma_load_3d_pair(b_dst, &tmB0, bar, nc, k0, e);
-              tma_load_3d_pair(b_dst + kBoxBytes, &tmB0, bar, nc + 64, k0, e);
+              tma_load_3d_pair_hint(b_dst, &tmB0, bar, nc, k0, e, pol_b);
+              tma_load_3d_pair_hint(b_dst + kBoxBytes, &tmB0, bar, nc + 64, k0, e, pol_b);
             }
           } else {
             mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
-            tma_load_2d(a_dst, &tmA, &full[stage], k0, row0);
+            tma_load_2d_hint(a_dst, &tmA, &full[stage], k0, row0, pol_a);
             if (DUAL) {
-              tma_load_3d(b_dst, &tmB0, &full[stage], n0, k0, e);
-              tma_load_3d(b_dst + kBoxBytes, &tmB0, &full[stage], n0 + 64, k0, e);
-              tma_load_3d(b_dst + 2 * kBoxBytes, &tmB1, &full[stage], n0, k0, e);
-              tma_load_3d(b_dst + 3 * kBoxBytes, &tmB1, &full[stage], n0 + 64, k0, e);
+              tma_load_3d_hint(b_dst, &tmB0, &full[stage], n0, k0, e, pol_b);
+              tma_load_3d_hint(b_dst + kBoxBytes, &tmB0, &full[stage], n0 + 64, k0, e, pol_b);
+              tma_load_3d_hint(b_dst + 2 * kBoxBytes, &tmB1, &full[stage], n0, k0, e, pol_b);
+              tma_load_3d_hint(b_dst + 3 * kBoxBytes, &tmB1, &full[stage], n0 + 64, k0, e, pol_b);
             } else {
 #pragma unroll
               for (int j = 0; j < 4; ++j)
-                tma_load_3d(b_dst + j * kBoxBytes, &tmB0, &full[stage], n0 + 64 * j, k0, e);
+                tma_load_3d_hint(b_dst + j * kBoxBytes, &tmB0, &full[stage], n0 + 64 * j, k0, e,
+                                 pol_b);
             }
           }
           if (++stage == S::kStages) {
@@ -511,6 +517,21 @@ int column_group(bool pairs, int64_t n_blocks) {
   return static_cast<int>(pairs ? n_blocks : std::min<int64_t>(kGroup, n_blocks));
 }
 
+// L2 priorities of the GEMM operands: an expert's A rows are read again by every column block
+// of that expert, its weights by the few row blocks running at the same time. Default: A rows
+// evict_last, weights evict_normal. MOE_GEMM_L2=<a>,<b> (each -1, 0 or 1) overrides.
+void l2_priorities(int* a, int* b) {
+  *a = 1;
+  *b = 0;
+  if (const char* env = std::getenv("MOE_GEMM_L2")) {
+    int x = 0, y = 0;
+    if (std::sscanf(env, "%d,%d", &x, &y) == 2) {
+      *a = std::max(-1, std::min(1, x));
+      *b = std::max(-1, std::min(1, y));
+    }
+  }
+}
+
 template <bool DUAL, int ACT>
 cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUtensorMap& b0,
                          const CUtensorMap& b1, GemmParams gp, int n_tile,
@@ -518,6 +539,7 @@ cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUten
   const int64_t R = p.N * p.k;
   const int64_t n_blocks = (gp.n_out + n_tile - 1) / n_tile;
   gp.n_group = column_group(use_pairs(p), n_blocks);
+  l2_priorities(&gp.l2_a, &gp.l2_b);
   if (use_pairs(p)) {
     const int64_t tiles = ((R + 255) / 256 + p.E) * n_blocks;
     return launch_gemm<DUAL, ACT, true>(a, b0, b1, gp, tiles, stream);
