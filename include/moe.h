@@ -328,6 +328,21 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
 /* Host only. Workspace bytes for moe_forward_host. */
 moe_status moe_workspace_size_host(const moe_problem* p, size_t* bytes);
 
+/* Row gather: dst[i] = src[index[i]] for i < n_rows, rows of row_bytes bytes. The local
+ * reorder steps of expert parallelism (Grok-1 book 5.6: tokens travel by all-to-all to the
+ * device holding their expert and back; MoE series 4.1): rows received from every source rank
+ * are put in expert-major order before the expert GEMMs, and the expert outputs back in
+ * source-rank order before the return exchange. src: [n_src_rows, row_bytes] (may be NULL when
+ * n_src_rows == 0), index: [n_rows] int32, dst: [n_rows, row_bytes]; device memory, src/dst
+ * 16-byte aligned, dst not overlapping src. row_bytes: a positive multiple of 4 (16-byte
+ * words when it is a multiple of 16). An index outside [0, n_src_rows) sets
+ * MOE_DEVERR_BAD_INDEX in the workspace's error word (moe_get_device_error) and its dst row
+ * is zero-filled; nothing outside the buffers is read or written. ws: any workspace (at
+ * least 256 bytes; only its error word is used). Enqueued on `stream`. */
+moe_status moe_gather_rows(const void* src, int64_t n_src_rows, const int32_t* index,
+                           int64_t n_rows, int64_t row_bytes, void* dst, void* ws,
+                           size_t ws_bytes, void* stream);
+
 /* Zero the device error word of a new workspace (asynchronous, on `stream`). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 

@@ -1,0 +1,117 @@
+"""GPU checks of the expert-parallel pieces: moe_gather_rows (the local reorders) and
+ep.forward on this library's kernels over an NCCL group of one rank (the exchanges run as
+NCCL all-to-alls on one GPU; the multi-rank bookkeeping is covered on CPU with gloo)."""
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+import oracle
+from top_routing_expert_fp32_b200 import configs, ep, inputs
+from gpu_helpers import NEAR_TIE, TOL_BF16, normwise_rel_err, np_host, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from top_routing_expert_fp32_b200 import abi as a
+    return a
+
+
+@pytest.mark.parametrize("n_src,n,shape,dtype", [
+    (1000, 2500, (4096,), torch.bfloat16),    # 8 KB rows, repeated indices
+    (37, 37, (6,), torch.bfloat16),           # 12-byte rows: 4-byte words
+    (513, 1, (3, 8), torch.float32),          # 96-byte rows
+    (64, 0, (8,), torch.bfloat16),            # nothing to gather
+])
+def test_gather_rows_matches_indexing(abi, n_src, n, shape, dtype):
+    g = torch.Generator(device="cuda").manual_seed(n_src + n)
+    src = torch.randn((n_src,) + shape, generator=g, device="cuda").to(dtype)
+    index = torch.randint(0, n_src, (n,), generator=g, device="cuda", dtype=torch.int32)
+    dst = torch.full((max(n, 1),) + shape, float("nan"), device="cuda", dtype=dtype)[:n]
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    abi.gather_rows(src, index, dst, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    ref = src[index.long()]
+    assert torch.equal(dst.view(torch.uint8), ref.view(torch.uint8))
+
+
+def test_gather_rows_bad_index_is_reported_and_zero_filled(abi):
+    # The kernel's own bounds check turns an out-of-range index into MOE_DEVERR_BAD_INDEX and
+    # a zero row; nothing outside src is read.
+    src = torch.randn((16, 64), device="cuda").to(torch.bfloat16)
+    index = torch.tensor([3, -1, 16, 15, 2**31 - 1], dtype=torch.int32, device="cuda")
+    dst = torch.full((5, 64), 7.0, device="cuda", dtype=torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    abi.gather_rows(src, index, dst, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == abi.DEVERR_BAD_INDEX
+    assert torch.equal(dst[0], src[3]) and torch.equal(dst[3], src[15])
+    assert (dst[[1, 2, 4]].float() == 0).all()
+    assert abi.device_error(ws) == 0          # reading the error word clears it
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+@pytest.fixture(scope="module")
+def nccl_group():
+    from datetime import timedelta
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=timedelta(seconds=60))
+    yield None
+    dist.destroy_process_group()
+
+
+def _cfg(N, D, F, E, k, **kw):
+    return configs.MoEConfig("ep", N=N, D=D, F=F, E=E, k=k, dtype=configs.DTYPE_BF16,
+                             activation=configs.ACT_SILU, renormalize=1, **kw)
+
+
+@pytest.mark.parametrize("cfg", [
+    _cfg(300, 256, 512, 8, 2),
+    _cfg(500, 128, 384, 16, 2, capacity_factor=1.0, router_bias_var=2.0),
+    _cfg(257, 384, 640, 8, 1),
+], ids=["e8k2", "capacity_e16", "k1"])
+def test_ep_forward_one_rank_matches_oracle_and_forward(abi, nccl_group, cfg):
+    inp = inputs.make_inputs(cfg, "cuda")
+    comp = ep.CudaCompute(cfg, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3)
+    out, info = ep.forward(comp, inp.X, cfg.E)
+    torch.cuda.synchronize()
+    assert comp.device_error() == 0
+    # same layer through moe_forward
+    layer_out = torch.empty_like(out)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    idx = torch.empty((cfg.N, cfg.k), dtype=torch.int32, device="cuda")
+    abi.forward(p, inp.X, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, layer_out, ws, topk_idx=idx)
+    torch.cuda.synchronize()
+    assert normwise_rel_err(to_f64(out), to_f64(layer_out)).max() <= 1e-2
+    # and the oracle, on every token whose selection is not a near tie
+    Xn = np_host(inp.X)
+    ref = oracle.forward(Xn, inp.W_r.cpu().numpy(), None if inp.bias is None else
+                         inp.bias.cpu().numpy(), np_host(inp.W1), np_host(inp.W2),
+                         np_host(inp.W3), k=cfg.k, cf=cfg.capacity_factor, renorm=1,
+                         act=cfg.activation, dtype=oracle.BF16)
+    l64, _ = oracle.router_logits(Xn, oracle.BF16, inp.W_r.cpu().numpy(),
+                                  None if inp.bias is None else inp.bias.cpu().numpy())
+    flips = (idx.cpu().numpy() != ref["idx"]).any(1)
+    assert (oracle.topk_margin(l64, cfg.k)[flips] < NEAR_TIE).all()
+    if cfg.capacity_factor > 0 and flips.any():
+        pytest.skip("near-tie flip under capacity changes other tokens' slots")
+    err = normwise_rel_err(to_f64(out)[~flips], ref["out"][~flips])
+    assert err.max() <= TOL_BF16, f"max normwise rel err {err.max():.3g}"
+    plan = info["plan"]
+    assert plan.send_rows == plan.recv_rows
+    if not flips.any():
+        assert plan.send_rows == [int(ref["offsets"][cfg.E])]
+        assert plan.local_offsets.tolist() == ref["offsets"].tolist()

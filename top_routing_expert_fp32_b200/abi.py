@@ -27,6 +27,7 @@ EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_workspace_size_host", "moe
            "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_ex",
            "moe_forward_host", "moe_expert_up_w8", "moe_expert_down_w8", "moe_forward_w8",
            "moe_pack_w8", "moe_expert_up_w8p", "moe_expert_down_w8p", "moe_forward_w8p",
+           "moe_gather_rows",
            "moe_workspace_init", "moe_get_device_error", "moe_status_string", "moe_last_error",
            "moe_version")
 
@@ -52,7 +53,7 @@ def _load() -> ctypes.CDLL:
         raise ImportError(f"{LIB_PATH} is missing: run `python -m top_routing_expert_fp32_b200.build`"
                           " (or __graft_entry__.build()) first")
     L = ctypes.CDLL(LIB_PATH)
-    P, S = ctypes.c_void_p, ctypes.c_size_t
+    P, S, I64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
     PP = ctypes.POINTER(moe_problem)
     sig = {
         "moe_capacity": [PP, ctypes.POINTER(ctypes.c_int64)],
@@ -73,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "moe_expert_down_w8": [PP, P, P, P, P, P, P, S, P],
         "moe_forward_w8": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "moe_pack_w8": [PP, P, P, P, P, P, P, P],
+        "moe_gather_rows": [P, I64, P, I64, I64, P, P, S, P],
         "moe_expert_up_w8p": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_down_w8p": [PP, P, P, P, P, P, P, S, P],
         "moe_forward_w8p": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
@@ -217,6 +219,13 @@ def expert_up_w8(p, X_perm, offsets, W1q, S1, W2q, S2, H, ws, stream=None):
 def expert_down_w8(p, H, offsets, W3q, S3, Y, ws, stream=None):
     _check(lib.moe_expert_down_w8(ctypes.byref(p), _ptr(H), _ptr(offsets), _ptr(W3q), _ptr(S3),
                                   _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def gather_rows(src, index, dst, ws, stream=None):
+    """dst[i] = src[index[i]] (row-wise); src / dst: 2-D device tensors of equal row size."""
+    rb = dst[0].numel() * dst.element_size()
+    _check(lib.moe_gather_rows(_ptr(src), src.shape[0], _ptr(index), index.numel(), rb, _ptr(dst),
+                               _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def pack_w8(p, W1q, W2q, W3q, W1p, W2p, W3p, stream=None):

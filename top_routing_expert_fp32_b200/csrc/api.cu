@@ -856,6 +856,25 @@ moe_status moe_expert_down_w8p(const moe_problem* p, const void* H, const int32_
                      static_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_gather_rows(const void* src, int64_t n_src_rows, const int32_t* index,
+                           int64_t n_rows, int64_t row_bytes, void* dst, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (n_rows < 0 || n_src_rows < 0)
+    return fail(MOE_ERR_INVALID_ARG, "n_rows and n_src_rows must be >= 0");
+  if (row_bytes <= 0 || row_bytes % 4 != 0)
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 4");
+  MOE_TRY(need(ws, "ws", 256));
+  if (ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace smaller than 256 bytes");
+  if (n_rows == 0) return MOE_OK;
+  MOE_TRY(need(index, "index", 4));
+  MOE_TRY(need(dst, "dst"));
+  if (n_src_rows > 0) MOE_TRY(need(src, "src"));
+  MOE_CUDA(launch_gather_rows(src, n_src_rows, index, n_rows, row_bytes, dst,
+                              static_cast<int*>(ws), static_cast<cudaStream_t>(stream)),
+           "gather rows");
+  return MOE_OK;
+}
+
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(need(ws, "ws", 256));
   if (ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace smaller than 256 bytes");

@@ -267,7 +267,49 @@ __global__ void __launch_bounds__(32)
   }
 }
 
+// dst[i] = src[index[i]] for i < n_rows: one warp per row, 16-byte words when the row length
+// allows (else 4-byte words). An index outside [0, n_src) is recorded as MOE_DEVERR_BAD_INDEX
+// and its row is zero-filled instead of read.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint8_t* __restrict__ src, int64_t n_src,
+                       const int32_t* __restrict__ index, int64_t n_rows, int64_t row_bytes,
+                       uint8_t* __restrict__ dst, int* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * wpb;
+  const bool wide = (row_bytes & 15) == 0;
+  for (int64_t i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n_rows; i += nwarps) {
+    const int64_t r = index[i];
+    uint8_t* d = dst + i * row_bytes;
+    const bool bad = r < 0 || r >= n_src;
+    if (bad && lane == 0) record_error(err, MOE_DEVERR_BAD_INDEX);
+    const uint8_t* s = src + (bad ? 0 : r) * row_bytes;
+    if (wide) {
+      const int64_t words = row_bytes >> 4;
+      for (int64_t j = lane; j < words; j += 32)
+        reinterpret_cast<uint4*>(d)[j] =
+            bad ? make_uint4(0, 0, 0, 0) : __ldg(reinterpret_cast<const uint4*>(s) + j);
+    } else {
+      const int64_t words = row_bytes >> 2;
+      for (int64_t j = lane; j < words; j += 32)
+        reinterpret_cast<uint32_t*>(d)[j] =
+            bad ? 0u : __ldg(reinterpret_cast<const uint32_t*>(s) + j);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const void* src, int64_t n_src, const int32_t* index,
+                               int64_t n_rows, int64_t row_bytes, void* dst, int* err,
+                               cudaStream_t stream) {
+  if (n_rows == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n_rows + 7) / 8, int64_t(num_sms()) * 8);
+  gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint8_t*>(src), n_src, index, n_rows, row_bytes,
+      static_cast<uint8_t*>(dst), err);
+  return cudaGetLastError();
+}
 
 int dispatch_num_chunks(int64_t records) {
   return static_cast<int>(std::max<int64_t>(1, (records + kDispatchChunk - 1) / kDispatchChunk));

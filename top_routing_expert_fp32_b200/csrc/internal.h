@@ -93,6 +93,12 @@ cudaError_t launch_slot_assign(const moe_problem& p, int64_t capacity, const int
 cudaError_t launch_gather(const moe_problem& p, const void* X, const int32_t* row_token,
                           const int32_t* offsets, void* X_perm, int* err, cudaStream_t stream);
 
+// dst[i] = src[index[i]] for i < n_rows (rows of row_bytes bytes, a multiple of 4; 16-byte
+// aligned pointers). Out-of-range indices: MOE_DEVERR_BAD_INDEX in *err, row zero-filled.
+cudaError_t launch_gather_rows(const void* src, int64_t n_src, const int32_t* index,
+                               int64_t n_rows, int64_t row_bytes, void* dst, int* err,
+                               cudaStream_t stream);
+
 // Grouped expert GEMMs, bf16 operands, tcgen05 tensor cores.
 //   up:   H = act(X_perm W1_e) (.) (X_perm W2_e)      down: Y = H W3_e
 cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
