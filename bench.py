@@ -475,6 +475,129 @@ def run_gpu(args, cfg, world, rank, device):
     return line
 
 
+def run_gpu_ep(args, cfg, world, rank, device):
+    """Expert-parallel layer (ep.forward): experts in contiguous blocks over the ranks, each
+    rank routing its own cfg.N tokens (weak scaling). Every step: route + dispatch, count and
+    row exchanges (NCCL all_to_all_single), expert-major reorder, the rank's grouped GEMMs,
+    reorder back, return exchange, combine. Device time per step, max over ranks."""
+    import torch
+    from top_routing_expert_fp32_b200 import configs, ep, inputs
+
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+    full = inputs.make_inputs(cfg, device)
+    e0, e1 = ep.expert_ranges(cfg.E, world)[rank]
+    W1, W2, W3 = (w[e0:e1].clone() for w in (full.W1, full.W2, full.W3))
+    X = full.X if rank == 0 else inputs.randn((cfg.N, cfg.D), 1.0, full.X.dtype, device,
+                                              cfg.seed + 1 + rank, inputs.TID_X)
+    W_r, bias = full.W_r, full.bias
+    del full
+    torch.cuda.empty_cache()
+    comp = ep.CudaCompute(cfg, W_r, bias, W1, W2, W3, device)
+    N, D, F, k = cfg.N, cfg.D, cfg.F, cfg.k
+    es = X.element_size()
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.int32, device=device)
+    flush_sum = torch.empty((), dtype=torch.int64, device=device)
+
+    def flush_l2():
+        flush.fill_(1)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        ep.forward(comp, X, cfg.E)
+    torch.cuda.synchronize(device)
+    assert comp.device_error() == 0
+    barrier(device)
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    t_wall0 = time.time()
+    e0v = torch.cuda.Event(enable_timing=True)
+    e1v = torch.cuda.Event(enable_timing=True)
+    total = 0.0
+    kept = 0
+    off_rank = 0
+    for _ in range(args.steps):
+        flush_l2()
+        e0v.record(stream)
+        _, info = ep.forward(comp, X, cfg.E)
+        e1v.record(stream)
+        e1v.synchronize()
+        total += e0v.elapsed_time(e1v)
+        plan = info["plan"]
+        kept = sum(plan.send_rows)
+        # rows leaving this rank: its records for other ranks' experts, then the outputs it
+        # returns to other ranks
+        off_rank = ((kept - plan.send_rows[rank]) +
+                    (sum(plan.recv_rows) - plan.recv_rows[rank])) * D * es
+    t_wall1 = time.time()
+    sampler.stop()
+    mx = reduce_max(total, device)
+    agg = aggregate(N, world, mx, args.steps)
+    tc, hbm = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    # Step bound: the expert GEMM FLOPs of this rank's received rows at the bf16 peak, or the
+    # rows this rank sends off-rank (both exchanges) at the measured 770 GB/s peer copy rate.
+    recv = sum(plan.recv_rows)
+    flops = 6.0 * recv * D * F
+    t_tc = flops / (tc * 1e12)
+    t_link = off_rank / 770e9
+    step_s = agg["ms_per_step"] / 1e3
+    roof = {"kernel": "whole expert-parallel step (expert GEMMs of the received rows; "
+                      "off-rank rows over NVLink)",
+            "bound": "tensor" if t_tc >= t_link else "nvlink",
+            "achieved": (flops / step_s / 1e12) if t_tc >= t_link else off_rank / step_s / 1e9,
+            "peak": tc if t_tc >= t_link else 770.0,
+            "unit": "TFLOP/s" if t_tc >= t_link else "GB/s",
+            "peak_source": (f"{peak_src} (MEASURED_PEAKS.json), bf16 burst" if t_tc >= t_link
+                            else "measured 8-GPU peer copy per direction (pool figure)"),
+            "traffic": None}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+
+    xh = X.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(X)
+
+    def e2e_call():
+        xd.copy_(xh, non_blocking=True)
+        out, _ = ep.forward(comp, xd, cfg.E)
+        oh.copy_(out, non_blocking=True)
+
+    e2e_call()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    et = 0.0
+    for _ in range(args.steps):
+        flush_l2()
+        e0v.record(stream)
+        e2e_call()
+        e1v.record(stream)
+        e1v.synchronize()
+        et += e0v.elapsed_time(e1v)
+    e_max = reduce_max(et, device)
+    barrier(device)
+    launches = (2 if cfg.dtype == configs.DTYPE_BF16 else 1) + 3 + 2 + 2 + 1
+    return {
+        "metric": METRIC, "value": agg["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": agg["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_name(cfg),
+        "data": "synthetic, seeded: X~N(0,1) per rank, W_r/W1/W2~N(0,1/D), W3~N(0,1/F)",
+        "config": {"workload": workload_desc(cfg), "tokens_per_gpu": N,
+                   "parallelism": f"ep{world}: experts in contiguous blocks, rank {rank} holds "
+                                  f"{e0}..{e1 - 1}; NCCL all_to_all_single exchanges",
+                   "l2": "flushed between steps (512 MiB write + read-back, outside the step events)",
+                   "kept_records_per_rank": kept,
+                   "a2a_bytes_model_per_step": ep.a2a_bytes(N * world, D, k, es),
+                   "off_rank_bytes_per_step_rank0": off_rank},
+        "roofline": roof,
+        "e2e": {"value": N * world * args.steps / (e_max / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": N * D * es, "d2h_bytes_per_step": N * D * es,
+                "api": "ep.forward between pinned-host copies of X and out; copies in the "
+                       "timed region"},
+        "gpu_launches": launches * args.steps,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -491,6 +614,9 @@ def main():
     ap.add_argument("--weights", default="bf16", choices=["bf16", "w8", "w8p"],
                     help="expert weights: bf16, or int8 with per-column fp32 scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="replicas: one independent layer per GPU; ep: experts split over the "
+                         "GPUs, rows exchanged by all-to-all (bf16 weights)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -522,19 +648,31 @@ def main():
 
     import torch
     import torch.distributed as dist
+    from datetime import timedelta
+    ep_mode = args.parallel == "ep"
+    if ep_mode and args.weights != "bf16":
+        raise SystemExit("--parallel ep runs bf16 expert weights")
     if world > 1:
-        from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+    elif ep_mode:  # the exchanges need a process group, even of one rank
+        import socket
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
-    line = run_gpu(args, cfg, world, rank, device)
+    line = (run_gpu_ep if ep_mode else run_gpu)(args, cfg, world, rank, device)
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = oracle_tokens_per_s(cfg, w8=args.weights != "bf16")
         else:
             line["cpu_baseline"] = None
         print(json.dumps(line))
-    if world > 1:
+    if dist.is_initialized():
         dist.destroy_process_group()
     return 0
 

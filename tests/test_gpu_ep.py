@@ -115,3 +115,22 @@ def test_ep_forward_one_rank_matches_oracle_and_forward(abi, nccl_group, cfg):
     if not flips.any():
         assert plan.send_rows == [int(ref["offsets"][cfg.E])]
         assert plan.local_offsets.tolist() == ref["offsets"].tolist()
+
+
+def test_ep_forward_one_rank_full_size_mixtral(abi, nccl_group):
+    # The benchmark's layer (N=4096, D=4096, F=14336, E=8, k=2) through ep.forward against
+    # moe_forward on the same inputs (the oracle checks moe_forward at this size).
+    cfg = configs.CONFIGS["mixtral"]
+    inp = inputs.make_inputs(cfg, "cuda")
+    comp = ep.CudaCompute(cfg, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3)
+    out, info = ep.forward(comp, inp.X, cfg.E)
+    ref = torch.empty_like(out)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    abi.forward(p, inp.X, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, ref, ws)
+    torch.cuda.synchronize()
+    assert comp.device_error() == 0 and abi.device_error(ws) == 0
+    assert info["plan"].send_rows == [cfg.N * cfg.k]
+    assert normwise_rel_err(to_f64(out), to_f64(ref)).max() <= 1e-2
+    del inp, comp, out, ref, ws
+    torch.cuda.empty_cache()

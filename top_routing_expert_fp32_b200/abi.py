@@ -8,6 +8,7 @@ fallback: if the library is missing or fails to load, importing this module rais
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
@@ -223,7 +224,7 @@ def expert_down_w8(p, H, offsets, W3q, S3, Y, ws, stream=None):
 
 def gather_rows(src, index, dst, ws, stream=None):
     """dst[i] = src[index[i]] (row-wise); src / dst: 2-D device tensors of equal row size."""
-    rb = dst[0].numel() * dst.element_size()
+    rb = math.prod(dst.shape[1:]) * dst.element_size()
     _check(lib.moe_gather_rows(_ptr(src), src.shape[0], _ptr(index), index.numel(), rb, _ptr(dst),
                                _ptr(ws), ws.numel(), _stream(stream)))
 
