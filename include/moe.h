@@ -316,8 +316,8 @@ moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,
  * (page-locked memory gives asynchronous copies), the weights and W_r/bias are device
  * pointers. Enqueues the host->device copy of X, the forward, and the device->host copy
  * of out on `stream`, then waits for the stream, so out_host is valid on return. Uses
- * the workspace (moe_workspace_size + N*D*2*sizeof(element) bytes, see
- * moe_workspace_size_host). Without capacity (capacity_factor <= 0) and with N >= 1024 the
+ * the workspace (moe_workspace_size_host bytes: moe_workspace_size plus the device copies of
+ * X and out, double-buffered for moe_forward_host_many). Without capacity (capacity_factor <= 0) and with N >= 1024 the
  * batch runs as two halves, the copies of one half overlapping the other half's layer on an
  * internal copy stream; each token's output is then the layer on its own half-batch (the same
  * result up to the rounding of the router's split of D). Needs routing_mode = TOPK. */
@@ -325,7 +325,23 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
                             const float* bias, const void* W1, const void* W2, const void* W3,
                             void* out_host, void* ws, size_t ws_bytes, void* stream);
 
-/* Host only. Workspace bytes for moe_forward_host. */
+/* A sequence of host batches through the layer, for serving loops: batch b's X is
+ * X_host + b*N*D*s and its output goes to out_host + b*N*D*s (both [n_batches, N, D], pinned
+ * host memory for asynchronous copies; the caller owns them). Each batch is a complete
+ * moe_forward call on its N tokens (capacity per batch) and its output equals moe_forward's bit
+ * for bit. Device buffers for X and the output are double-buffered in the workspace
+ * (moe_workspace_size_host), with input copies on one internal copy stream and output copies on
+ * another, so batch b+1's input copy and batch b-1's output copy overlap batch b's layer on
+ * `stream`. Returns after every output copy has completed (the stream is synchronised).
+ * n_batches == 0 or N == 0 is a no-op. Errors as moe_forward_host; after a failure the outputs
+ * of batches from the failing one on are unspecified. Plain top-k routing only. */
+moe_status moe_forward_host_many(const moe_problem* p, int64_t n_batches, const void* X_host,
+                                 const float* W_r, const float* bias, const void* W1,
+                                 const void* W2, const void* W3, void* out_host, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* Host only. Workspace bytes for moe_forward_host and moe_forward_host_many (moe_workspace_size
+ * plus 4*N*D*sizeof(element), each part 256-byte aligned). */
 moe_status moe_workspace_size_host(const moe_problem* p, size_t* bytes);
 
 /* Row gather: dst[i] = src[index[i]] for i < n_rows, rows of row_bytes bytes. The local

@@ -189,3 +189,28 @@ def test_routing_mode_checks_on_host(abi):
     st = abi.lib.moe_route_ex(ctypes.byref(p), 16, 16, None, None, None, 16, 16, None, None, 256,
                               ws_bytes, None)
     assert st == 1 and b"noise" in abi.lib.moe_last_error()
+
+
+def test_streamed_host_entry_and_gather_reject_bad_arguments_on_host(abi):
+    # Checked before anything is enqueued (no GPU needed).
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.MoEConfig("h", N=64, D=64, F=64, E=8, k=2, dtype=configs.DTYPE_BF16,
+                            activation=0, renormalize=1)
+    p = abi.problem(cfg)
+    b = ctypes.c_size_t()
+    assert abi.lib.moe_workspace_size_host(ctypes.byref(p), ctypes.byref(b)) == 0
+    need_h = b.value
+    # the host workspace holds the layer's plus four N x D activation buffers
+    assert need_h >= abi.workspace_size(p) + 4 * 64 * 64 * 2
+    fwd = lambda nb, ws_bytes, x=4096: abi.lib.moe_forward_host_many(
+        ctypes.byref(p), nb, x, 4096, None, 4096, 4096, 4096, 4096, 4096, ws_bytes, None)
+    assert fwd(-1, need_h) == abi.MOE_ERR_INVALID_ARG
+    assert fwd(2, need_h - 1) == abi.MOE_ERR_INVALID_ARG          # workspace too small
+    assert fwd(2, need_h, x=None) == abi.MOE_ERR_INVALID_ARG      # no host X
+    assert b"X_host" in abi.lib.moe_last_error()
+    g = abi.lib.moe_gather_rows
+    assert g(4096, 10, 4096, 5, 6, 4096, 4096, 256, None) == abi.MOE_ERR_INVALID_ARG  # 6 % 4
+    assert g(4096, 10, 4096, -1, 8, 4096, 4096, 256, None) == abi.MOE_ERR_INVALID_ARG
+    assert g(4096, 10, 4096, 5, 8, 4096, 4096, 128, None) == abi.MOE_ERR_INVALID_ARG  # small ws
+    assert g(4096, 10, None, 5, 8, 4096, 4096, 256, None) == abi.MOE_ERR_INVALID_ARG  # no index
+    assert g(4096, 10, 4096, 5, 8, 4100, 4096, 256, None) == abi.MOE_ERR_INVALID_ARG  # dst align

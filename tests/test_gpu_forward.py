@@ -198,3 +198,41 @@ def test_forward_host_two_halves_equal_forward_on_each_half(abi):
         abi.forward(ph, inp.X[lo:hi].contiguous(), inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, o, wsh)
         torch.cuda.synchronize()
         assert torch.equal(o.cpu().view(torch.int16), oh[lo:hi].view(torch.int16))
+
+
+@pytest.mark.parametrize("cfg,nb", [
+    (configs.MoEConfig("many", N=700, D=256, F=512, E=8, k=2, dtype=configs.DTYPE_BF16,
+                       activation=configs.ACT_SILU, renormalize=1), 5),
+    (configs.MoEConfig("many_cap", N=500, D=128, F=256, E=16, k=2, dtype=configs.DTYPE_BF16,
+                       activation=configs.ACT_SILU, renormalize=1, capacity_factor=1.0), 3),
+    (configs.MoEConfig("many_one", N=64, D=256, F=512, E=8, k=2, dtype=configs.DTYPE_BF16,
+                       activation=configs.ACT_GELU_ERF, renormalize=0), 1),
+], ids=["e8_5batches", "capacity_3batches", "one_batch"])
+def test_forward_host_many_equals_forward_per_batch(abi, cfg, nb):
+    # Each batch of the streamed call is a complete layer call on its own tokens (capacity per
+    # batch): its output must be moe_forward's on that batch, bit for bit, whatever the overlap.
+    inp = inputs.make_inputs(cfg, "cuda")
+    Xb = torch.stack([inputs.randn((cfg.N, cfg.D), 1.0, torch.bfloat16, "cuda", 40 + b,
+                                   inputs.TID_X) for b in range(nb)])
+    p = abi.problem(cfg)
+    ws = abi.workspace(p, host=True)
+    xh = Xb.cpu().pin_memory()
+    oh = torch.full_like(xh, float("nan")).pin_memory()
+    abi.forward_host_many(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws)
+    assert abi.device_error(ws) == 0
+    wsd = abi.workspace(p)
+    for b in range(nb):
+        o = torch.empty((cfg.N, cfg.D), dtype=torch.bfloat16, device="cuda")
+        abi.forward(p, Xb[b], inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, o, wsd)
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu().view(torch.int16), oh[b].view(torch.int16)), f"batch {b}"
+
+
+def test_forward_host_many_zero_batches_is_a_no_op(abi):
+    cfg = SMALL[1]
+    inp = inputs.make_inputs(cfg, "cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p, host=True)
+    xh = torch.empty((0, cfg.N, cfg.D), dtype=torch.bfloat16).pin_memory()
+    oh = torch.empty_like(xh)
+    abi.forward_host_many(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws)

@@ -66,7 +66,8 @@ struct Layout {
   size_t err, colsum_part, zl_part, wt, counts, idx, gate, pos, dropped, load, offsets, row_token,
       xperm, h, y;
   size_t total;       // moe_forward and every other entry point
-  size_t xin, xout;   // moe_forward_host only
+  size_t xin, xout;   // moe_forward_host / moe_forward_host_many
+  size_t xin2, xout2; // second buffers of moe_forward_host_many
   size_t total_host;
 };
 
@@ -98,6 +99,8 @@ Layout make_layout(const moe_problem& p) {
   L.total = o;
   L.xin = take(es * static_cast<size_t>(p.N) * static_cast<size_t>(p.D));
   L.xout = take(es * static_cast<size_t>(p.N) * static_cast<size_t>(p.D));
+  L.xin2 = take(es * static_cast<size_t>(p.N) * static_cast<size_t>(p.D));
+  L.xout2 = take(es * static_cast<size_t>(p.N) * static_cast<size_t>(p.D));
   L.total_host = o;
   return L;
 }
@@ -587,21 +590,22 @@ moe_status moe_forward_ex(const moe_problem* p, const void* X, const float* W_r,
                       static_cast<cudaStream_t>(stream));
 }
 
-// A non-blocking stream per device for the host copies of moe_forward_host (created on first
-// use, kept for the life of the process).
-cudaError_t copy_stream(cudaStream_t* out) {
-  static cudaStream_t streams[64] = {};
+// Non-blocking streams per device for the host copies of moe_forward_host[_many] (created on
+// first use, kept for the life of the process): `which` 0 carries host-to-device copies (and
+// both directions in moe_forward_host), 1 device-to-host copies.
+cudaError_t copy_stream(cudaStream_t* out, int which = 0) {
+  static cudaStream_t streams[64][2] = {};
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (streams[dev] == nullptr) {
-    e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+  if (streams[dev][which] == nullptr) {
+    e = cudaStreamCreateWithFlags(&streams[dev][which], cudaStreamNonBlocking);
     if (e != cudaSuccess) return e;
   }
-  *out = streams[dev];
+  *out = streams[dev][which];
   return cudaSuccess;
 }
 
@@ -689,6 +693,90 @@ moe_status moe_forward_host(const moe_problem* p, const void* X_host, const floa
     step(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   }
   for (int i = 0; i < 6; ++i)
+    if (ev[i] != nullptr) cudaEventDestroy(ev[i]);
+  return st;
+}
+
+moe_status moe_forward_host_many(const moe_problem* p, int64_t n_batches, const void* X_host,
+                                 const float* W_r, const float* bias, const void* W1,
+                                 const void* W2, const void* W3, void* out_host, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  MOE_TRY(check_problem(p));
+  if (n_batches < 0) return fail(MOE_ERR_INVALID_ARG, "n_batches < 0");
+  MOE_TRY(check_ws(*p, ws, ws_bytes, true));
+  MOE_TRY(need_topk(*p));
+  if (p->N > 0 && n_batches > 0) {
+    MOE_TRY(need(X_host, "X_host", 1));
+    MOE_TRY(need(out_host, "out_host", 1));
+  }
+  MOE_TRY(need(W_r, "W_r"));
+  MOE_TRY(opt(bias, "bias", 4));
+  MOE_TRY(need(W1, "W1"));
+  MOE_TRY(need(W2, "W2"));
+  MOE_TRY(need(W3, "W3"));
+  if (p->N == 0 || n_batches == 0) return MOE_OK;
+  const Layout L = make_layout(*p);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = elem_size(*p) * static_cast<size_t>(p->N) * static_cast<size_t>(p->D);
+  void* xin[2] = {at<void>(ws, L.xin), at<void>(ws, L.xin2)};
+  void* xout[2] = {at<void>(ws, L.xout), at<void>(ws, L.xout2)};
+  cudaStream_t cs_in = nullptr, cs_out = nullptr;
+  MOE_CUDA(copy_stream(&cs_in, 0), "copy stream");
+  MOE_CUDA(copy_stream(&cs_out, 1), "copy stream");
+  Experts w;
+  w.W1 = W1;
+  w.W2 = W2;
+  w.W3 = W3;
+  // Batch b uses buffer pair b % 2. Its input copy waits until batch b-2's layer has read that
+  // buffer, its layer until batch b-2's output copy has read the output buffer, so the input
+  // copy of batch b+1 and the output copy of batch b-1 run under batch b's layer.
+  cudaEvent_t ev[7] = {};  // start, in_done[2], comp_done[2], out_done[2]
+  cudaEvent_t* in_done = ev + 1;
+  cudaEvent_t* comp_done = ev + 3;
+  cudaEvent_t* out_done = ev + 5;
+  moe_status st = MOE_OK;
+  for (int i = 0; i < 7 && st == MOE_OK; ++i)
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess)
+      st = fail(MOE_ERR_CUDA, "cudaEventCreateWithFlags");
+  auto step = [&](cudaError_t e, const char* what) {
+    if (st == MOE_OK && e != cudaSuccess) st = cuda_fail(e, what);
+  };
+  int64_t issued = 0;  // batches whose output copy was enqueued
+  if (st == MOE_OK) {
+    // The copies follow whatever the caller's stream has queued before this call.
+    step(cudaEventRecord(ev[0], s), "event");
+    step(cudaStreamWaitEvent(cs_in, ev[0], 0), "wait");
+    step(cudaStreamWaitEvent(cs_out, ev[0], 0), "wait");
+    for (int64_t b = 0; b < n_batches && st == MOE_OK; ++b) {
+      const int slot = static_cast<int>(b & 1);
+      const uint8_t* xh = static_cast<const uint8_t*>(X_host) + static_cast<size_t>(b) * bytes;
+      uint8_t* oh = static_cast<uint8_t*>(out_host) + static_cast<size_t>(b) * bytes;
+      if (b >= 2) step(cudaStreamWaitEvent(cs_in, comp_done[slot], 0), "wait");
+      step(cudaMemcpyAsync(xin[slot], xh, bytes, cudaMemcpyHostToDevice, cs_in), "H2D");
+      step(cudaEventRecord(in_done[slot], cs_in), "event");
+      step(cudaStreamWaitEvent(s, in_done[slot], 0), "wait");
+      if (b >= 2) step(cudaStreamWaitEvent(s, out_done[slot], 0), "wait");
+      if (st == MOE_OK)
+        st = forward_impl(*p, xin[slot], W_r, bias, nullptr, w, xout[slot], nullptr, nullptr,
+                          nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, ws, s);
+      step(cudaEventRecord(comp_done[slot], s), "event");
+      step(cudaStreamWaitEvent(cs_out, comp_done[slot], 0), "wait");
+      step(cudaMemcpyAsync(oh, xout[slot], bytes, cudaMemcpyDeviceToHost, cs_out), "D2H");
+      step(cudaEventRecord(out_done[slot], cs_out), "event");
+      if (st == MOE_OK) issued = b + 1;
+    }
+  }
+  // Join: the caller's stream waits for every enqueued output copy, then the host waits.
+  for (int i = 0; i < 2 && i < issued; ++i) cudaStreamWaitEvent(s, out_done[i], 0);
+  if (issued > 0 || st != MOE_OK) {
+    const cudaError_t e = cudaStreamSynchronize(s);
+    if (st == MOE_OK && e != cudaSuccess) st = cuda_fail(e, "cudaStreamSynchronize");
+    if (st != MOE_OK) {  // after an error, wait for the copy streams too before returning
+      cudaStreamSynchronize(cs_in);
+      cudaStreamSynchronize(cs_out);
+    }
+  }
+  for (int i = 0; i < 7; ++i)
     if (ev[i] != nullptr) cudaEventDestroy(ev[i]);
   return st;
 }
