@@ -68,12 +68,16 @@ def _ffn_w8(abi, counts, D, F, act, seed=0, packed=False):
     ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
     ([700, 0, 257, 1100], 512, 400, configs.ACT_GELU_ERF),
 ])
-@pytest.mark.parametrize("kernel", ["smem", "tmem", "packed"])
+@pytest.mark.parametrize("kernel", ["smem", "tmem", "packed", "tmem_a_in_smem",
+                                    "packed_a_in_smem"])
 def test_expert_ffn_w8_matches_oracle(abi, monkeypatch, counts, D, F, act, kernel):
-    # smem: converted weights in shared memory (larger batches); tmem: transposed product with
-    # the converted weights as the tensor-memory operand (few rows per expert); packed: the
-    # tmem kernel on K-contiguous weights from moe_pack_w8.
-    monkeypatch.setenv("MOE_W8_KERNEL", "tmem" if kernel == "packed" else kernel)
+    # smem: the shared-memory kernel (larger batches); tmem: the transposed kernel for few rows
+    # per expert, its converted weights the MMA's A operand in tensor memory (default) or, for
+    # the *_a_in_smem cases, in shared memory; packed: the transposed kernel on K-contiguous
+    # weights from moe_pack_w8.
+    monkeypatch.setenv("MOE_W8_KERNEL", "smem" if kernel == "smem" else "tmem")
+    monkeypatch.setenv("MOE_W8T_A", "smem" if kernel.endswith("_a_in_smem") else "tmem")
+    kernel = kernel.replace("_a_in_smem", "")
     cfg, Xp, w, offsets, H, Y, R = _ffn_w8(abi, counts, D, F, act, packed=kernel == "packed")
     rec_e = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
     ref = oracle.expert_ffn_w8(np.arange(R, dtype=np.int32), rec_e, np_host(Xp), oracle.BF16,
@@ -124,10 +128,12 @@ def test_pack_w8_is_exact_transpose(abi, E, k, n):
     assert torch.equal(wp.W3q, w.W3q.transpose(1, 2))
 
 
-def test_packed_reproduces_tmem_kernel_bit_for_bit(abi, monkeypatch):
+@pytest.mark.parametrize("a_loc", ["smem", "tmem"])
+def test_packed_reproduces_tmem_kernel_bit_for_bit(abi, monkeypatch, a_loc):
     # The same bf16 values of q enter the same MMAs in the same order, only the staging layout
-    # differs, so H and Y match the unpacked tensor-memory kernel bit for bit.
+    # differs, so H and Y match the unpacked transposed kernel bit for bit.
     monkeypatch.setenv("MOE_W8_KERNEL", "tmem")
+    monkeypatch.setenv("MOE_W8T_A", a_loc)
     counts, D, F = [0, 65, 3, 130, 64, 1], 336, 208
     _, _, _, _, Hu, Yu, R = _ffn_w8(abi, counts, D, F, configs.ACT_GELU_TANH, seed=9)
     _, _, _, _, Hp, Yp, _ = _ffn_w8(abi, counts, D, F, configs.ACT_GELU_TANH, seed=9,
