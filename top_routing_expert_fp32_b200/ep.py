@@ -178,6 +178,9 @@ class CudaCompute(LocalCompute):
         self.device = torch.device(device)
         self.p = abi.problem(cfg)
         self.ws = abi.workspace(self.p, self.device)
+        self._rows = 0          # received rows the local-layer buffers below are sized for
+        self._ws_loc = None
+        self._H = None
 
     def route_dispatch(self, X) -> dict:
         a, cfg, dev = self.abi, self.cfg, self.device
@@ -202,13 +205,16 @@ class CudaCompute(LocalCompute):
         Y = torch.empty((R, self.cfg.D), dtype=X_loc.dtype, device=self.device)
         if R == 0 or e1 == e0:
             return Y
-        # The local experts as a layer of their own: R rows, one slot each, E_local experts.
+        # The local experts as a layer of their own: R rows, one slot each, E_local experts. Its
+        # workspace and H are kept and regrown only when more rows arrive than ever before.
         p = a.problem(self.cfg.with_(N=R, k=1, E=e1 - e0, capacity_factor=0.0, min_capacity=0))
-        ws = a.workspace(p, self.device)
+        if R > self._rows:
+            self._ws_loc = a.workspace(p, self.device)
+            self._H = torch.empty((R, self.cfg.F), dtype=X_loc.dtype, device=self.device)
+            self._rows = R
         off = torch.from_numpy(np.ascontiguousarray(local_offsets, dtype=np.int32)).to(self.device)
-        H = torch.empty((R, self.cfg.F), dtype=X_loc.dtype, device=self.device)
-        a.expert_up(p, X_loc, off, self.W1, self.W2, H, ws)
-        a.expert_down(p, H, off, self.W3, Y, ws)
+        a.expert_up(p, X_loc, off, self.W1, self.W2, self._H, self._ws_loc)
+        a.expert_down(p, self._H, off, self.W3, Y, self._ws_loc)
         return Y
 
     def gather_rows(self, src, index):
@@ -230,4 +236,8 @@ class CudaCompute(LocalCompute):
         return out
 
     def device_error(self) -> int:
-        return self.abi.device_error(self.ws)
+        """First nonzero device error code of the rank's workspaces (0 if none); clears them."""
+        codes = [self.abi.device_error(self.ws)]
+        if self._ws_loc is not None:
+            codes.append(self.abi.device_error(self._ws_loc))
+        return next((c for c in codes if c != 0), 0)
