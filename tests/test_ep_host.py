@@ -143,7 +143,8 @@ def _worker(rank, world, port, case, results):
     (2, dict(E=8, D=32, F=48, k=2, N=40, cf=1.0)),
     (3, dict(E=8, D=16, F=32, k=2, N=33, cf=0.0)),     # expert blocks of 3, 3, 2
     (3, dict(E=4, D=16, F=32, k=1, N=25, cf=1.25)),    # blocks of 2, 1, 1
-], ids=["w2", "w2_capacity", "w3_uneven", "w3_k1_capacity"])
+    (3, dict(E=2, D=16, F=32, k=2, N=20, cf=0.0)),     # rank 2 owns no expert
+], ids=["w2", "w2_capacity", "w3_uneven", "w3_k1_capacity", "w3_more_ranks_than_experts"])
 def test_ep_forward_equals_single_device_layer_gloo(world, case):
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
