@@ -5,7 +5,7 @@
 //   with renorm_kept, a token that lost some slots spreads the whole weight over the kept
 //   ones, gate / sum of kept gates).
 //
-// One block per token, each thread owns 16-byte column chunks of the row. The k rows are read
+// One warp per token; each lane owns 16-byte column chunks of the row. The k rows are read
 // with 16-byte loads, accumulated in fp32 in ascending j (fixed order, no atomics), and
 // rounded once to the output dtype. HBM-bound: reads the kept Y rows once, writes out once.
 #include "common.cuh"
@@ -14,8 +14,8 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kMaxK = 8;
+constexpr int kWarps = 8;  // tokens per block
+constexpr int kThreads = 32 * kWarps;
 
 template <typename T>
 struct Vec16;
@@ -52,74 +52,88 @@ struct Vec16<float> {
   }
 };
 
-template <typename T, int KMAX, bool BATCH>
+// wpt warps per token (1, or kWarps for batches too small to fill the GPU), kWarps / wpt
+// tokens per block, no block-wide barrier. Lanes 0..k-1 of each warp read the token's records
+// (expert, position, drop flag, gate) and the warp shares them by shuffles; every lane then
+// streams 16-byte chunks of the k rows, kBatch chunks of all k rows loaded before any is used
+// (about 8 loads in flight per lane).
+template <typename T, int KMAX, int WPT>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4* __restrict__ Y, const int32_t* __restrict__ idx,
                    const float* __restrict__ gate, const int32_t* __restrict__ offsets,
                    const int32_t* __restrict__ pos, const uint8_t* __restrict__ dropped,
                    uint4* __restrict__ out, int64_t N, int k, int E, int64_t chunks_per_row,
                    bool renorm_kept, int* err) {
+  constexpr int wpt = WPT;
   constexpr int V = Vec16<T>::kElems;
-  __shared__ int64_t s_row[kMaxK];
-  __shared__ float s_g[kMaxK];
-  const int64_t t = blockIdx.x;
-  if (threadIdx.x < k) {
-    const int j = threadIdx.x;
-    const int64_t rec = t * k + j;
+  constexpr int kBatch = KMAX >= 8 ? 1 : 8 / KMAX;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * (kWarps / wpt) + warp / wpt;
+  const int64_t first = 32 * (warp % wpt) + lane;  // this lane's first chunk
+  const int64_t step = 32 * wpt;
+  if (t >= N) return;  // uniform over the warp
+  int64_t my_row = -1;
+  float my_g = 0.f;
+  if (lane < k) {
+    const int64_t rec = t * k + lane;
     const int e = idx[rec];
     bool keep = dropped == nullptr || dropped[rec] == 0;
     if (e < 0 || e >= E) {
       record_error(err, MOE_DEVERR_BAD_INDEX);
       keep = false;
     }
-    s_row[j] = keep ? static_cast<int64_t>(offsets[e]) + pos[rec] : -1;
-    s_g[j] = gate[rec];
+    my_row = keep ? static_cast<int64_t>(offsets[e]) + pos[rec] : -1;
+    my_g = gate[rec];
   }
-  __syncthreads();
-  if (renorm_kept && threadIdx.x == 0) {
+  int64_t row[KMAX];
+  float g[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    row[j] = __shfl_sync(0xffffffffu, my_row, j);
+    g[j] = __shfl_sync(0xffffffffu, my_g, j);
+    if (j >= k) row[j] = -1;
+  }
+  if (renorm_kept) {  // MoE series 2.2 case A: the kept gates share the whole weight
     float kept_sum = 0.f;
     int kept = 0;
-    for (int j = 0; j < k; ++j)
-      if (s_row[j] >= 0) {
-        kept_sum += s_g[j];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (row[j] >= 0) {
+        kept_sum += g[j];
         ++kept;
       }
-    if (kept > 0 && kept < k)
-      for (int j = 0; j < k; ++j)
-        if (s_row[j] >= 0) s_g[j] = s_g[j] / kept_sum;
+    if (kept > 0 && kept < k) {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (row[j] >= 0) g[j] = g[j] / kept_sum;
+    }
   }
-  if (renorm_kept) __syncthreads();
-  // With BATCH (long rows), kBatch chunks per thread are loaded (all k rows) before any is
-  // used, so a thread keeps about 8 16-byte loads in flight instead of one round trip per
-  // chunk; short rows keep the register count (and occupancy) of one chunk at a time.
-  constexpr int kBatch = (!BATCH || KMAX >= 8) ? 1 : 8 / KMAX;
-  for (int64_t c0 = threadIdx.x; c0 < chunks_per_row; c0 += kThreads * kBatch) {
+  for (int64_t c0 = first; c0 < chunks_per_row; c0 += step * kBatch) {
     uint4 yv[kBatch][KMAX];
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-      const int64_t c = c0 + b * kThreads;
+      const int64_t c = c0 + b * step;
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         yv[b][j] = make_uint4(0u, 0u, 0u, 0u);
-        if (j < k && c < chunks_per_row && s_row[j] >= 0)
-          yv[b][j] = __ldg(Y + s_row[j] * chunks_per_row + c);
+        if (c < chunks_per_row && row[j] >= 0) yv[b][j] = __ldg(Y + row[j] * chunks_per_row + c);
       }
     }
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-      const int64_t c = c0 + b * kThreads;
+      const int64_t c = c0 + b * step;
       if (c >= chunks_per_row) break;
       float acc[V];
 #pragma unroll
       for (int i = 0; i < V; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
-        if (j >= k || s_row[j] < 0) continue;
+        if (row[j] < 0) continue;
         float y[V];
         Vec16<T>::unpack(yv[b][j], y);
-        const float g = s_g[j];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = fmaf(g, y[i], acc[i]);
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(g[j], y[i], acc[i]);
       }
       out[t * chunks_per_row + c] = Vec16<T>::pack(acc);
     }
@@ -134,21 +148,23 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
   if (p.N == 0) return cudaSuccess;
   const int64_t elem = p.dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int64_t chunks = p.D * elem / 16;
-  const dim3 grid(static_cast<unsigned>(p.N));
+  // A warp per token once there are enough tokens for 16 warps per SM (about 64 KB of loads
+  // in flight per SM), else a block of kWarps warps per token.
+  const int wpt = p.N >= static_cast<int64_t>(num_sms()) * 16 ? 1 : kWarps;
+  const int tpb = kWarps / wpt;
+  const dim3 grid(static_cast<unsigned>((p.N + tpb - 1) / tpb));
   const uint4* y = static_cast<const uint4*>(Y);
   uint4* o = static_cast<uint4*>(out);
-  const bool batch = chunks >= 4 * kThreads;
   const bool rk = p.drop_policy == MOE_DROP_RENORM_KEPT && dropped != nullptr;
-#define MOE_COMBINE(T, KM)                                                                     \
-  do {                                                                                         \
-    if (batch)                                                                                 \
-      combine_kernel<T, KM, true><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,   \
-                                                                 dropped, o, p.N, p.k, p.E,    \
-                                                                 chunks, rk, err);             \
-    else                                                                                       \
-      combine_kernel<T, KM, false><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,  \
-                                                                  dropped, o, p.N, p.k, p.E,   \
-                                                                  chunks, rk, err);            \
+#define MOE_COMBINE(T, KM)                                                                      \
+  do {                                                                                          \
+    if (wpt == 1)                                                                               \
+      combine_kernel<T, KM, 1><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,       \
+                                                              dropped, o, p.N, p.k, p.E, chunks, \
+                                                              rk, err);                         \
+    else                                                                                        \
+      combine_kernel<T, KM, kWarps><<<grid, kThreads, 0, stream>>>(                             \
+          y, idx, gate, offsets, pos, dropped, o, p.N, p.k, p.E, chunks, rk, err);              \
   } while (0)
   if (p.dtype == MOE_DTYPE_BF16) {
     if (p.k <= 1) MOE_COMBINE(__nv_bfloat16, 1);
