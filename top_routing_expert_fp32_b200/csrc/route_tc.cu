@@ -27,6 +27,7 @@
 // Every barrier wait is bounded in time; on a timeout the CTA records MOE_DEVERR_WAIT_TIMEOUT,
 // unwinds, drains its MMAs and frees its tensor memory.
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "internal.h"
@@ -406,6 +407,13 @@ TcShape tc_shape(int64_t N, int D, int E) {
   const int64_t want = std::max<int64_t>(1, kUnitTarget / std::max<int64_t>(1, s.tiles));
   s.S = 1;
   while (s.S * 2 <= kMaxCluster && s.S * 2 <= want && s.S * 2 <= s.num_kb) s.S *= 2;
+  if (const char* env = std::getenv("MOE_ROUTE_CLUSTER")) {  // testing and tuning
+    const int v = std::atoi(env);
+    if (v == 1 || v == 2 || v == 4 || v == 8) {
+      s.S = v;
+      while (s.S > 1 && s.S > s.num_kb) s.S /= 2;  // every CTA keeps at least one k-block
+    }
+  }
   s.num_clusters = static_cast<int>(
       std::max<int64_t>(1, std::min<int64_t>(s.tiles, kUnitTarget / s.S)));
   // Shared memory: [stages][A 16 KB | B] [partials 128 x zstride] [summed logits] [barriers]
