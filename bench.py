@@ -683,7 +683,8 @@ def main():
     ep_mode = args.parallel == "ep"
     if ep_mode and args.weights != "bf16":
         raise SystemExit("--parallel ep runs bf16 expert weights")
-    if world > 1:
+    launched = "MASTER_ADDR" in os.environ  # under torchrun: its env:// rendezvous and store
+    if world > 1 or (ep_mode and launched):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     elif ep_mode:  # the exchanges need a process group, even of one rank
