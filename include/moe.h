@@ -359,6 +359,15 @@ moe_status moe_gather_rows(const void* src, int64_t n_src_rows, const int32_t* i
                            int64_t n_rows, int64_t row_bytes, void* dst, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* Failure-detection self-test; it changes no result. Enqueues one kernel that waits on a
+ * barrier that nothing completes (the state of a pipeline wait whose producer has stopped),
+ * bounded by timeout_us of wall time, with the same bounded wait the pipeline kernels use. It
+ * then records MOE_DEVERR_WAIT_TIMEOUT in the workspace's error word and returns:
+ * moe_get_device_error reports the code and clears it, and the context stays usable. ws: any
+ * workspace (at least 256 bytes). timeout_us in [1, 10^7], else MOE_ERR_INVALID_ARG. */
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t timeout_us,
+                                     void* stream);
+
 /* Zero the device error word of a new workspace (asynchronous, on `stream`). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 

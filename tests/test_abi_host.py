@@ -214,3 +214,11 @@ def test_streamed_host_entry_and_gather_reject_bad_arguments_on_host(abi):
     assert g(4096, 10, 4096, 5, 8, 4096, 4096, 128, None) == abi.MOE_ERR_INVALID_ARG  # small ws
     assert g(4096, 10, None, 5, 8, 4096, 4096, 256, None) == abi.MOE_ERR_INVALID_ARG  # no index
     assert g(4096, 10, 4096, 5, 8, 4100, 4096, 256, None) == abi.MOE_ERR_INVALID_ARG  # dst align
+
+
+def test_selftest_wait_timeout_rejects_bad_arguments_on_host(abi):
+    st = abi.lib.moe_selftest_wait_timeout
+    assert st(None, 256, 1000, None) == abi.MOE_ERR_INVALID_ARG
+    assert st(4096, 128, 1000, None) == abi.MOE_ERR_INVALID_ARG      # workspace too small
+    assert st(4096, 256, 0, None) == abi.MOE_ERR_INVALID_ARG         # timeout out of range
+    assert st(4096, 256, 10**8, None) == abi.MOE_ERR_INVALID_ARG

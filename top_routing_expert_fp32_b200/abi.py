@@ -28,7 +28,7 @@ EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_workspace_size_host", "moe
            "moe_expert_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_forward_ex",
            "moe_forward_host", "moe_expert_up_w8", "moe_expert_down_w8", "moe_forward_w8",
            "moe_pack_w8", "moe_expert_up_w8p", "moe_expert_down_w8p", "moe_forward_w8p",
-           "moe_gather_rows", "moe_forward_host_many",
+           "moe_gather_rows", "moe_forward_host_many", "moe_selftest_wait_timeout",
            "moe_workspace_init", "moe_get_device_error", "moe_status_string", "moe_last_error",
            "moe_version")
 
@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "moe_pack_w8": [PP, P, P, P, P, P, P, P],
         "moe_gather_rows": [P, I64, P, I64, I64, P, P, S, P],
         "moe_forward_host_many": [PP, I64, P, P, P, P, P, P, P, P, S, P],
+        "moe_selftest_wait_timeout": [P, S, I64, P],
         "moe_expert_up_w8p": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_down_w8p": [PP, P, P, P, P, P, P, S, P],
         "moe_forward_w8p": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
@@ -274,6 +275,10 @@ def forward_host_many(p, X_host: torch.Tensor, W_r, bias, W1, W2, W3, out_host: 
     _check(lib.moe_forward_host_many(ctypes.byref(p), nb, _ptr(X_host), _ptr(W_r), _ptr(bias),
                                      _ptr(W1), _ptr(W2), _ptr(W3), _ptr(out_host), _ptr(ws),
                                      ws.numel(), _stream(stream)))
+
+
+def selftest_wait_timeout(ws, timeout_us: int, stream=None):
+    _check(lib.moe_selftest_wait_timeout(_ptr(ws), ws.numel(), int(timeout_us), _stream(stream)))
 
 
 def device_error(ws, stream=None) -> int:

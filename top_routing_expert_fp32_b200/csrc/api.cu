@@ -963,6 +963,19 @@ moe_status moe_gather_rows(const void* src, int64_t n_src_rows, const int32_t* i
   return MOE_OK;
 }
 
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t timeout_us,
+                                     void* stream) {
+  MOE_TRY(need(ws, "ws", 256));
+  if (ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace smaller than 256 bytes");
+  if (timeout_us < 1 || timeout_us > 10000000)
+    return fail(MOE_ERR_INVALID_ARG, "timeout_us must be in [1, 1e7]");
+  MOE_CUDA(launch_wait_timeout_probe(static_cast<int*>(ws),
+                                     static_cast<uint64_t>(timeout_us) * 1000ull,
+                                     static_cast<cudaStream_t>(stream)),
+           "wait-timeout self-test");
+  return MOE_OK;
+}
+
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(need(ws, "ws", 256));
   if (ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace smaller than 256 bytes");

@@ -119,6 +119,10 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
                            const float* gate, const int32_t* offsets, const int32_t* pos,
                            const uint8_t* dropped, void* out, int* err, cudaStream_t stream);
 
+// Failure-detection self-test: one bounded wait on a barrier nothing completes; records
+// MOE_DEVERR_WAIT_TIMEOUT in *err after timeout_ns and returns.
+cudaError_t launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_t stream);
+
 int num_sms();
 
 // Message returned by moe_last_error() on the calling thread.
