@@ -236,3 +236,33 @@ def test_forward_host_many_zero_batches_is_a_no_op(abi):
     xh = torch.empty((0, cfg.N, cfg.D), dtype=torch.bfloat16).pin_memory()
     oh = torch.empty_like(xh)
     abi.forward_host_many(p, xh, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, oh, ws)
+
+
+def test_concurrent_layers_on_two_streams_equal_sequential(abi):
+    # Calls on different streams with their own workspaces share no state: run two layers
+    # (different sizes and policies) concurrently and compare with sequential runs, bit for bit.
+    cfgs = [configs.MoEConfig("s0", N=1500, D=256, F=512, E=8, k=2, dtype=configs.DTYPE_BF16,
+                              activation=configs.ACT_SILU, renormalize=1),
+            configs.MoEConfig("s1", N=900, D=128, F=256, E=16, k=2, dtype=configs.DTYPE_BF16,
+                              activation=configs.ACT_GELU_ERF, renormalize=0,
+                              capacity_factor=1.0)]
+    inps = [inputs.make_inputs(c, "cuda", seed=20 + i) for i, c in enumerate(cfgs)]
+    ps = [abi.problem(c) for c in cfgs]
+    wss = [abi.workspace(p) for p in ps]
+    seq = []
+    for c, inp, p, ws in zip(cfgs, inps, ps, wss):
+        o = torch.empty((c.N, c.D), dtype=torch.bfloat16, device="cuda")
+        abi.forward(p, inp.X, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, o, ws)
+        seq.append(o)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.empty_like(o) for o in seq]
+    for _ in range(3):
+        for c, inp, p, ws, st, o in zip(cfgs, inps, ps, wss, streams, outs):
+            abi.forward(p, inp.X, inp.W_r, inp.bias, inp.W1, inp.W2, inp.W3, o, ws,
+                        stream=st)
+    torch.cuda.synchronize()
+    for ws in wss:
+        assert abi.device_error(ws) == 0
+    for a, b in zip(seq, outs):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))

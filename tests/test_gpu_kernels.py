@@ -278,7 +278,11 @@ def test_expert_ffn_empty(abi, oracle_lib):
 @pytest.mark.parametrize("N,D,E,k,cf,dtype", [
     (1000, 4096, 8, 2, 0.0, configs.DTYPE_BF16), (500, 2048, 64, 2, 1.0, configs.DTYPE_BF16),
     (64, 64, 4, 2, 0.0, configs.DTYPE_F32), (300, 72, 5, 3, 0.4, configs.DTYPE_BF16),
-    (257, 1024, 8, 1, 0.5, configs.DTYPE_F32)])
+    (257, 1024, 8, 1, 0.5, configs.DTYPE_F32),
+    # a warp per token (N >= 16 per SM) and a block per token, with up to 8 records per token
+    (3000, 264, 8, 2, 0.0, configs.DTYPE_BF16), (2500, 136, 64, 8, 1.0, configs.DTYPE_BF16),
+    (200, 264, 64, 8, 1.0, configs.DTYPE_BF16), (100, 96, 13, 5, 0.0, configs.DTYPE_F32),
+    (2400, 100, 16, 6, 0.6, configs.DTYPE_F32)])
 def test_combine(abi, oracle_lib, N, D, E, k, cf, dtype):
     tdt = inputs.torch_dtype(dtype)
     d, ref, _ = _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=11)
@@ -303,6 +307,7 @@ def test_combine(abi, oracle_lib, N, D, E, k, cf, dtype):
 
 
 @pytest.mark.parametrize("N,D,E,k,cf,dtype", [
+    (2500, 136, 64, 8, 0.7, configs.DTYPE_BF16), (200, 96, 13, 5, 0.5, configs.DTYPE_F32),
     (500, 2048, 64, 2, 1.0, configs.DTYPE_BF16), (300, 72, 5, 3, 0.4, configs.DTYPE_BF16),
     (257, 1024, 8, 4, 0.5, configs.DTYPE_F32), (1000, 4096, 8, 2, 0.6, configs.DTYPE_BF16)])
 def test_combine_case_a_reweight(abi, oracle_lib, N, D, E, k, cf, dtype):
