@@ -65,11 +65,12 @@ def test_a2a_bytes_formula():
 class OracleCompute(ep.LocalCompute):
     """Each step of a rank's layer by the oracle (fp32 inputs, fp64 arithmetic)."""
 
-    def __init__(self, W_r, bias, W1, W2, W3, k, cf, renorm, act):
+    def __init__(self, W_r, bias, W1, W2, W3, k, cf, renorm, act, order=0, policy=0):
         import oracle
         self.o = oracle
         self.W_r, self.bias, self.W1, self.W2, self.W3 = W_r, bias, W1, W2, W3
         self.k, self.cf, self.renorm, self.act = k, cf, renorm, act
+        self.order, self.policy = order, policy
 
     def route_dispatch(self, X):
         o = self.o
@@ -77,7 +78,7 @@ class OracleCompute(ep.LocalCompute):
         E = self.W_r.shape[1]
         _, l32 = o.router_logits(X, o.F32, self.W_r, self.bias)
         ro = o.route(l32, k=self.k, renorm=self.renorm)
-        do = o.dispatch(ro["idx"], E, o.capacity(N, self.k, E, self.cf))
+        do = o.dispatch(ro["idx"], E, o.capacity(N, self.k, E, self.cf), order=self.order)
         X_perm = torch.from_numpy(np.ascontiguousarray(X[do["row_token"]], dtype=np.float32))
         return dict(offsets=torch.from_numpy(do["offsets"].astype(np.int32)), X_perm=X_perm,
                     idx=ro["idx"], gate=ro["gate"], pos=do["pos"], dropped=do["dropped"])
@@ -105,7 +106,7 @@ class OracleCompute(ep.LocalCompute):
             for j in range(k):
                 if not r["dropped"][t, j]:
                     Yrec[t, j] = Y[off[r["idx"][t, j]] + r["pos"][t, j]]
-        return torch.from_numpy(self.o.combine(r["gate"], r["dropped"], Yrec))
+        return torch.from_numpy(self.o.combine(r["gate"], r["dropped"], Yrec, self.policy))
 
 
 def _weights(E, D, F, seed=5):
@@ -127,10 +128,11 @@ def _worker(rank, world, port, case, results):
         W_r, bias, W1, W2, W3 = _weights(E, D, F)
         N = case["N"] + 7 * rank                        # ragged batches across ranks
         X = np.random.default_rng(100 + rank).standard_normal((N, D)).astype(np.float32)
-        comp = OracleCompute(W_r, bias, W1, W2, W3, k, cf, 1, 0)
+        order, policy = case.get("order", 0), case.get("policy", 0)
+        comp = OracleCompute(W_r, bias, W1, W2, W3, k, cf, 1, 0, order, policy)
         out, info = ep.forward(comp, X, E)
         ref = oracle.forward(X, W_r, bias, W1, W2, W3, k=k, cf=cf, renorm=1, act=0,
-                             dtype=oracle.F32)
+                             dtype=oracle.F32, order=order, drop_policy=policy)
         results[rank] = (float(np.abs(out.numpy() - ref["out"]).max()),
                          int(ref["dropped"].sum()), info["plan"].send_rows,
                          info["plan"].recv_rows)
@@ -144,7 +146,10 @@ def _worker(rank, world, port, case, results):
     (3, dict(E=8, D=16, F=32, k=2, N=33, cf=0.0)),     # expert blocks of 3, 3, 2
     (3, dict(E=4, D=16, F=32, k=1, N=25, cf=1.25)),    # blocks of 2, 1, 1
     (3, dict(E=2, D=16, F=32, k=2, N=20, cf=0.0)),     # rank 2 owns no expert
-], ids=["w2", "w2_capacity", "w3_uneven", "w3_k1_capacity", "w3_more_ranks_than_experts"])
+    # token-major capacity order and the case-A reweight of kept gates (MoE series 2.2)
+    (2, dict(E=6, D=16, F=32, k=3, N=45, cf=0.8, order=1, policy=1)),
+], ids=["w2", "w2_capacity", "w3_uneven", "w3_k1_capacity", "w3_more_ranks_than_experts",
+        "w2_token_major_case_a"])
 def test_ep_forward_equals_single_device_layer_gloo(world, case):
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
