@@ -472,6 +472,15 @@ def run_gpu(args, cfg, world, rank, device):
         del xh_many, oh_many
     h2d = N * D * es
     d2h = N * D * es
+    # The layer's diagnostics (an extra, untimed route call that also writes prob_colsum).
+    colsum = torch.empty((E,), dtype=torch.float32, device=device)
+    abi.route(p, inp.X, inp.W_r, inp.bias, None, idx, gate, colsum, ws)
+    abi.dispatch(p, inp.X, idx, load, offsets, pos, dropped, row_token, X_perm, ws)
+    torch.cuda.synchronize(device)
+    load_h = load.cpu().double()
+    diagnostics = {"balance_loss": abi.balance_loss(p, load, colsum),
+                   "drop_rate": abi.drop_rate(p, dropped),
+                   "load_max_over_mean": float(load_h.max() / load_h.mean())}
     barrier(device)
 
     line = {
@@ -487,6 +496,7 @@ def run_gpu(args, cfg, world, rank, device):
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "flushed between steps (512 MiB write + read-back, outside the step events)",
                    "kept_records": kept,
+                   "diagnostics": diagnostics,
                    "grouped_gemm_TFLOP/s": gemm_tflops,
                    "grouped_gemm_frac_bf16_peak": gemm_tflops / tc,
                    "kernels": kern},

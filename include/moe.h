@@ -359,6 +359,18 @@ moe_status moe_gather_rows(const void* src, int64_t n_src_rows, const int32_t* i
                            int64_t n_rows, int64_t row_bytes, void* dst, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* Host only: the layer's diagnostics, in fp64 from host copies of its [E] and [N,k] outputs.
+ * Balance loss (MoE formula-to-code walkthrough 2.1-2.3; MoE series 7.3):
+ *   loss = E * sum_e f_e * P_e,  f_e = load[e] / (N*k),  P_e = prob_colsum[e] / N,
+ * with load from moe_dispatch (records per expert before capacity) and prob_colsum from
+ * moe_route (the column sums of the full softmax); uniform routing gives exactly 1 for any k.
+ * Drop rate (walkthrough 3.3): dropped records / (N*k) over the routing slots, dropped [N,k]
+ * from moe_dispatch. Pointers are host pointers; N == 0 gives 0. Errors: MOE_ERR_INVALID_ARG
+ * for a NULL pointer or an invalid problem. */
+moe_status moe_balance_loss(const moe_problem* p, const int32_t* load, const float* prob_colsum,
+                            double* loss);
+moe_status moe_drop_rate(const moe_problem* p, const uint8_t* dropped, double* rate);
+
 /* Failure-detection self-test; it changes no result. Enqueues one kernel that waits on a
  * barrier that nothing completes (the state of a pipeline wait whose producer has stopped),
  * bounded by timeout_us of wall time, with the same bounded wait the pipeline kernels use. It

@@ -6,7 +6,9 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -222,3 +224,35 @@ def test_selftest_wait_timeout_rejects_bad_arguments_on_host(abi):
     assert st(4096, 128, 1000, None) == abi.MOE_ERR_INVALID_ARG      # workspace too small
     assert st(4096, 256, 0, None) == abi.MOE_ERR_INVALID_ARG         # timeout out of range
     assert st(4096, 256, 10**8, None) == abi.MOE_ERR_INVALID_ARG
+
+
+def test_diagnostics_host_functions_match_the_oracle(abi, oracle_lib):
+    # Host-only entry points (no device work): balance loss E * sum f_e P_e and drop rate.
+    from top_routing_expert_fp32_b200 import configs
+    rng = np.random.default_rng(7)
+    for N, E, k in ((64, 4, 2), (1000, 64, 2), (333, 13, 5), (5, 8, 1)):
+        cfg = configs.MoEConfig("d", N=N, D=64, F=64, E=E, k=k, dtype=configs.DTYPE_BF16,
+                                activation=0, renormalize=1)
+        p = abi.problem(cfg)
+        load = rng.multinomial(N * k, rng.dirichlet(np.ones(E))).astype(np.int32)
+        colsum = (rng.dirichlet(np.ones(E)) * N).astype(np.float32)
+        got = abi.balance_loss(p, torch.from_numpy(load), torch.from_numpy(colsum))
+        want = oracle_lib.balance_loss(N, k, load, colsum.astype(np.float64))
+        assert got == pytest.approx(want, rel=1e-12, abs=0)
+        # uniform routing: exactly 1 whatever k ([W] 2.2)
+        if (N * k) % E == 0 and N % E == 0:
+            u = abi.balance_loss(p, torch.full((E,), N * k // E, dtype=torch.int32),
+                                 torch.full((E,), N / E, dtype=torch.float32))
+            assert u == pytest.approx(1.0, rel=1e-12)
+        dropped = (rng.random((N, k)) < 0.3).astype(np.uint8)
+        assert abi.drop_rate(p, torch.from_numpy(dropped)) == pytest.approx(
+            oracle_lib.drop_rate(dropped), rel=0, abs=0)
+    cfg0 = configs.MoEConfig("d0", N=0, D=64, F=64, E=4, k=2, dtype=configs.DTYPE_BF16,
+                             activation=0, renormalize=1)
+    p0 = abi.problem(cfg0)
+    z = torch.zeros(4, dtype=torch.int32)
+    assert abi.balance_loss(p0, z, z.float()) == 0.0
+    assert abi.drop_rate(p0, torch.zeros((0, 2), dtype=torch.uint8)) == 0.0
+    out = ctypes.c_double()
+    assert abi.lib.moe_balance_loss(ctypes.byref(p0), None, 16, ctypes.byref(out)) == \
+        abi.MOE_ERR_INVALID_ARG

@@ -266,3 +266,39 @@ def test_concurrent_layers_on_two_streams_equal_sequential(abi):
         assert abi.device_error(ws) == 0
     for a, b in zip(seq, outs):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["capacity", "mixtral"])
+def test_diagnostics_from_the_layer_match_the_oracle(abi, name):
+    # Balance loss and drop rate (moe_balance_loss / moe_drop_rate) from the GPU layer's own
+    # load, prob_colsum and dropped, against the oracle's routing of the same inputs.
+    cfg = configs.CONFIGS[name]
+    inp = inputs.make_inputs(cfg, "cuda", weights=False)
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    r = alloc_route_out(cfg.N, cfg.E, cfg.k)
+    d = alloc_dispatch_out(cfg.N, cfg.E, cfg.k)
+    X_perm = torch.empty((cfg.N * cfg.k, cfg.D), dtype=inp.X.dtype, device="cuda")
+    abi.route(p, inp.X, inp.W_r, inp.bias, r["logits"], r["idx"], r["gate"], r["colsum"], ws)
+    abi.dispatch(p, inp.X, r["idx"], d["load"], d["offsets"], d["pos"], d["dropped"],
+                 d["row_token"], X_perm, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    loss = abi.balance_loss(p, d["load"], r["colsum"])
+    rate = abi.drop_rate(p, d["dropped"])
+    Xn = np_host(inp.X)
+    bias = None if inp.bias is None else inp.bias.cpu().numpy()
+    l64, l32 = oracle.router_logits(Xn, oracle_dtype(cfg), inp.W_r.cpu().numpy(), bias)
+    ro = oracle.route(l32, k=cfg.k, renorm=cfg.renormalize)
+    flips = int((r["idx"].cpu().numpy() != ro["idx"]).any(1).sum())
+    do = oracle.dispatch(ro["idx"], cfg.E, oracle.capacity(cfg.N, cfg.k, cfg.E,
+                                                           cfg.capacity_factor))
+    ref_loss = oracle.balance_loss(cfg.N, cfg.k, do["load"], ro["colsum"])
+    ref_rate = oracle.drop_rate(do["dropped"])
+    # a near-tie flip moves one record between experts: 1 / (N k) in f, a few in the drops
+    assert loss == pytest.approx(ref_loss, rel=1e-4 + 4 * flips / (cfg.N * cfg.k))
+    assert abs(rate - ref_rate) <= 2 * flips / (cfg.N * cfg.k) + 1e-12
+    if name == "capacity":
+        assert rate > 0.0
+    del X_perm
+    torch.cuda.empty_cache()

@@ -29,6 +29,7 @@ EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_workspace_size_host", "moe
            "moe_forward_host", "moe_expert_up_w8", "moe_expert_down_w8", "moe_forward_w8",
            "moe_pack_w8", "moe_expert_up_w8p", "moe_expert_down_w8p", "moe_forward_w8p",
            "moe_gather_rows", "moe_forward_host_many", "moe_selftest_wait_timeout",
+           "moe_balance_loss", "moe_drop_rate",
            "moe_workspace_init", "moe_get_device_error", "moe_status_string", "moe_last_error",
            "moe_version")
 
@@ -78,6 +79,8 @@ def _load() -> ctypes.CDLL:
         "moe_gather_rows": [P, I64, P, I64, I64, P, P, S, P],
         "moe_forward_host_many": [PP, I64, P, P, P, P, P, P, P, P, S, P],
         "moe_selftest_wait_timeout": [P, S, I64, P],
+        "moe_balance_loss": [PP, P, P, ctypes.POINTER(ctypes.c_double)],
+        "moe_drop_rate": [PP, P, ctypes.POINTER(ctypes.c_double)],
         "moe_expert_up_w8p": [PP, P, P, P, P, P, P, P, P, S, P],
         "moe_expert_down_w8p": [PP, P, P, P, P, P, P, S, P],
         "moe_forward_w8p": [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
@@ -275,6 +278,23 @@ def forward_host_many(p, X_host: torch.Tensor, W_r, bias, W1, W2, W3, out_host: 
     _check(lib.moe_forward_host_many(ctypes.byref(p), nb, _ptr(X_host), _ptr(W_r), _ptr(bias),
                                      _ptr(W1), _ptr(W2), _ptr(W3), _ptr(out_host), _ptr(ws),
                                      ws.numel(), _stream(stream)))
+
+
+def balance_loss(p, load, prob_colsum) -> float:
+    """load [E] int32, prob_colsum [E] fp32: host tensors (device tensors are copied)."""
+    ld = load.detach().to("cpu", torch.int32).contiguous()
+    cs = prob_colsum.detach().to("cpu", torch.float32).contiguous()
+    out = ctypes.c_double()
+    _check(lib.moe_balance_loss(ctypes.byref(p), _ptr(ld), _ptr(cs), ctypes.byref(out)))
+    return out.value
+
+
+def drop_rate(p, dropped) -> float:
+    """dropped [N,k] uint8: a host tensor (a device tensor is copied)."""
+    d = dropped.detach().to("cpu", torch.uint8).contiguous()
+    out = ctypes.c_double()
+    _check(lib.moe_drop_rate(ctypes.byref(p), _ptr(d), ctypes.byref(out)))
+    return out.value
 
 
 def selftest_wait_timeout(ws, timeout_us: int, stream=None):

@@ -963,6 +963,35 @@ moe_status moe_gather_rows(const void* src, int64_t n_src_rows, const int32_t* i
   return MOE_OK;
 }
 
+moe_status moe_balance_loss(const moe_problem* p, const int32_t* load, const float* prob_colsum,
+                            double* loss) {
+  MOE_TRY(check_problem(p));
+  if (load == nullptr || prob_colsum == nullptr || loss == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "load, prob_colsum and loss must not be NULL");
+  *loss = 0.0;
+  if (p->N == 0) return MOE_OK;
+  const double records = static_cast<double>(p->N) * static_cast<double>(p->k);
+  const double tokens = static_cast<double>(p->N);
+  double sum = 0.0;
+  for (int32_t e = 0; e < p->E; ++e)  // f_e = share of the records, P_e = mean probability
+    sum += (static_cast<double>(load[e]) / records) * (static_cast<double>(prob_colsum[e]) / tokens);
+  *loss = static_cast<double>(p->E) * sum;
+  return MOE_OK;
+}
+
+moe_status moe_drop_rate(const moe_problem* p, const uint8_t* dropped, double* rate) {
+  MOE_TRY(check_problem(p));
+  if (rate == nullptr) return fail(MOE_ERR_INVALID_ARG, "rate must not be NULL");
+  *rate = 0.0;
+  const int64_t records = p->N * static_cast<int64_t>(p->k);
+  if (records == 0) return MOE_OK;
+  if (dropped == nullptr) return fail(MOE_ERR_INVALID_ARG, "dropped must not be NULL");
+  int64_t n = 0;
+  for (int64_t r = 0; r < records; ++r) n += dropped[r] != 0 ? 1 : 0;
+  *rate = static_cast<double>(n) / static_cast<double>(records);
+  return MOE_OK;
+}
+
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t timeout_us,
                                      void* stream) {
   MOE_TRY(need(ws, "ws", 256));
