@@ -202,12 +202,18 @@ moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk
  *   - Limit: ceil(N*k / 1024) * E <= 16384 counters (e.g. N*k <= 262144 records at E = 64);
  *     larger problems return MOE_ERR_UNSUPPORTED -- use moe_dispatch.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     (cudaGetSymbolAddress) and, under CUDA's lazy module loading, may load this library's
+ *     kernels into the device's context, which takes device memory the driver allocates
+ *     itself. Make that first call during set-up, before any stream capture and before the
+ *     code that must not allocate starts. After cudaDeviceReset the device gets a new
+ *     context and the next call looks the address up again.
  *   - Every call shares the one array: calls that may overlap on the GPU (different streams,
  *     or different host threads on one device) race and must be serialised by the caller.
  *     Each call rewrites every counter it reads, so no clearing is needed between calls.
- *   - Out-of-range expert indices are treated as dropped but not reported (there is no
- *     workspace error word).
+ *   - Out-of-range expert indices are treated as dropped but not reported, and neither is a
+ *     gather whose bounded wait on its copy barrier ran out (X_perm may then be partly
+ *     written): there is no workspace error word on this path. Callers that need those
+ *     reports use moe_dispatch.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
 moe_status moe_dispatch_noalloc(const moe_problem* p, const void* X, const int32_t* topk_idx,
                                 int32_t* load, int32_t* offsets, int32_t* pos, uint8_t* dropped,
@@ -239,7 +245,12 @@ moe_status moe_expert_down(const moe_problem* p, const void* H, const int32_t* o
  * with g = topk_gate, except under MOE_DROP_RENORM_KEPT for a token with both dropped and kept
  * slots: g[t,j] = topk_gate[t,j] / (sum of its kept slots' gates, fp32, ascending j).
  * Accumulated in fp32 in ascending j, rounded once to the output dtype; a token whose slots
- * are all dropped gets 0. `dropped` may be NULL (nothing dropped). No atomics. */
+ * are all dropped gets 0. `dropped` may be NULL only without a capacity
+ * (capacity_factor <= 0: nothing is dropped); with a capacity it is required
+ * (MOE_ERR_INVALID_ARG otherwise). A kept record whose expert index or position falls outside
+ * its expert's segment [offsets[e], offsets[e+1]) contributes nothing and is not read; no
+ * workspace is passed here, so it is not reported (moe_forward reports it as
+ * MOE_DEVERR_BAD_INDEX). No atomics. */
 moe_status moe_combine(const moe_problem* p, const void* Y, const int32_t* topk_idx,
                        const float* topk_gate, const int32_t* offsets, const int32_t* pos,
                        const uint8_t* dropped, void* out, void* stream);

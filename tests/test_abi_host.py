@@ -256,3 +256,18 @@ def test_diagnostics_host_functions_match_the_oracle(abi, oracle_lib):
     out = ctypes.c_double()
     assert abi.lib.moe_balance_loss(ctypes.byref(p0), None, 16, ctypes.byref(out)) == \
         abi.MOE_ERR_INVALID_ARG
+
+
+def test_combine_needs_the_drop_flags_under_a_capacity(abi):
+    # With a capacity some records are dropped and only `dropped` says which; without it the
+    # kernel would take every position as a row of Y. Rejected on the host; accepted (still
+    # nothing enqueued here: N = 0) without a capacity.
+    from top_routing_expert_fp32_b200 import configs
+    for cf, want in ((1.25, abi.MOE_ERR_INVALID_ARG), (0.0, abi.MOE_OK)):
+        cfg = configs.MoEConfig("c", N=0, D=64, F=64, E=8, k=2, dtype=configs.DTYPE_BF16,
+                                activation=0, renormalize=1, capacity_factor=cf)
+        p = abi.problem(cfg)
+        st = abi.lib.moe_combine(ctypes.byref(p), 4096, 4096, 4096, 4096, 4096, None, 4096, None)
+        assert st == want, abi.lib.moe_last_error()
+        if want != abi.MOE_OK:
+            assert b"dropped" in abi.lib.moe_last_error()

@@ -1,7 +1,12 @@
 """moe_dispatch_noalloc: the dispatch step for callers that cannot give the library device
 memory (no cudaMalloc once they run, or all device memory owned by their own pool). Its
 results must equal moe_dispatch's, call after call, with the counters kept in the library's
-fixed array instead of a workspace. This file is collected last on purpose."""
+fixed array instead of a workspace, and a call after the first must leave the device's free
+memory unchanged.
+
+The file name sorts last so that pytest collects it after every other test file: a run that
+stops at the first failure (-x) has then already run the rest of the suite when this one
+fails. It also passes when run alone in a fresh process."""
 import ctypes
 
 import numpy as np
@@ -34,7 +39,7 @@ def test_noalloc_rejects_oversized_problems_on_host():
     assert st == abi.MOE_ERR_INVALID_ARG   # row_token is required
 
 
-def _run_both(abi, cfg, idx_np, X=None):
+def _run_both(abi, cfg, idx_np, X=None, check_free=False):
     N, E, k = cfg.N, cfg.E, cfg.k
     p = abi.problem(cfg)
     idx = torch.from_numpy(idx_np).cuda()
@@ -52,9 +57,14 @@ def _run_both(abi, cfg, idx_np, X=None):
     ws = abi.workspace(p)
     abi.dispatch(p, X, idx, ref["load"], ref["offsets"], ref["pos"], ref["dropped"],
                  ref["row_token"], ref["X_perm"], ws)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
     abi.dispatch_noalloc(p, X, idx, got["load"], got["offsets"], got["pos"], got["dropped"],
                          got["row_token"], got["X_perm"])
     torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    if check_free:  # the device's free memory (cudaMemGetInfo) is what an allocation would take
+        assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
     kept = int(ref["offsets"][E].item())
     for key in ("load", "offsets", "pos", "dropped"):
         assert torch.equal(ref[key], got[key]), key
@@ -81,5 +91,5 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice_in_a_row():
     cfg2 = _cfg(3001, 8, 2, 0.0)
     idx2 = oracle.route(inputs.make_logits(cfg2.N, cfg2.E, seed=22).numpy(), k=2,
                         renorm=1)["idx"]
-    kept2 = _run_both(abi, cfg2, idx2)
+    kept2 = _run_both(abi, cfg2, idx2, check_free=True)
     assert kept2 == cfg2.N * cfg2.k

@@ -201,6 +201,7 @@ T* at(void* ws, size_t off) {
 
 moe_status run_up(const moe_problem& p, const void* X_perm, const int32_t* offsets,
                   const void* W1, const void* W2, void* H, int* err, cudaStream_t stream) {
+  NvtxRange range("moe expert up");
   if (p.dtype == MOE_DTYPE_BF16) {
     MOE_TRY(check_sm100());
     MOE_CUDA(launch_ffn_up_sm100(p, X_perm, offsets, W1, W2, H, err, wait_timeout_ns(), stream),
@@ -213,6 +214,7 @@ moe_status run_up(const moe_problem& p, const void* X_perm, const int32_t* offse
 
 moe_status run_down(const moe_problem& p, const void* H, const int32_t* offsets, const void* W3,
                     void* Y, int* err, cudaStream_t stream) {
+  NvtxRange range("moe expert down");
   if (p.dtype == MOE_DTYPE_BF16) {
     MOE_TRY(check_sm100());
     MOE_CUDA(launch_ffn_down_sm100(p, H, offsets, W3, Y, err, wait_timeout_ns(), stream),
@@ -252,6 +254,7 @@ bool use_w8t(const moe_problem& p) {
 moe_status run_up_w8(const moe_problem& p, const void* X_perm, const int32_t* offsets,
                      const int8_t* Q1, const float* S1, const int8_t* Q2, const float* S2,
                      void* H, bool packed, int* err, cudaStream_t stream) {
+  NvtxRange range("moe expert up (8-bit)");
   MOE_TRY(check_sm100());
   if (packed || use_w8t(p))
     MOE_CUDA(launch_ffn_up_w8t(p, X_perm, offsets, Q1, S1, Q2, S2, H, packed, err,
@@ -267,6 +270,7 @@ moe_status run_up_w8(const moe_problem& p, const void* X_perm, const int32_t* of
 moe_status run_down_w8(const moe_problem& p, const void* H, const int32_t* offsets,
                        const int8_t* Q3, const float* S3, void* Y, bool packed, int* err,
                        cudaStream_t stream) {
+  NvtxRange range("moe expert down (8-bit)");
   MOE_TRY(check_sm100());
   if (packed || use_w8t(p))
     MOE_CUDA(launch_ffn_down_w8t(p, H, offsets, Q3, S3, Y, packed, err, wait_timeout_ns(),
@@ -309,6 +313,7 @@ moe_status need_topk(const moe_problem& p) {
 moe_status route_impl(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                       const float* noise, float* logits, int32_t* topk_idx, float* topk_gate,
                       float* prob_colsum, float* z_loss, void* ws, cudaStream_t s) {
+  NvtxRange range("moe route");
   const Layout L = make_layout(p);
   if (p.N == 0) {
     if (prob_colsum) MOE_CUDA(cudaMemsetAsync(prob_colsum, 0, sizeof(float) * p.E, s), "memset");
@@ -348,11 +353,15 @@ moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, c
     return MOE_OK;
   }
   MOE_TRY(route_impl(p, X, W_r, bias, noise, logits, idx, gate, prob_colsum, z_loss, ws, stream));
-  MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps, dr,
-                              row_token, err, stream),
-           "slot assign");
-  MOE_CUDA(launch_gather(p, X, row_token, off, xperm, err, stream), "gather");
+  {
+    NvtxRange range("moe dispatch");
+    MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps,
+                                dr, row_token, err, stream),
+             "slot assign");
+    MOE_CUDA(launch_gather(p, X, row_token, off, xperm, err, stream), "gather");
+  }
   MOE_TRY(run_ffn(p, xperm, off, w, h, y, err, stream));
+  NvtxRange range("moe combine");
   MOE_CUDA(launch_combine(p, y, idx, gate, off, ps, dr, out, err, stream), "combine");
   return MOE_OK;
 }
@@ -449,6 +458,7 @@ moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* err = at<int>(ws, L.err);
   int32_t* rt = row_token ? row_token : at<int32_t>(ws, L.row_token);
+  NvtxRange range("moe dispatch");
   MOE_CUDA(launch_slot_assign(*p, capacity_of(*p), topk_idx, at<int32_t>(ws, L.counts), load,
                               offsets, pos, dropped, rt, err, s),
            "slot assign");
@@ -516,8 +526,13 @@ moe_status moe_combine(const moe_problem* p, const void* Y, const int32_t* topk_
   MOE_TRY(need(topk_gate, "topk_gate", 4));
   MOE_TRY(need(offsets, "offsets", 4));
   MOE_TRY(need(pos, "pos", 4));
-  MOE_TRY(opt(dropped, "dropped", 1));
+  // Under a capacity some records may be dropped, and only the flags say which.
+  if (p->capacity_factor > 0.0)
+    MOE_TRY(need(dropped, "dropped (required when capacity_factor > 0)", 1));
+  else
+    MOE_TRY(opt(dropped, "dropped", 1));
   MOE_TRY(need(out, "out"));
+  NvtxRange range("moe combine");
   MOE_CUDA(launch_combine(*p, Y, topk_idx, topk_gate, offsets, pos, dropped, out, nullptr,
                           static_cast<cudaStream_t>(stream)),
            "combine");

@@ -83,7 +83,19 @@ __global__ void __launch_bounds__(kThreads)
       record_error(err, MOE_DEVERR_BAD_INDEX);
       keep = false;
     }
-    my_row = keep ? static_cast<int64_t>(offsets[e]) + pos[rec] : -1;
+    if (keep) {
+      // A kept record's row lies inside its expert's segment; a position outside it (a
+      // dropped record passed without its flag, or a corrupt pos) is reported and skipped,
+      // so no row past the segment, or past the end of Y, is ever read.
+      const int32_t ps = pos[rec];
+      const int32_t seg0 = offsets[e];
+      if (ps < 0 || ps >= offsets[e + 1] - seg0) {
+        record_error(err, MOE_DEVERR_BAD_INDEX);
+        keep = false;
+      } else {
+        my_row = static_cast<int64_t>(seg0) + ps;
+      }
+    }
     my_g = gate[rec];
   }
   int64_t row[KMAX];

@@ -10,9 +10,20 @@
 
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/moe.h"
 
 namespace moe {
+
+// NVTX range around the enqueueing of one stage (route, dispatch, expert up/down, combine),
+// seen by profilers that attach to NVTX (ncu --nvtx, nsys); header-only, a no-op otherwise.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Upper bound on router partial-sum blocks (the launcher never exceeds it).
 int route_num_blocks(int64_t N, int E);

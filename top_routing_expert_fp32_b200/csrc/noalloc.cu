@@ -20,21 +20,44 @@ namespace {
 constexpr int kScratchInts = 16384;  // 64 KiB
 static __device__ __align__(256) int32_t g_dispatch_counts[kScratchInts];
 
-// Device address of g_dispatch_counts, looked up once per device with that device current.
-// In host code the symbol itself is only a host-side stand-in, never a device address.
+// The calling thread's current CUDA context (driver handle), or nullptr if it cannot be read.
+CUcontext current_context() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  static GetCurrent fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<GetCurrent>(nullptr);
+    return reinterpret_cast<GetCurrent>(ptr);
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_dispatch_counts, looked up once per device (and context) with that
+// device current. In host code the symbol itself is only a host-side stand-in, never a device
+// address. The address belongs to the context the module was loaded into: after
+// cudaDeviceReset the device gets a new primary context, whose handle differs, and the
+// address is looked up again.
 cudaError_t scratch_address(int32_t** out) {
   static std::mutex mu;
   static int32_t* addr[64] = {nullptr};
+  static CUcontext ctx[64] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const CUcontext cur = current_context();  // nullptr before the device's first runtime call
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || cur == nullptr || ctx[dev] != cur) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_dispatch_counts);
+    e = cudaGetSymbolAddress(&p, g_dispatch_counts);  // sets up the primary context if needed
     if (e != cudaSuccess) return e;
     addr[dev] = static_cast<int32_t*>(p);
+    ctx[dev] = current_context();
   }
   *out = addr[dev];
   return cudaSuccess;
