@@ -89,6 +89,81 @@ def test_route_from_x(abi, oracle_lib, dtype, N, D, E, k, renorm, bias_var):
     np.testing.assert_allclose(o["colsum"].cpu().numpy(), ref["colsum"], rtol=1e-4, atol=1e-4)
 
 
+# Routing from X, checked on the GPU's own logits: the kernels that compute the logits take the
+# routing decision in registers (bf16 X: the tensor-core router at every cluster size; fp32 X:
+# the narrow and wide SIMT routers). Duplicate columns of W_r (and of the bias) make the
+# logits of those experts bit-identical, so exact ties reach the in-kernel selection.
+ROUTE_X_TIES = [
+    # dtype, N, D, E, k, renorm, bias_var, cluster (MOE_ROUTE_CLUSTER; None = automatic)
+    (configs.DTYPE_BF16, 515, 1024, 8, 2, 1, 0.0, 1),
+    (configs.DTYPE_BF16, 515, 1024, 8, 2, 0, 1.0, 2),
+    (configs.DTYPE_BF16, 515, 1024, 8, 3, 1, 0.0, 4),
+    (configs.DTYPE_BF16, 515, 1024, 8, 2, 0, 0.0, 8),
+    (configs.DTYPE_BF16, 130, 4096, 8, 2, 1, 0.0, None),
+    (configs.DTYPE_BF16, 1000, 2048, 64, 2, 1, 2.0, 1),
+    (configs.DTYPE_BF16, 300, 2048, 64, 8, 0, 2.0, 8),
+    (configs.DTYPE_BF16, 777, 512, 13, 5, 0, 1.0, 2),
+    (configs.DTYPE_BF16, 64, 6144, 8, 2, 0, 0.0, None),
+    (configs.DTYPE_BF16, 257, 640, 33, 3, 1, 0.0, 4),
+    (configs.DTYPE_F32, 300, 200, 8, 2, 1, 0.0, None),     # narrow
+    (configs.DTYPE_F32, 130, 100, 16, 4, 0, 1.0, None),    # narrow, 16 experts
+    (configs.DTYPE_F32, 300, 200, 24, 2, 0, 0.0, None),    # wide
+    (configs.DTYPE_F32, 129, 64, 64, 8, 1, 2.0, None),     # wide, 64 experts
+]
+
+
+@pytest.mark.parametrize("dtype,N,D,E,k,renorm,bias_var,cluster", ROUTE_X_TIES)
+def test_route_from_x_bitexact_on_own_logits_with_ties(abi, oracle_lib, monkeypatch, dtype, N,
+                                                       D, E, k, renorm, bias_var, cluster):
+    if cluster is None:
+        monkeypatch.delenv("MOE_ROUTE_CLUSTER", raising=False)
+    else:
+        monkeypatch.setenv("MOE_ROUTE_CLUSTER", str(cluster))
+    cfg = _cfg(N, D, 64, E, k, dtype=dtype, renorm=renorm, bias_var=bias_var)
+    inp = inputs.make_inputs(cfg, "cuda", seed=5, weights=False)
+    # expert e + E/2 (and e + 1 for a few odd E) repeats expert e's column and bias
+    W_r = inp.W_r.clone()
+    bias = None if inp.bias is None else inp.bias.clone()
+    pairs = [(e, e + E // 2) for e in range(0, E // 2, 2)] or [(0, 0)]
+    for src, dst in pairs:
+        W_r[:, dst] = W_r[:, src]
+        if bias is not None:
+            bias[dst] = bias[src]
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    o = alloc_route_out(N, E, k)
+    abi.route(p, inp.X, W_r, bias, o["logits"], o["idx"], o["gate"], o["colsum"], ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    lg = o["logits"].cpu().numpy()
+    for src, dst in pairs:   # the ties are real: equal columns give bit-identical logits
+        assert np.array_equal(lg[:, src].view(np.int32), lg[:, dst].view(np.int32))
+    # router arithmetic: within the fp32 accumulation bound of the fp64 logits
+    Wn = W_r.cpu().numpy()
+    l64, _ = oracle_lib.router_logits(np_host(inp.X), oracle_dtype(cfg), Wn,
+                                      None if bias is None else bias.cpu().numpy())
+    scale = np.abs(to_f64(inp.X)) @ np.abs(Wn.astype(np.float64))
+    assert (np.abs(lg.astype(np.float64) - l64) <= 1e-5 * scale + 1e-6).all()
+    # selection, order (lower index first on ties) and gates: bit-exact on the same logits
+    ref = oracle_lib.route(lg, k=k, renorm=renorm)
+    idx = o["idx"].cpu().numpy()
+    assert np.array_equal(idx, ref["idx"])
+    np.testing.assert_allclose(o["gate"].cpu().numpy(), ref["gate"], rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(o["colsum"].cpu().numpy(), ref["colsum"], rtol=1e-5, atol=1e-5)
+    # some selections were decided by the tie rule: both copies of a tied expert selected,
+    # the lower index first
+    tie_decided = 0
+    for src, dst in pairs:
+        if src == dst:
+            continue
+        both = (idx == src).any(1) & (idx == dst).any(1)
+        first_src = np.argmax(idx == src, axis=1) < np.argmax(idx == dst, axis=1)
+        assert first_src[both].all()
+        tie_decided += int(both.sum())
+    if E >= 4 and k >= 2:
+        assert tie_decided > 0
+
+
 # ------------------------------------------------------------------ dispatch (bit-exact)
 
 def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, X=None,
