@@ -1,6 +1,7 @@
 """Throughput benchmark of the MoE FFN forward layer on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+python bench.py --all-workloads [--table PATH]   (one line per workload, and a markdown table)
 
 A step is one pass of the whole hot path (route -> dispatch -> expert up/down -> combine)
 over one batch of the workload, enqueued through the C ABI with CUDA events between the
@@ -9,8 +10,11 @@ kernels (the same kernels moe_forward launches). Inputs are resident in HBM; L2 
 line. With N>1 (torchrun) every rank runs an independent replica on its own GPU (the layer
 has no data-path collective); value = tokens of all ranks / max-over-ranks time.
 
---impl reference times the CPU oracle on the host cores (a bounded token sample of the same
-workload) and prints the same line with "impl": "reference".
+--impl reference times the CPU oracle on the host cores: K steps after W warm-up steps, each
+step the oracle's forward on a bounded token sample of the same workload (the throughput is
+extrapolated to the workload's N), and prints the same line with "impl": "reference".
+
+Without --steps, K is chosen after the warm-up so that the timed region lasts about 1.5 s.
 """
 from __future__ import annotations
 
@@ -31,6 +35,12 @@ if ROOT not in sys.path:
 METRIC = "MoE fwd tokens/s; grouped-GEMM TFLOP/s & %bf16 peak; route/combine % HBM BW"
 L2_FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Datasheet figures of one B200 (dense, no sparsity), for the second denominator of every
+# fraction: 2.25 PFLOP/s bf16 at the 1965 MHz maximum SM clock, 8 TB/s HBM3e.
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
+DATASHEET_SM_MHZ = 1965.0
+TIMED_REGION_TARGET_S = 1.5
 
 
 # ------------------------------------------------------------------ small host helpers
@@ -109,7 +119,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period_s: float = 0.05):
+    def __init__(self, device_index: int, period_s: float = 0.01):
         self.samples = []  # (t, sm_mhz, reasons_mask)
         self.period = period_s
         self.ok = False
@@ -192,48 +202,117 @@ def traffic_from_profile(kernel: str, workload: str):
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def oracle_tokens_per_s(cfg, budget_s: float = 12.0, w8: bool = False):
-    """The oracle (as it stands) on a bounded token sample of the workload. Without capacity the
-    tokens are independent, so a prefix of the batch is the same computation per token; with
-    capacity the sample is its own batch of n tokens (capacity recomputed for n)."""
-    import numpy as np
-    import torch
-    import oracle
-    from top_routing_expert_fp32_b200 import configs, inputs
+class OracleSample:
+    """The oracle (as it stands) on token samples of the workload: step(n, first) runs its
+    full forward on tokens [first, first + n) (wrapping around N) and returns the seconds it
+    took. Without capacity the tokens are independent, so a sample costs per token what the
+    whole batch costs; with capacity the sample is its own batch of n tokens (capacity
+    recomputed for n)."""
 
-    inp = inputs.make_inputs(cfg, "cpu", weights=not w8)
-    od = oracle.BF16 if cfg.dtype == configs.DTYPE_BF16 else oracle.F32
-    X = oracle.torch_to_numpy(inp.X)
-    Wr = inp.W_r.numpy()
-    b = None if inp.bias is None else inp.bias.numpy()
-    opts = dict(k=cfg.k, cf=cfg.capacity_factor, renorm=cfg.renormalize, act=cfg.activation,
-                dtype=od, min_capacity=cfg.min_capacity, order=cfg.capacity_order,
-                drop_policy=cfg.drop_policy)
-    if w8:
-        q = inputs.make_w8_weights(cfg, "cpu")
-        qs = [t.numpy() for t in (q.W1q, q.S1, q.W2q, q.S2, q.W3q, q.S3)]
-    else:
-        W1, W2, W3 = (oracle.torch_to_numpy(w) for w in (inp.W1, inp.W2, inp.W3))
-
-    def run(n):
-        t = time.perf_counter()
+    def __init__(self, cfg, w8: bool = False, inp=None, wq=None):
+        """inp / wq: the GPU arm's own input tensors (copied to the host here), else the
+        same recipe drawn on the host."""
+        import oracle
+        from top_routing_expert_fp32_b200 import configs, inputs
+        self.cfg, self.w8, self.oracle = cfg, w8, oracle
+        self.same_values = inp is not None
+        if inp is None:
+            inp = inputs.make_inputs(cfg, "cpu", weights=not w8)
+        if w8 and wq is None:
+            wq = inputs.make_w8_weights(cfg, "cpu")
+        self.od = oracle.BF16 if cfg.dtype == configs.DTYPE_BF16 else oracle.F32
+        self.X = oracle.torch_to_numpy(inp.X.cpu())
+        self.Wr = inp.W_r.cpu().numpy()
+        self.b = None if inp.bias is None else inp.bias.cpu().numpy()
+        self.opts = dict(k=cfg.k, cf=cfg.capacity_factor, renorm=cfg.renormalize,
+                         act=cfg.activation, dtype=self.od, min_capacity=cfg.min_capacity,
+                         order=cfg.capacity_order, drop_policy=cfg.drop_policy)
         if w8:
-            oracle.forward_w8(X[:n], Wr, b, *qs, **opts)
+            self.qs = [t.cpu().numpy() for t in (wq.W1q, wq.S1, wq.W2q, wq.S2, wq.W3q, wq.S3)]
         else:
-            oracle.forward(X[:n], Wr, b, W1, W2, W3, **opts)
+            self.W = [oracle.torch_to_numpy(w.cpu()) for w in (inp.W1, inp.W2, inp.W3)]
+        self.cores = oracle.num_threads()
+
+    def routing_check(self, gpu_idx) -> dict:
+        """Tokens whose GPU top-k (set or order) differs from the oracle's routing of its fp64
+        logits, and the largest top-k margin among them (near ties are below 1e-4)."""
+        o = self.oracle
+        l64, l32 = o.router_logits(self.X, self.od, self.Wr, self.b)
+        ro = o.route(l32, k=self.cfg.k, renorm=self.cfg.renormalize)
+        flips = (gpu_idx != ro["idx"]).any(1)
+        margin = o.topk_margin(l64, self.cfg.k)
+        return {"tokens": int(self.cfg.N), "flips": int(flips.sum()),
+                "max_margin_of_flips": float(margin[flips].max()) if flips.any() else None,
+                "near_tie_margin": 1e-4}
+
+    def step(self, n: int, first: int = 0) -> float:
+        import numpy as np
+        N = self.cfg.N
+        n = max(1, min(n, N))
+        rows = (np.arange(first, first + n) % N) if first + n > N else slice(first, first + n)
+        X = np.ascontiguousarray(self.X[rows])
+        t = time.perf_counter()
+        if self.w8:
+            self.oracle.forward_w8(X, self.Wr, self.b, *self.qs, **self.opts)
+        else:
+            self.oracle.forward(X, self.Wr, self.b, *self.W, **self.opts)
         return time.perf_counter() - t
 
-    n = min(cfg.N, max(1, oracle.num_threads()))
-    dt = run(n)
-    while dt < budget_s / 8 and n < cfg.N:
-        n = min(cfg.N, n * 2)
-        dt = run(n)
-    if dt < budget_s / 2 and n < cfg.N:
-        n = min(cfg.N, max(n + 1, int(n * (budget_s / 2) / max(dt, 1e-3))))
-        dt = run(n)
-    return dict(value=n / dt, unit="tokens/s", cores=oracle.num_threads(), kind="oracle",
-                sample=f"first {n} of {cfg.N} tokens of the workload, full forward in fp64, "
-                       f"{dt:.1f} s wall")
+    def calibrate(self, seconds: float) -> int:
+        """Tokens per sample so that one step takes about `seconds` (at least one token per
+        host thread's worth of records)."""
+        n = max(1, -(-self.cores // self.cfg.k))
+        dt = self.step(n)
+        while dt < seconds / 4 and n < self.cfg.N:
+            n = min(self.cfg.N, n * 2)
+            dt = self.step(n)
+        return max(1, min(self.cfg.N, int(n * seconds / max(dt, 1e-4))))
+
+
+def oracle_tokens_per_s(cfg, budget_s: float = 12.0, w8: bool = False, sampler=None):
+    """cpu_baseline of the GPU arm: the oracle on one bounded token sample of the workload
+    (about budget_s of CPU work), extrapolated to tokens/s."""
+    o = sampler or OracleSample(cfg, w8)
+    n = o.calibrate(budget_s / 2)
+    dt = o.step(n)
+    vals = "the GPU arm's input values" if o.same_values else "inputs of the same recipe"
+    return dict(value=n / dt, unit="tokens/s", cores=o.cores, kind="oracle",
+                sample=f"first {n} of {cfg.N} tokens of the workload ({vals}), full forward "
+                       f"in fp64, {dt:.1f} s wall; tokens/s extrapolated from the sample",
+                extrapolated=n < cfg.N)
+
+
+def run_reference(args, cfg, w8: bool, packed: bool) -> dict:
+    """The reference arm: the oracle as it stands, W warm-up steps and then exactly K timed
+    steps, each its full forward on a bounded sample of the workload's tokens (consecutive
+    slices, wrapping around N). The whole run is sized to end within a few minutes."""
+    o = OracleSample(cfg, w8)
+    per_step = min(6.0, 150.0 / max(1, args.steps + args.warmup))
+    n = o.calibrate(per_step)
+    first = 0
+    for _ in range(args.warmup):
+        o.step(n, first)
+        first = (first + n) % cfg.N
+    total = 0.0
+    for _ in range(args.steps):
+        total += o.step(n, first)
+        first = (first + n) % cfg.N
+    value = args.steps * n / total
+    sample = (f"{n} of {cfg.N} tokens per step (consecutive slices), full forward in fp64, "
+              f"{total:.1f} s wall over {args.steps} steps; tokens/s extrapolated to the "
+              f"workload")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * cfg.N / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic, seeded: the GPU arm's recipe and shapes, drawn on the host",
+            "config": {"workload": workload_desc(cfg, w8, packed),
+                       "sample_tokens_per_step": n},
+            "extrapolated": n < cfg.N,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": o.cores,
+                             "kind": "oracle", "sample": sample, "extrapolated": n < cfg.N},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -320,12 +399,19 @@ def run_gpu(args, cfg, world, rank, device):
     def new_events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
 
+    warm = []
     for _ in range(args.warmup):
-        step(new_events())
+        ev = new_events()
+        step(ev)
+        warm.append(ev)
         flush_l2()
     torch.cuda.synchronize(device)
     if abi.device_error(ws) != 0:
         raise RuntimeError("device error during warm-up")
+    if args.steps is None:  # enough steps for a timed region of about TIMED_REGION_TARGET_S
+        t_step = min(ev[0].elapsed_time(ev[5]) for ev in warm[-2:]) / 1e3
+        want = max(20, min(20000, math.ceil(TIMED_REGION_TARGET_S / max(t_step, 1e-6))))
+        args.steps = int(reduce_max(float(want), device))
 
     sampler = ClockSampler(device.index).start()
     barrier(device)
@@ -370,9 +456,10 @@ def run_gpu(args, cfg, world, rank, device):
     }
     for n in ("route", "combine"):
         kern[n]["frac_hbm"] = kern[n]["GB/s"] / hbm
-        kern[n]["frac_8TBs"] = kern[n]["GB/s"] / 8000.0
+        kern[n]["frac_8TBs"] = kern[n]["GB/s"] / DATASHEET_HBM_GBS
     for n in ("up", "down"):
         kern[n]["frac_bf16_peak"] = kern[n]["TFLOP/s"] / tc
+        kern[n]["frac_bf16_datasheet"] = kern[n]["TFLOP/s"] / DATASHEET_BF16_TFLOPS
     ffn_ms = mean["up"] + mean["down"]
     gemm_tflops = 6.0 * kept * D * F / ffn_ms / 1e9
 
@@ -399,6 +486,12 @@ def run_gpu(args, cfg, world, rank, device):
                 "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                 "frac": gbs / hbm, "peak_source": psrc, "bytes_per_launch": bytes_up}
     roof["min_us"] = {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6}
+    roof["denominator"] = ("peak = the measured " + ("cuBLAS bf16 GEMM burst" if
+                           roof["bound"] == "tensor" else "HBM copy bandwidth") +
+                           "; frac_datasheet uses the B200 datasheet figure")
+    roof["peak_datasheet"] = (DATASHEET_BF16_TFLOPS if roof["bound"] == "tensor"
+                              else DATASHEET_HBM_GBS)
+    roof["frac_datasheet"] = roof["achieved"] / roof["peak_datasheet"]
     roof["experts_used"] = used
     # Same two-sided bound for both GEMMs: frac_roofline = bound time / measured time.
     bytes_down = kept * F * es + used * (D * F * ew + (D * 4 if w8 else 0)) + kept * D * es
@@ -513,6 +606,16 @@ def run_gpu(args, cfg, world, rank, device):
         "gpu_launches": sum(launches.values()) * args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
+    line["clocks"]["timed_region_s"] = t_wall1 - t_wall0
+    mhz = line["clocks"].get("sm_mhz")
+    if roof["bound"] == "tensor" and mhz:
+        # Tensor throughput scales with the SM clock: the achieved rate against the datasheet
+        # peak scaled to the median clock of the timed region.
+        roof["frac_datasheet_at_run_clock"] = roof["achieved"] / (
+            DATASHEET_BF16_TFLOPS * float(mhz) / DATASHEET_SM_MHZ)
+    # For the oracle leg (not printed): the routing of the benched inputs, and the inputs.
+    line["_gpu_idx"] = idx.cpu().numpy()
+    line["_inp"], line["_wq"] = inp, wq
     return line
 
 
@@ -641,10 +744,57 @@ def run_gpu_ep(args, cfg, world, rank, device):
 
 # ------------------------------------------------------------------ main
 
+ALL_WORKLOADS = ["tiny_f32", "mixtral", "grok1", "capacity", "capacity_k1", "capacity_gshard",
+                 "decode"]
+
+
+def oracle_leg(line, cfg, w8: bool, budget_s: float = 12.0):
+    """Rank 0 at N=1 only, after the GPU work: the oracle timed on a sample of the GPU arm's own
+    inputs (cpu_baseline), and the GPU routing compared with the oracle's (near-tie flips)."""
+    o = OracleSample(cfg, w8, inp=line["_inp"], wq=line["_wq"])
+    line["cpu_baseline"] = oracle_tokens_per_s(cfg, budget_s=budget_s, w8=w8, sampler=o)
+    line["config"]["routing_vs_oracle"] = o.routing_check(line["_gpu_idx"])
+
+
+def strip_private(line):
+    for key in [k for k in line if k.startswith("_")]:
+        del line[key]
+    return line
+
+
+def table_row(line) -> str:
+    c = line["config"]
+    k = c["kernels"]
+    d = c.get("diagnostics", {})
+    rv = c.get("routing_vs_oracle", {})
+    cb = line.get("cpu_baseline") or {}
+    clk = line.get("clocks", {})
+    r = line["roofline"]
+    return ("| {w} | {v:.4g} | {ms:.3f} | {up:.0f} ({upf:.2f}) | {dn:.0f} ({dnf:.2f}) | "
+            "{rt:.1f} ({rtf:.2f}) | {cb:.1f} ({cbf:.2f}) | {roof:.2f} {bound} | {e2e:.4g} | "
+            "{bl:.4f} | {dr:.4f} | {lm:.3f} | {fl} | {cpu} | {mhz} / {rs} |").format(
+        w=c["workload"].split(":")[0], v=line["value"], ms=line["ms_per_step"],
+        up=k["up"]["TFLOP/s"], upf=k["up"]["frac_roofline"], dn=k["down"]["TFLOP/s"],
+        dnf=k["down"]["frac_roofline"], rt=k["route"]["ms"] * 1e3,
+        rtf=k["route"]["frac_hbm"], cb=k["combine"]["ms"] * 1e3, cbf=k["combine"]["frac_hbm"],
+        roof=r["frac"], bound=r["bound"], e2e=line["e2e"]["value"],
+        bl=d.get("balance_loss", float("nan")), dr=d.get("drop_rate", float("nan")),
+        lm=d.get("load_max_over_mean", float("nan")), fl=rv.get("flips", "-"),
+        cpu=f"{cb['value']:.3g} ({cb.get('cores')} thr)" if cb else "-",
+        mhz=clk.get("sm_mhz"), rs=",".join(clk.get("reasons", [])) or "-")
+
+
+TABLE_HEAD = ("| workload | tokens/s | ms/step | up TF/s (roof) | down TF/s (roof) | route us "
+              "(frac HBM) | combine us (frac HBM) | roofline frac | e2e tokens/s | balance loss "
+              "| drop rate | load max/mean | near-tie flips | CPU oracle tokens/s | SM MHz / "
+              "reasons |\n|" + "---|" * 15)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for a timed region of about 1.5 s)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=None)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
@@ -658,6 +808,11 @@ def main():
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
                     help="replicas: one independent layer per GPU; ep: experts split over the "
                          "GPUs, rows exchanged by all-to-all (bf16 weights)")
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="one line per workload (1 GPU), each with diagnostics, near-tie flips "
+                         "against the oracle's routing and the oracle's CPU throughput")
+    ap.add_argument("--table", default=None,
+                    help="with --all-workloads: also write a markdown table to this path")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -668,30 +823,46 @@ def main():
     if args.ffn is not None:
         cfg = cfg.with_(F=args.ffn, name=f"{cfg.name}_f{args.ffn}")
     world, rank, local = dist_env()
+    w8 = args.weights != "bf16"
 
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = oracle_tokens_per_s(cfg, budget_s=min(20.0, 6.0 * args.steps),
-                                 w8=args.weights != "bf16")
-        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": 1e3 * cfg.N / cb["value"], "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic, seeded (same inputs as the GPU arm)",
-                "config": {"workload": workload_desc(cfg, args.weights != "bf16",
-                                                     args.weights == "w8p")},
-                "cpu_baseline": cb,
-                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
+        if args.steps is None:
+            args.steps = 20
+        line = run_reference(args, cfg, w8, args.weights == "w8p")
+        line["n_gpus"] = world
         print(json.dumps(line))
         return 0
 
     import torch
     import torch.distributed as dist
     from datetime import timedelta
+
+    if args.all_workloads:
+        if world != 1:
+            raise SystemExit("--all-workloads runs on one GPU")
+        device = torch.device("cuda", local)
+        rows = []
+        steps = args.steps
+        for name in ALL_WORKLOADS:
+            c = configs.CONFIGS[name]
+            args.steps = steps if steps is not None else 10
+            line = run_gpu(args, c, 1, 0, device)
+            if not args.no_cpu_baseline:
+                oracle_leg(line, c, w8, budget_s=8.0)
+            strip_private(line)
+            print(json.dumps(line), flush=True)
+            rows.append(table_row(line))
+            del line
+            torch.cuda.empty_cache()
+        if args.table:
+            with open(args.table, "w") as f:
+                f.write(TABLE_HEAD + "\n" + "\n".join(rows) + "\n")
+        return 0
+
     ep_mode = args.parallel == "ep"
-    if ep_mode and args.weights != "bf16":
+    if ep_mode and w8:
         raise SystemExit("--parallel ep runs bf16 expert weights")
     launched = "MASTER_ADDR" in os.environ  # under torchrun: its env:// rendezvous and store
     if world > 1 or (ep_mode and launched):
@@ -707,13 +878,17 @@ def main():
                                 world_size=1, timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
+    if ep_mode and args.steps is None:
+        args.steps = 20
     line = (run_gpu_ep if ep_mode else run_gpu)(args, cfg, world, rank, device)
     if rank == 0:
-        if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = oracle_tokens_per_s(cfg, w8=args.weights != "bf16")
+        if not args.no_cpu_baseline and world == 1 and not ep_mode:
+            oracle_leg(line, cfg, w8)
         else:
             line["cpu_baseline"] = None
-        print(json.dumps(line))
+        print(json.dumps(strip_private(line)))
+    else:
+        strip_private(line)
     if dist.is_initialized():
         dist.destroy_process_group()
     return 0

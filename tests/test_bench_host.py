@@ -55,3 +55,38 @@ def test_workload_description_states_the_policies():
     assert "8-bit expert weights" in s and "K-contiguous" in s
     assert "renormalised" in bench.workload_desc(configs.CONFIGS["mixtral"])
     assert "no-renorm" in bench.workload_desc(configs.CONFIGS["grok1"])
+
+
+def test_reference_arm_runs_exactly_k_sampled_steps(oracle_lib):
+    # --impl reference: the oracle on the host, W warm-up and exactly K timed steps, each on a
+    # token sample; the line states the sample and whether the rate is extrapolated.
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl",
+                        "reference", "--workload", "tiny_f32", "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 3
+    assert line["value"] > 0 and line["unit"] == "tokens/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    n = line["config"]["sample_tokens_per_step"]
+    assert 1 <= n <= 64 and line["extrapolated"] == (n < 64)
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["ms_per_step"] == pytest.approx(1e3 * 64 / line["value"])
+
+
+def test_table_row_formats_a_line():
+    line = {"value": 1.0e6, "ms_per_step": 2.0, "e2e": {"value": 9.0e5},
+            "roofline": {"frac": 0.8, "bound": "tensor"},
+            "clocks": {"sm_mhz": 1965, "reasons": []},
+            "cpu_baseline": {"value": 40.0, "cores": 16},
+            "config": {"workload": "mixtral: N=4096", "diagnostics": {
+                "balance_loss": 1.0, "drop_rate": 0.0, "load_max_over_mean": 1.02},
+                "routing_vs_oracle": {"flips": 0},
+                "kernels": {"up": {"TFLOP/s": 1300, "frac_roofline": 0.8},
+                            "down": {"TFLOP/s": 1300, "frac_roofline": 0.8},
+                            "route": {"ms": 0.01, "frac_hbm": 0.5},
+                            "combine": {"ms": 0.02, "frac_hbm": 0.7}}}}
+    row = bench.table_row(line)
+    assert row.startswith("| mixtral |") and row.count("|") == bench.TABLE_HEAD.split("\n")[0].count("|")

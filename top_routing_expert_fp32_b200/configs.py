@@ -94,7 +94,7 @@ CONFIGS = {
 }
 
 # The workload the throughput benchmark times on one GPU.
-BENCH_WORKLOAD = "mixtral"
+BENCH_WORKLOAD = "grok1"
 
 
 def active_ffn_flops(N_kept_records: int, D: int, F: int) -> float:
