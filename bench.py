@@ -368,10 +368,9 @@ def run_gpu(args, cfg, world, rank, device):
     stream = torch.cuda.current_stream(device)
 
     names = ["route", "dispatch", "up", "down", "combine"]
-    # Kernels per step: route = W_r split + tensor-core router (bf16 X) or one SIMT router
-    # (fp32 X); dispatch = count + assign + gather; one launch each for up, down, combine.
-    launches = {"route": 2 if cfg.dtype == configs.DTYPE_BF16 else 1, "dispatch": 3, "up": 1,
-                "down": 1, "combine": 1}
+    # Kernels per step: one router (tensor-core for bf16 X, SIMT for fp32 X), one cooperative
+    # dispatch (count, slot assignment and gather), one launch each for up, down, combine.
+    launches = {"route": 1, "dispatch": 1, "up": 1, "down": 1, "combine": 1}
 
     def step(ev):
         ev[0].record(stream)
@@ -718,7 +717,7 @@ def run_gpu_ep(args, cfg, world, rank, device):
         et += e0v.elapsed_time(e1v)
     e_max = reduce_max(et, device)
     barrier(device)
-    launches = (2 if cfg.dtype == configs.DTYPE_BF16 else 1) + 3 + 2 + 2 + 1
+    launches = 1 + 1 + 2 + 2 + 1  # route, dispatch, 2 reorders, up + down, combine
     return {
         "metric": METRIC, "value": agg["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": agg["ms_per_step"],

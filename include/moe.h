@@ -41,7 +41,8 @@
  *     MOE_ERR_CUDA (work enqueued before it by the same call stays enqueued).
  *     moe_last_error() gives a message for the calling thread.
  *   - Workspace: a device buffer of moe_workspace_size() bytes, 256-byte aligned, owned by
- *     the caller. Its first 256 bytes hold the device error word: zero them once with
+ *     the caller. Its first 256 bytes hold the device error word and the expert GEMMs'
+ *     tile counters (which every GEMM launch returns to zero): zero them once with
  *     moe_workspace_init() before the first use. Calls that share a workspace must be
  *     ordered on one stream (they reuse its scratch regions).
  *   - Determinism: identical inputs give bitwise identical outputs; no floating-point

@@ -37,14 +37,18 @@ def test_traffic_used_only_while_the_kernel_sources_are_unchanged(tmp_path, monk
     assert bench.traffic_from_profile("up", "mixtral") is None
 
 
-def test_committed_traffic_matches_the_current_sources():
-    # Every committed capture names the sources it was taken on; the ones the benchmark reads
-    # for its default line must hash to the current files.
+def test_committed_traffic_is_used_exactly_when_its_sources_are_current():
+    # Every committed capture names the sources it was taken on; the benchmark reports a
+    # capture's bytes only while those sources hash as they did when it was taken, and null
+    # otherwise (the kernel has changed since the counters were read).
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         d = json.load(f)
-    e = d["up"]["mixtral"]
-    assert e["source_sha"] == bench.source_hash(e["sources"])
-    assert bench.traffic_from_profile("up", "mixtral") == e["bytes_per_launch"]
+    assert d
+    for kernel, per in d.items():
+        for workload, e in per.items():
+            current = e["source_sha"] == bench.source_hash(e["sources"])
+            got = bench.traffic_from_profile(kernel, workload)
+            assert got == (e["bytes_per_launch"] if current else None), (kernel, workload)
 
 
 def test_workload_description_states_the_policies():

@@ -134,3 +134,64 @@ def test_ep_forward_one_rank_full_size_mixtral(abi, nccl_group):
     assert normwise_rel_err(to_f64(out), to_f64(ref)).max() <= 1e-2
     del inp, comp, out, ref, ws
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg,world", [
+    (_cfg(300, 256, 512, 8, 2), 2),
+    (_cfg(400, 128, 384, 5, 2, capacity_factor=1.0, router_bias_var=2.0), 2),   # 3 + 2 experts
+    (_cfg(257, 384, 640, 8, 1), 3),                                             # 3 + 3 + 2
+], ids=["e8k2_world2", "capacity_e5_world2", "k1_world3"])
+def test_ep_ranks_with_expert_subsets_on_one_gpu(abi, cfg, world):
+    # The compute of every rank of an expert-parallel layer, run here on one GPU: each rank
+    # routes and dispatches its own tokens over all E experts, runs the grouped FFN of its own
+    # expert block on the rows it receives (sliced weights, rows in the planned expert-major
+    # order), reorders the outputs back and combines what comes back to it. The exchanges
+    # themselves are replayed by indexing (the NCCL path is ep.forward; the multi-rank
+    # bookkeeping is tested on gloo). Every rank's output must equal the oracle's experts on
+    # its own routing.
+    ranges = ep.expert_ranges(cfg.E, world)
+    full = inputs.make_inputs(cfg, "cuda")
+    Xs = [full.X] + [inputs.randn((cfg.N, cfg.D), 1.0, full.X.dtype, "cuda", cfg.seed + 1 + r,
+                                  inputs.TID_X) for r in range(1, world)]
+    comps = [ep.CudaCompute(cfg, full.W_r, full.bias,
+                            *(w[e0:e1].contiguous() for w in (full.W1, full.W2, full.W3)))
+             for (e0, e1) in ranges]
+    routed = [comps[s].route_dispatch(Xs[s]) for s in range(world)]
+    offs = [r["offsets"].cpu().numpy().astype(np.int64) for r in routed]
+    back = [[None] * world for _ in range(world)]   # back[source][owner]
+    for r, (e0, e1) in enumerate(ranges):
+        recv_counts = np.array([[offs[s][e + 1] - offs[s][e] for e in range(e0, e1)]
+                                for s in range(world)], dtype=np.int64)
+        plan = ep.plan_exchange(offs[r], recv_counts, ranges)
+        assert plan.send_rows == [int(offs[r][b] - offs[r][a]) for a, b in ranges]
+        X_recv = torch.cat([routed[s]["X_perm"][offs[s][e0]:offs[s][e1]] for s in range(world)])
+        assert X_recv.shape[0] == sum(plan.recv_rows)
+        X_loc = comps[r].gather_rows(X_recv, plan.to_expert_major)
+        Y_loc = comps[r].expert_ffn(X_loc, plan.local_offsets, (e0, e1))
+        Y_recv = comps[r].gather_rows(Y_loc, plan.to_source_major)
+        base = np.concatenate([[0], np.cumsum(plan.recv_rows)])
+        for s in range(world):
+            back[s][r] = Y_recv[base[s]:base[s + 1]]
+    for s in range(world):
+        Y_back = torch.cat(back[s])       # owners in expert order = the source's X_perm order
+        out = comps[s].combine(Y_back, routed[s])
+        torch.cuda.synchronize()
+        assert comps[s].device_error() == 0
+        idx = routed[s]["idx"].cpu().numpy()
+        gate = routed[s]["gate"].cpu().numpy().astype(np.float64)
+        dropped = routed[s]["dropped"].cpu().numpy()
+        C = oracle.capacity(cfg.N, cfg.k, cfg.E, cfg.capacity_factor)
+        do = oracle.dispatch(idx, cfg.E, C)
+        assert np.array_equal(do["offsets"], offs[s]) and np.array_equal(do["dropped"], dropped)
+        kept = np.argwhere(dropped == 0)
+        Xn = np_host(Xs[s])
+        Y = oracle.expert_ffn(kept[:, 0].astype(np.int32), idx[dropped == 0].astype(np.int32),
+                              Xn, np_host(full.W1), np_host(full.W2), np_host(full.W3),
+                              oracle.BF16, cfg.activation)
+        ref = np.zeros((cfg.N, cfg.D))
+        for (t, j), y in zip(kept, Y):
+            ref[t] += gate[t, j] * y
+        err = normwise_rel_err(to_f64(out), ref)
+        assert err.max() <= TOL_BF16, f"rank {s}: max normwise rel err {err.max():.3g}"
+    del comps, routed, full
+    torch.cuda.empty_cache()

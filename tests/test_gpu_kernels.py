@@ -197,6 +197,10 @@ def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, 
     nk = int(ref["offsets"][E])
     assert np.array_equal(d["row_token"].cpu().numpy()[:nk], ref["row_token"])
     assert abi.device_error(ws) == 0
+    # the one-launch dispatch's grid-barrier counters (workspace header ints 20, 21) are back
+    # at zero for the next call
+    hdr = ws[:256].view(torch.int32).cpu()
+    assert hdr[20].item() == 0 and hdr[21].item() == 0
     return d, ref, X_perm
 
 
@@ -207,6 +211,13 @@ def _dispatch_case(abi, oracle_lib, N, E, k, cf, seed, skew=0.0, all_one=False, 
     (1025, 2, 1, 0.5, 0)])
 def test_dispatch_bitexact(abi, oracle_lib, N, E, k, cf, skew):
     _dispatch_case(abi, oracle_lib, N, E, k, cf, seed=N + E + k, skew=skew)
+
+
+def test_dispatch_more_chunks_than_resident_blocks(abi, oracle_lib):
+    # 700,000 records = 684 chunks of 1024: more than the blocks that fit on the device at once,
+    # so the one-launch dispatch's blocks loop over chunks; twice in a row on one workspace.
+    for cf in (1.25, 0.0):
+        _dispatch_case(abi, oracle_lib, 350000, 8, 2, cf, seed=77, skew=0.2)
 
 
 @pytest.mark.parametrize("N,E,k,cf,skew,minc", [
@@ -336,6 +347,53 @@ def test_expert_ffn_tile_groups(abi, oracle_lib, monkeypatch, counts, D, F, tile
     monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
     monkeypatch.setenv("MOE_GEMM_NGROUP", ngroup)
     _ffn_case(abi, oracle_lib, counts, D, F, configs.ACT_SILU, seed=3)
+
+
+@pytest.mark.parametrize("counts,D,F", [
+    ([5], 64, 128),                                   # 1 tile: surplus CTAs take none
+    ([129, 127, 128, 0, 5, 256, 1, 64], 256, 384),
+    ([2000, 1500, 0, 2600], 256, 2048),               # many tiles per CTA
+])
+@pytest.mark.parametrize("tile_rows", ["128", "256"])
+@pytest.mark.parametrize("order", ["dynamic", "static"])
+def test_expert_ffn_tile_counter_returns_to_zero(abi, oracle_lib, monkeypatch, counts, D, F,
+                                                 tile_rows, order):
+    # Tiles are handed out in order by a counter in the workspace header (ints 16 and 17);
+    # every launch returns it to zero, so back-to-back launches on one workspace give the same
+    # bits and see every tile. The static round-robin order (MOE_GEMM_SCHED=static) gives the
+    # same results.
+    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
+    monkeypatch.setenv("MOE_GEMM_SCHED", order)
+    E = len(counts)
+    R = int(sum(counts))
+    cfg = _cfg(R, D, F, E, 1)
+    Xp = inputs.randn((R, D), 1.0, torch.bfloat16, "cuda", 7, 1)
+    W1 = inputs.randn((E, D, F), 1 / math.sqrt(D), torch.bfloat16, "cuda", 7, 3)
+    W2 = inputs.randn((E, D, F), 1 / math.sqrt(D), torch.bfloat16, "cuda", 7, 4)
+    W3 = inputs.randn((E, F, D), 1 / math.sqrt(F), torch.bfloat16, "cuda", 7, 5)
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32,
+                           device="cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    outs = []
+    for _ in range(3):
+        H = torch.full((R, F), float("nan"), dtype=torch.bfloat16, device="cuda")
+        Y = torch.full((R, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        abi.expert_ffn(p, Xp, offsets, W1, W2, W3, H, Y, ws)
+        torch.cuda.synchronize()
+        hdr = ws[:256].view(torch.int32).cpu()
+        assert hdr[16].item() == 0 and hdr[17].item() == 0
+        outs.append((H, Y))
+    assert abi.device_error(ws) == 0
+    for H, Y in outs[1:]:
+        assert torch.equal(H.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(Y.view(torch.int16), outs[0][1].view(torch.int16))
+    sel = np.unique(np.concatenate([np.arange(0, R, max(1, R // 50)), [R - 1]]))
+    rec_e = np.repeat(np.arange(E, dtype=np.int32), counts)[sel]
+    ref = oracle_lib.expert_ffn(sel.astype(np.int32), rec_e, np_host(Xp), np_host(W1),
+                                np_host(W2), np_host(W3), oracle.BF16, configs.ACT_SILU)
+    err = normwise_rel_err(to_f64(outs[0][1][sel]), ref)
+    assert err.max() <= TOL_BF16, f"max normwise rel err {err.max():.3g}"
 
 
 def test_expert_ffn_f32(abi, oracle_lib):

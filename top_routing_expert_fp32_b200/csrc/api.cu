@@ -59,11 +59,20 @@ uint64_t wait_timeout_ns() {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The workspace header (its first 256 bytes, zeroed by moe_workspace_init): int 0 is the
+// device error word, ints 16 and 17 the grouped GEMMs' tile counter and finished count (zero
+// at rest; each GEMM launch returns them to zero when it ends).
+constexpr int kSchedInt = 16;
+int* sched_of(int* header) { return header + kSchedInt; }
+// Ints 20 and 21: the fused dispatch's grid-barrier arrivals and finished count (zero at rest).
+constexpr int kDispatchBarInt = 20;
+int* dispatch_bar_of(int* header) { return header + kDispatchBarInt; }
+
 size_t elem_size(const moe_problem& p) { return p.dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 
 // Device workspace regions (byte offsets from the workspace base).
 struct Layout {
-  size_t err, colsum_part, zl_part, wt, counts, idx, gate, pos, dropped, load, offsets, row_token,
+  size_t err, colsum_part, zl_part, counts, idx, gate, pos, dropped, load, offsets, row_token,
       xperm, h, y;
   size_t total;       // moe_forward and every other entry point
   size_t xin, xout;   // moe_forward_host / moe_forward_host_many
@@ -84,7 +93,6 @@ Layout make_layout(const moe_problem& p) {
   L.err = take(256);
   L.colsum_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)) * p.E);
   L.zl_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)));
-  L.wt = take(route_tc_wt_bytes(p));
   L.counts = take(sizeof(int32_t) * static_cast<size_t>(dispatch_num_chunks(R)) * p.E);
   L.idx = take(sizeof(int32_t) * R);
   L.gate = take(sizeof(float) * R);
@@ -204,7 +212,8 @@ moe_status run_up(const moe_problem& p, const void* X_perm, const int32_t* offse
   NvtxRange range("moe expert up");
   if (p.dtype == MOE_DTYPE_BF16) {
     MOE_TRY(check_sm100());
-    MOE_CUDA(launch_ffn_up_sm100(p, X_perm, offsets, W1, W2, H, err, wait_timeout_ns(), stream),
+    MOE_CUDA(launch_ffn_up_sm100(p, X_perm, offsets, W1, W2, H, err, sched_of(err),
+                                 wait_timeout_ns(), stream),
              "expert up-projection (tcgen05)");
   } else {
     MOE_CUDA(launch_ffn_up_f32(p, X_perm, offsets, W1, W2, H, stream), "expert up-projection");
@@ -217,7 +226,8 @@ moe_status run_down(const moe_problem& p, const void* H, const int32_t* offsets,
   NvtxRange range("moe expert down");
   if (p.dtype == MOE_DTYPE_BF16) {
     MOE_TRY(check_sm100());
-    MOE_CUDA(launch_ffn_down_sm100(p, H, offsets, W3, Y, err, wait_timeout_ns(), stream),
+    MOE_CUDA(launch_ffn_down_sm100(p, H, offsets, W3, Y, err, sched_of(err), wait_timeout_ns(),
+                                   stream),
              "expert down-projection (tcgen05)");
   } else {
     MOE_CUDA(launch_ffn_down_f32(p, H, offsets, W3, Y, stream), "expert down-projection");
@@ -322,7 +332,7 @@ moe_status route_impl(const moe_problem& p, const void* X, const float* W_r, con
   }
   MOE_CUDA(launch_route(p, X, W_r, bias, noise, logits, topk_idx, topk_gate,
                         at<float>(ws, L.colsum_part), prob_colsum, at<float>(ws, L.zl_part), z_loss,
-                        at<__nv_bfloat16>(ws, L.wt), at<int>(ws, L.err), wait_timeout_ns(), s),
+                        at<int>(ws, L.err), wait_timeout_ns(), s),
            "route");
   return MOE_OK;
 }
@@ -355,10 +365,10 @@ moe_status forward_impl(const moe_problem& p, const void* X, const float* W_r, c
   MOE_TRY(route_impl(p, X, W_r, bias, noise, logits, idx, gate, prob_colsum, z_loss, ws, stream));
   {
     NvtxRange range("moe dispatch");
-    MOE_CUDA(launch_slot_assign(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off, ps,
-                                dr, row_token, err, stream),
-             "slot assign");
-    MOE_CUDA(launch_gather(p, X, row_token, off, xperm, err, stream), "gather");
+    MOE_CUDA(launch_dispatch_fused(p, capacity_of(p), idx, at<int32_t>(ws, L.counts), ld, off,
+                                   ps, dr, row_token, X, xperm, err, dispatch_bar_of(err),
+                                   wait_timeout_ns(), stream),
+             "dispatch");
   }
   MOE_TRY(run_ffn(p, xperm, off, w, h, y, err, stream));
   NvtxRange range("moe combine");
@@ -459,10 +469,11 @@ moe_status moe_dispatch(const moe_problem* p, const void* X, const int32_t* topk
   int* err = at<int>(ws, L.err);
   int32_t* rt = row_token ? row_token : at<int32_t>(ws, L.row_token);
   NvtxRange range("moe dispatch");
-  MOE_CUDA(launch_slot_assign(*p, capacity_of(*p), topk_idx, at<int32_t>(ws, L.counts), load,
-                              offsets, pos, dropped, rt, err, s),
-           "slot assign");
-  if (gather) MOE_CUDA(launch_gather(*p, X, rt, offsets, X_perm, err, s), "gather");
+  MOE_CUDA(launch_dispatch_fused(*p, capacity_of(*p), topk_idx, at<int32_t>(ws, L.counts), load,
+                                 offsets, pos, dropped, rt, gather ? X : nullptr,
+                                 gather ? X_perm : nullptr, err, dispatch_bar_of(err),
+                                 wait_timeout_ns(), s),
+           "dispatch");
   return MOE_OK;
 }
 

@@ -298,6 +298,214 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ------------------------------------------------------------------ fused dispatch
+//
+// Count, slot assignment and gather in one cooperative launch (every block resident at
+// once). Phase 1: blocks b < nchunks count chunk b per expert (as count_kernel). Grid
+// barrier. Phase 2: the same blocks assign their chunks' positions, drop flags and row map
+// (as assign_kernel; block 0 also writes load and offsets). Grid barrier. Phase 3: every
+// block copies rows X_perm[row] = X[row_token[row]] for row < offsets[E], one warp per row
+// at a time, 16-byte words with four loads in flight per lane. Data another block wrote in an
+// earlier phase is read at L2 (ld.global.cg). The barrier counters live in the workspace
+// header (zero at rest); the last block to finish returns them to zero, also after a barrier
+// timed out. Bit-exact with the three-kernel path.
+
+constexpr int kFusedThreads = 512;
+
+struct FusedArgs {
+  const int32_t* idx;
+  const uint8_t* X;        // nullptr: no gather (phase 3 and its barrier are skipped)
+  uint8_t* X_perm;
+  int32_t* counts;         // [nchunks][E]
+  int32_t* load;
+  int32_t* offsets;
+  int32_t* pos;
+  uint8_t* dropped;
+  int32_t* row_token;
+  int* err;
+  int* bar;                // [2]: barrier arrivals (one or two per block), blocks finished
+  int64_t N, R, C;
+  int k, E, nchunks;
+  bool token_major;
+  uint32_t row_words;      // 16-byte words per row
+  uint64_t timeout_ns;
+};
+
+// Arrive on the grid barrier and wait until `target` arrivals have been made (bounded).
+// Returns false to every thread of the block when the wait ran out.
+__device__ bool grid_barrier(int* bar, int target, uint64_t timeout_ns, int* err) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this block's writes before its arrival
+    atomicAdd(bar, 1);
+    int ok = 1;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (v >= target) break;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        ok = 0;
+        record_error(err, MOE_DEVERR_WAIT_TIMEOUT);
+        break;
+      }
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+__global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs a) {
+  __shared__ int hist[kMaxE];
+  __shared__ int s_base[kMaxE];
+  __shared__ int s_tot[kMaxE];
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_wpre[kFusedThreads / 32][kMaxE];
+  const int E = a.E;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int kWarps = kFusedThreads / 32;
+  const int G = static_cast<int>(gridDim.x);
+  bool ok = true;
+
+  // Phase 1: per-chunk histograms.
+  for (int c = blockIdx.x; c < a.nchunks; c += G) {
+    for (int e = threadIdx.x; e < E; e += kFusedThreads) hist[e] = 0;
+    __syncthreads();
+    const int64_t r0 = static_cast<int64_t>(c) * kDispatchChunk;
+    const int64_t r1 = std::min<int64_t>(r0 + kDispatchChunk, a.R);
+    for (int64_t r = r0 + threadIdx.x; r < r1; r += kFusedThreads) {
+      int64_t t, j;
+      record_at(r, a.N, a.k, a.token_major, t, j);
+      const int e = a.idx[t * a.k + j];
+      if (e < 0 || e >= E) record_error(a.err, MOE_DEVERR_BAD_INDEX);
+      else atomicAdd(&hist[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kFusedThreads)
+      a.counts[static_cast<int64_t>(c) * E + e] = hist[e];
+    __syncthreads();
+  }
+  ok = grid_barrier(a.bar, G, a.timeout_ns, a.err);
+
+  // Phase 2: positions in record order (stable counting-sort rank), drop flags, row map.
+  for (int c = blockIdx.x; ok && c < a.nchunks; c += G) {
+    if (threadIdx.x < E) {
+      const int e = threadIdx.x;
+      int base = 0, total = 0;
+      for (int cc = 0; cc < a.nchunks; ++cc) {
+        const int v = __ldcg(a.counts + static_cast<int64_t>(cc) * E + e);
+        if (cc < c) base += v;
+        total += v;
+      }
+      s_base[e] = base;
+      s_tot[e] = total;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int run = 0;
+      for (int e = 0; e < E; ++e) {
+        s_off[e] = run;
+        const int64_t tot = s_tot[e];
+        run += static_cast<int>(tot < a.C ? tot : a.C);
+      }
+      s_off[E] = run;
+      if (c == 0) {
+        for (int e = 0; e < E; ++e) {
+          a.load[e] = s_tot[e];
+          a.offsets[e] = s_off[e];
+        }
+        a.offsets[E] = run;
+      }
+    }
+    __syncthreads();
+    int running = 0;  // thread e < E: records of expert e in earlier tiles of this chunk
+    const int64_t r0 = static_cast<int64_t>(c) * kDispatchChunk;
+    const int64_t r1 = std::min<int64_t>(r0 + kDispatchChunk, a.R);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int64_t tile = r0; tile < r1; tile += kFusedThreads) {
+      for (int i = threadIdx.x; i < kWarps * kMaxE; i += kFusedThreads) (&s_wpre[0][0])[i] = 0;
+      __syncthreads();
+      const int64_t r = tile + threadIdx.x;
+      const bool valid = r < r1;
+      int64_t j = 0, t = 0;
+      int e = -1;
+      if (valid) {
+        record_at(r, a.N, a.k, a.token_major, t, j);
+        e = a.idx[t * a.k + j];
+        if (e < 0 || e >= E) e = -1;  // recorded in phase 1
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -2);
+      const int rank = __popc(peers & lt_mask);
+      if (valid && e >= 0 && rank == 0) s_wpre[warp][e] = __popc(peers);
+      __syncthreads();
+      if (threadIdx.x < E) {
+        const int ee = threadIdx.x;
+        int run = running;
+        for (int w = 0; w < kWarps; ++w) {
+          const int cnt = s_wpre[w][ee];
+          s_wpre[w][ee] = run;
+          run += cnt;
+        }
+        running = run;
+      }
+      __syncthreads();
+      if (valid) {
+        const int64_t rec = t * a.k + j;
+        if (e >= 0) {
+          const int p = s_base[e] + s_wpre[warp][e] + rank;
+          const bool drop = p >= a.C;
+          a.pos[rec] = p;
+          a.dropped[rec] = drop ? 1 : 0;
+          if (!drop) a.row_token[s_off[e] + p] = static_cast<int32_t>(t);
+        } else {
+          a.pos[rec] = -1;
+          a.dropped[rec] = 1;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // Phase 3: the permutation, one warp per row.
+  if (a.X != nullptr) {
+    ok = grid_barrier(a.bar, 2 * G, a.timeout_ns, a.err) && ok;
+    if (ok) {
+      const int64_t rows = __ldcg(a.offsets + E);
+      const int64_t W = static_cast<int64_t>(G) * kWarps;
+      const uint32_t words = a.row_words;
+      for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + warp; row < rows; row += W) {
+        const int64_t tok = __ldcg(a.row_token + row);
+        const uint4* src = reinterpret_cast<const uint4*>(a.X) + tok * words;
+        uint4* dst = reinterpret_cast<uint4*>(a.X_perm) + row * words;
+        uint32_t w = lane;
+        for (; w + 96 < words; w += 128) {
+          const uint4 v0 = __ldg(src + w), v1 = __ldg(src + w + 32), v2 = __ldg(src + w + 64),
+                      v3 = __ldg(src + w + 96);
+          dst[w] = v0;
+          dst[w + 32] = v1;
+          dst[w + 64] = v2;
+          dst[w + 96] = v3;
+        }
+        for (; w < words; w += 32) dst[w] = __ldg(src + w);
+      }
+    }
+  }
+
+  // Last block out returns the barrier counters to zero for the next launch.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&a.bar[1], 1) == G - 1) {
+      atomicExch(&a.bar[0], 0);
+      atomicExch(&a.bar[1], 0);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_gather_rows(const void* src, int64_t n_src, const int32_t* index,
@@ -356,6 +564,81 @@ cudaError_t launch_gather(const moe_problem& p, const void* X, const int32_t* ro
                                             p.E, row_bytes, piece, stages,
                                             static_cast<uint8_t*>(X_perm), err);
   return cudaGetLastError();
+}
+
+// Blocks of the fused dispatch that fit on the device at once (cached per device).
+int fused_max_blocks() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_fused_kernel,
+                                                      kFusedThreads, 0) != cudaSuccess ||
+        per_sm <= 0) {
+      (void)cudaGetLastError();
+      per_sm = -1;
+    }
+    cache[dev] = per_sm > 0 ? per_sm * num_sms() : -1;
+  }
+  return cache[dev] > 0 ? cache[dev] : 0;
+}
+
+cudaError_t launch_dispatch_fused(const moe_problem& p, int64_t capacity, const int32_t* idx,
+                                  int32_t* chunk_counts, int32_t* load, int32_t* offsets,
+                                  int32_t* pos, uint8_t* dropped, int32_t* row_token,
+                                  const void* X, void* X_perm, int* err, int* bar,
+                                  uint64_t timeout_ns, cudaStream_t stream) {
+  const int64_t R = p.N * p.k;
+  const int nchunks = dispatch_num_chunks(R);
+  const uint32_t elem = p.dtype == MOE_DTYPE_BF16 ? 2u : 4u;
+  const int max_blocks = fused_max_blocks();
+  if (R == 0 || max_blocks < 1 || (static_cast<int64_t>(p.D) * elem) % 16 != 0) {
+    // Nothing to fuse (or no resident grid): the three-kernel path.
+    cudaError_t e = launch_slot_assign(p, capacity, idx, chunk_counts, load, offsets, pos,
+                                       dropped, row_token, err, stream);
+    if (e != cudaSuccess || X == nullptr) return e;
+    return launch_gather(p, X, row_token, offsets, X_perm, err, stream);
+  }
+  FusedArgs a;
+  a.idx = idx;
+  a.X = static_cast<const uint8_t*>(X);
+  a.X_perm = static_cast<uint8_t*>(X_perm);
+  a.counts = chunk_counts;
+  a.load = load;
+  a.offsets = offsets;
+  a.pos = pos;
+  a.dropped = dropped;
+  a.row_token = row_token;
+  a.err = err;
+  a.bar = bar;
+  a.N = p.N;
+  a.R = R;
+  a.C = capacity;
+  a.k = p.k;
+  a.E = p.E;
+  a.nchunks = nchunks;
+  a.token_major = p.capacity_order == MOE_ORDER_TOKEN_MAJOR;
+  a.row_words = static_cast<uint32_t>(static_cast<int64_t>(p.D) * elem / 16);
+  a.timeout_ns = timeout_ns;
+  // Enough warps for the gather (one row each in flight), at least one block per chunk.
+  const int64_t want_rows = X != nullptr ? R : 0;
+  const int64_t want = std::max<int64_t>(
+      nchunks, (want_rows + kFusedThreads / 32 - 1) / (kFusedThreads / 32));
+  // More chunks than resident blocks: blocks loop over chunks (still one launch).
+  const int grid = static_cast<int>(std::min<int64_t>(want, max_blocks));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max(grid, 1)));
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, dispatch_fused_kernel, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -24,6 +24,14 @@
 // CTAs resident at any moment work on several experts at once, so experts with few rows
 // (bound by streaming their weights) run beside experts with many rows (bound by the MMAs).
 // Per-expert row counts are read from device memory: the host never learns them.
+// Scheduling: tiles are handed out in order by a global counter (one atomic per tile, taken
+// by the TMA producer of the CTA, or of the pair's first CTA, one tile ahead) and passed to
+// the MMA issuer and the epilogue (and to the second CTA of a pair) through a small ring of
+// tile ids in shared memory. The tiles in flight are therefore always a window of
+// consecutive tiles: the row blocks that share a weight column block run together, and a
+// weight block or an expert's rows are read from DRAM about once, however unevenly the tiles
+// progress. The counter and a count of finished CTAs live in the workspace header (zeroed by
+// moe_workspace_init); the last CTA to finish resets both to zero, also after an error.
 // Every barrier wait is bounded in time; on a timeout the CTA records
 // MOE_DEVERR_WAIT_TIMEOUT, unwinds, drains its MMAs and frees its TMEM.
 #include <algorithm>
@@ -49,6 +57,7 @@ constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr int kMaxE = 64;
+constexpr int kRing = 4;                           // tile ids in flight between the roles
 
 // Per-variant shape: a single CTA computes 128-row tiles with the whole B; a CTA pair
 // computes 256-row tiles, each CTA holding its 128 A rows and half of the B columns.
@@ -83,8 +92,26 @@ struct GemmParams {
   int l2_a;                // L2 eviction priority of the A rows (+1 last, 0 normal, -1 first)
   int l2_b;                // and of the expert weights
   int* err;
+  int* sched;              // [2]: next tile to hand out, CTAs (or pairs) finished; zero at rest
+  int static_order;        // 1: CTA (pair) u takes tiles u, u + units, ... (no counter)
   uint64_t timeout_ns;
 };
+
+// Stores a 32-bit value into the shared memory of a CTA of this cluster (address from
+// mapa_shared); ordered before a later release.cluster arrival of the same thread.
+__device__ __forceinline__ void st_dsmem_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Every CTA (the first CTA of every pair) calls this once, last: the one that finishes last
+// returns the tile counter and the finished count to zero for the next launch.
+__device__ __forceinline__ void sched_finish(int* sched, int ctas) {
+  __threadfence();
+  if (atomicAdd(&sched[1], 1) == ctas - 1) {
+    atomicExch(&sched[0], 0);
+    atomicExch(&sched[1], 0);
+  }
+}
 
 template <bool DUAL, int ACT, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -102,8 +129,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + S::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
-  int* s_mstart = reinterpret_cast<int*>(s_tmem + 1);  // [E+1] first row block of expert e
+  uint64_t* ring_full = drain + 1;            // [kRing] a tile id is in its slot
+  uint64_t* ring_empty = ring_full + kRing;   // [kRing] every consumer has read the slot
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(ring_empty + kRing);
+  volatile int* s_ring = reinterpret_cast<volatile int*>(s_tmem + 1);  // [kRing] tile ids
+  int* s_mstart = const_cast<int*>(s_ring) + kRing;    // [E+1] first row block of expert e
   int* s_seg = s_mstart + (kMaxE + 1);                 // [E+1]
 
   constexpr int NT = DUAL ? 128 : 256;  // output columns per tile
@@ -113,8 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_kb = (p.K + BK - 1) / BK;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the CTA that issues the MMAs
   const bool mma_cta = rank == 0;
-  const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int tile_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int cta_unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -131,8 +161,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_tiles = m_total * n_blocks;
   const int group = min(max(p.n_group, 1), n_blocks);
   const int group_tiles = m_total * group;
-  // Uniform over the block (and over the pair: both CTAs see the same tile list).
-  if (first_tile >= total_tiles) return;
+  // More CTAs (pairs) than tiles: the surplus ones take no tile; they only count themselves
+  // finished. Uniform over the block and over the pair.
+  if (cta_unit >= total_tiles) {
+    if (threadIdx.x == 0 && mma_cta) sched_finish(p.sched, units);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -142,6 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
+    }
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&ring_full[r], 1);
+      // consumers of a tile id: the MMA issuer and 4 epilogue warps, plus (pairs) the second
+      // CTA's producer and its 4 epilogue warps
+      mbar_init(&ring_empty[r], PAIR ? 10 : 5);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -180,6 +220,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     n_blk = c * group + n_in;
   };
 
+  // Next tile id from the ring (consumers). The second CTA of a pair receives the ids from
+  // the first CTA (remote store + release.cluster arrival), so it waits with cluster scope
+  // and returns its slot with a remote arrival.
+  int r_slot = 0;
+  uint32_t r_phase = 0;
+  auto ring_take = [&](int& t) -> bool {
+    const bool ok = (PAIR && !mma_cta)
+                        ? mbar_wait_cluster(&ring_full[r_slot], r_phase, p.timeout_ns)
+                        : mbar_wait(&ring_full[r_slot], r_phase, p.timeout_ns);
+    if (ok) t = s_ring[r_slot];
+    return ok;
+  };
+  auto ring_release = [&]() {
+    if (PAIR && !mma_cta) mbar_arrive_cluster(mapa_shared(smem_u32(&ring_empty[r_slot]), 0));
+    else mbar_arrive(&ring_empty[r_slot]);
+  };
+  auto ring_advance = [&]() {
+    if (++r_slot == kRing) {
+      r_slot = 0;
+      r_phase ^= 1u;
+    }
+  };
+
   if (warp == 0) {
     if (lane == 0) {  // ---------------------------------------------------- TMA producer
       int stage = 0;
@@ -187,7 +250,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint64_t pol_a = l2_policy(p.l2_a);
       const uint64_t pol_b = l2_policy(p.l2_b);
-      for (int tile = first_tile; ok && tile < total_tiles; tile += tile_stride) {
+      // The first CTA takes tile ids from the counter (one ahead) and publishes them; the
+      // second CTA of a pair takes them from the ring.
+      int next = !mma_cta ? 0 : (p.static_order ? cta_unit : atomicAdd(&p.sched[0], 1));
+      while (ok) {
+        int tile = next;
+        if (mma_cta) {
+          // Pairs: the second CTA returns slots with release.cluster arrivals; acquire at
+          // cluster scope before storing the next id into its shared memory.
+          const bool free_slot =
+              PAIR ? mbar_wait_cluster(&ring_empty[r_slot], r_phase ^ 1u, p.timeout_ns)
+                   : mbar_wait(&ring_empty[r_slot], r_phase ^ 1u, p.timeout_ns);
+          if (!free_slot) {
+            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+            break;
+          }
+          s_ring[r_slot] = tile;
+          if (PAIR) st_dsmem_u32(mapa_shared(smem_u32(const_cast<int*>(&s_ring[r_slot])), 1),
+                                 static_cast<uint32_t>(tile));
+          mbar_arrive(&ring_full[r_slot]);
+          if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&ring_full[r_slot]), 1));
+          ring_advance();
+          if (tile >= total_tiles) break;
+          // its latency overlaps this tile's loads
+          next = p.static_order ? tile + units : atomicAdd(&p.sched[0], 1);
+        } else {
+          if (!ring_take(tile)) {
+            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+            break;
+          }
+          ring_release();
+          ring_advance();
+          if (tile >= total_tiles) break;
+        }
         int e, m_blk, n_blk;
         decode(tile, e, m_blk, n_blk);
         const int row0 = s_seg[e] + m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
@@ -242,8 +337,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int tile = first_tile; ok && tile < total_tiles; tile += tile_stride, ++it) {
+      for (int it = 0; ok; ++it) {
+        int tile = 0;
+        if (!ring_take(tile)) {
+          record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+          break;
+        }
+        ring_release();
+        ring_advance();
+        if (tile >= total_tiles) break;
         const int acc = it & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
@@ -299,8 +401,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {  // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // this warp may access TMEM lanes [32q, 32q+32)
     const uint32_t tempty_mma0 = PAIR ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
-    int it = 0;
-    for (int tile = first_tile; tile < total_tiles; tile += tile_stride, ++it) {
+    for (int it = 0;; ++it) {
+      int tile = 0;
+      const bool got = ring_take(tile);
+      if (__any_sync(0xffffffffu, !got)) {
+        if (lane == 0) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) ring_release();
+      ring_advance();
+      if (tile >= total_tiles) break;
       const int acc = it & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, p.timeout_ns);
@@ -383,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
     else tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0 && mma_cta) sched_finish(p.sched, units);
 }
 
 // ------------------------------------------------------------------ host side
@@ -517,6 +629,13 @@ int column_group(bool pairs, int64_t n_blocks) {
   return static_cast<int>(pairs ? n_blocks : std::min<int64_t>(kGroup, n_blocks));
 }
 
+// Tile order: handed out in order by the workspace counter (default), or the static
+// round-robin CTA u -> tiles u, u + units, ... (MOE_GEMM_SCHED=static; tuning and comparison).
+int static_order() {
+  const char* env = std::getenv("MOE_GEMM_SCHED");
+  return env != nullptr && std::strcmp(env, "static") == 0 ? 1 : 0;
+}
+
 // L2 priorities of the GEMM operands: an expert's A rows are read again by every column block
 // of that expert, its weights by the few row blocks running at the same time. Default: A rows
 // evict_last, weights evict_normal. MOE_GEMM_L2=<a>,<b> (each -1, 0 or 1) overrides.
@@ -539,6 +658,7 @@ cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUten
   const int64_t R = p.N * p.k;
   const int64_t n_blocks = (gp.n_out + n_tile - 1) / n_tile;
   gp.n_group = column_group(use_pairs(p), n_blocks);
+  gp.static_order = static_order();
   l2_priorities(&gp.l2_a, &gp.l2_b);
   if (use_pairs(p)) {
     const int64_t tiles = ((R + 255) / 256 + p.E) * n_blocks;
@@ -590,7 +710,7 @@ bool make_tensor_map_3d_u8_sw64(CUtensorMap* m, const void* ptr, uint64_t inner,
 }
 
 cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
-                                const void* W1, const void* W2, void* H, int* err,
+                                const void* W1, const void* W2, void* H, int* err, int* sched,
                                 uint64_t timeout_ns, cudaStream_t stream) {
   const int64_t R = p.N * p.k;
   if (R == 0) return cudaSuccess;
@@ -606,6 +726,7 @@ cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const 
   g.K = static_cast<int>(p.D);
   g.n_out = static_cast<int>(p.F);
   g.err = err;
+  g.sched = sched;
   g.timeout_ns = timeout_ns;
   switch (p.activation) {
     case MOE_ACT_SILU:
@@ -618,8 +739,8 @@ cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const 
 }
 
 cudaError_t launch_ffn_down_sm100(const moe_problem& p, const void* H, const int32_t* offsets,
-                                  const void* W3, void* Y, int* err, uint64_t timeout_ns,
-                                  cudaStream_t stream) {
+                                  const void* W3, void* Y, int* err, int* sched,
+                                  uint64_t timeout_ns, cudaStream_t stream) {
   const int64_t R = p.N * p.k;
   if (R == 0) return cudaSuccess;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
@@ -633,6 +754,7 @@ cudaError_t launch_ffn_down_sm100(const moe_problem& p, const void* H, const int
   g.K = static_cast<int>(p.F);
   g.n_out = static_cast<int>(p.D);
   g.err = err;
+  g.sched = sched;
   g.timeout_ns = timeout_ns;
   return launch_shape<false, MOE_ACT_SILU>(p, tA, tW3, tW3, g, 256, stream);
 }

@@ -30,25 +30,21 @@ int route_num_blocks(int64_t N, int E);
 
 // Router logits + softmax + top-k + gates. X == nullptr: `logits` is an input.
 // colsum_partial: [route_num_blocks][E] floats (or nullptr when prob_colsum is nullptr).
-// wt: scratch of the tensor-core router (route_tc_wt_bytes), used for bf16 X.
 // noise: [N][E] (p.routing_mode != TOPK). zl_partial: [route_num_blocks] floats, used when
 // z_loss (device scalar) is requested.
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          const float* noise, float* logits, int32_t* idx, float* gate,
                          float* colsum_partial, float* prob_colsum, float* zl_partial,
-                         float* z_loss, __nv_bfloat16* wt, int* err, uint64_t timeout_ns,
-                         cudaStream_t stream);
+                         float* z_loss, int* err, uint64_t timeout_ns, cudaStream_t stream);
 
-// Tensor-core router for bf16 X (logits from a three-term bf16 split of W_r, then the routing
-// decision in the same kernel). colsum_partial may be nullptr; *grid_out = blocks that wrote a
-// colsum partial row.
+// Tensor-core router for bf16 X (logits from a three-term bf16 split of W_r, made in the same
+// kernel, then the routing decision). colsum_partial may be nullptr; *grid_out = blocks that
+// wrote a colsum partial row.
 bool route_tc_supported(const moe_problem& p);
-size_t route_tc_wt_bytes(const moe_problem& p);
 cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
-                            const float* bias, const float* noise, __nv_bfloat16* wt,
-                            float* logits_out, int32_t* idx, float* gate, float* colsum_partial,
-                            float* zl_partial, int* grid_out, int* err, uint64_t timeout_ns,
-                            cudaStream_t stream);
+                            const float* bias, const float* noise, float* logits_out,
+                            int32_t* idx, float* gate, float* colsum_partial, float* zl_partial,
+                            int* grid_out, int* err, uint64_t timeout_ns, cudaStream_t stream);
 
 // 2-D bf16 tensor map (cols contiguous, row stride cols * 2 bytes), box box_cols x box_rows,
 // 128-byte swizzle, out-of-range elements read as zero.
@@ -100,6 +96,15 @@ cudaError_t launch_slot_assign(const moe_problem& p, int64_t capacity, const int
                                int32_t* pos, uint8_t* dropped, int32_t* row_token, int* err,
                                cudaStream_t stream);
 
+// Count, slot assignment and (when X != nullptr) the gather in one cooperative launch.
+// bar: two ints of the workspace header, zero at rest (returned to zero by the kernel).
+// Falls back to launch_slot_assign + launch_gather when no resident grid is available.
+cudaError_t launch_dispatch_fused(const moe_problem& p, int64_t capacity, const int32_t* idx,
+                                  int32_t* chunk_counts, int32_t* load, int32_t* offsets,
+                                  int32_t* pos, uint8_t* dropped, int32_t* row_token,
+                                  const void* X, void* X_perm, int* err, int* bar,
+                                  uint64_t timeout_ns, cudaStream_t stream);
+
 // X_perm[row] = X[row_token[row]] for row < offsets[E] (bulk-copy staged through shared memory).
 cudaError_t launch_gather(const moe_problem& p, const void* X, const int32_t* row_token,
                           const int32_t* offsets, void* X_perm, int* err, cudaStream_t stream);
@@ -112,12 +117,14 @@ cudaError_t launch_gather_rows(const void* src, int64_t n_src, const int32_t* in
 
 // Grouped expert GEMMs, bf16 operands, tcgen05 tensor cores.
 //   up:   H = act(X_perm W1_e) (.) (X_perm W2_e)      down: Y = H W3_e
+// sched: two ints of the workspace header, zero at rest (the in-order tile counter and the
+// count of finished CTAs; the kernel returns them to zero when it ends).
 cudaError_t launch_ffn_up_sm100(const moe_problem& p, const void* X_perm, const int32_t* offsets,
-                                const void* W1, const void* W2, void* H, int* err,
+                                const void* W1, const void* W2, void* H, int* err, int* sched,
                                 uint64_t timeout_ns, cudaStream_t stream);
 cudaError_t launch_ffn_down_sm100(const moe_problem& p, const void* H, const int32_t* offsets,
-                                  const void* W3, void* Y, int* err, uint64_t timeout_ns,
-                                  cudaStream_t stream);
+                                  const void* W3, void* Y, int* err, int* sched,
+                                  uint64_t timeout_ns, cudaStream_t stream);
 
 // The same two steps in fp32 on CUDA cores.
 cudaError_t launch_ffn_up_f32(const moe_problem& p, const void* X_perm, const int32_t* offsets,

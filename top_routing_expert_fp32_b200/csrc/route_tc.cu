@@ -12,18 +12,17 @@
 // concatenated [w0 | w1 | w2] columns gives the three partial dot products; they are added
 // smallest first, z = (z2 + z1) + z0.
 //
-// Kernels:
-//   split_wr_kernel : W_r [D][E] fp32 -> Wt [NB][D] bf16 (the K-major B operand); row
-//                     i * Ep + e holds term i of expert e, padding rows are zero.
-//   route_tc_kernel : clusters of S CTAs (S = 1, 2, 4 or 8), persistent over 128-token tiles;
-//                     CTA r of a cluster accumulates the r-th slice of D (split-K), so that
-//                     a batch of few tiles still spreads over the SMs. Warp 0 issues the TMA
-//                     loads, warp 1 the tcgen05.mma, warps 2-5 are the epilogue: each CTA puts
-//                     its partial logits in its own shared memory, the cluster synchronises
-//                     through mbarriers, and CTA r adds the S partials of tokens
-//                     [r*128/S, (r+1)*128/S) of the tile in slice order (distributed shared
-//                     memory loads), adds the bias and takes the routing decision. No global
-//                     round trip, no atomics; the result does not depend on timing.
+// Kernel (one launch per call): route_tc_kernel, clusters of S CTAs (S = 1, 2, 4 or 8),
+// persistent over 128-token tiles; CTA r of a cluster accumulates the r-th slice of D
+// (split-K), so that a batch of few tiles still spreads over the SMs. Warp 0 issues the TMA
+// loads of X, warps 6-7 write the B operand of each k-block straight from the fp32 W_r (the
+// three bf16 terms of its 64 x E slice, in the 128-byte-swizzled K-major layout the MMA
+// reads; row i * Ep + e holds term i of expert e, padding rows are zero), warp 1 issues the
+// tcgen05.mma, warps 2-5 are the epilogue: each CTA puts its partial logits in its own shared
+// memory, the cluster synchronises through mbarriers, and CTA r adds the S partials of tokens
+// [r*128/S, (r+1)*128/S) of the tile in slice order (distributed shared memory loads), adds
+// the bias and takes the routing decision. No global round trip, no atomics; the result does
+// not depend on timing.
 // Every barrier wait is bounded in time; on a timeout the CTA records MOE_DEVERR_WAIT_TIMEOUT,
 // unwinds, drains its MMAs and frees its tensor memory.
 #include <algorithm>
@@ -39,8 +38,9 @@ namespace {
 constexpr int kRows = 128;        // tokens per tile = accumulator lanes
 constexpr int BK = 64;            // k-block: one 128-byte swizzle row of bf16
 constexpr int UK = 16;            // K of one tcgen05.mma kind::f16
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
 constexpr int kEpiThreads = 128;  // warps 2-5
+constexpr int kConvThreads = 64;  // warps 6-7: the B operand from W_r
 constexpr int kABytes = kRows * BK * 2;  // 16 KB
 constexpr int kMaxStages = 8;
 constexpr int kMaxCluster = 8;
@@ -51,6 +51,7 @@ constexpr int kUnitTarget = 148;  // CTAs wanted per launch (one per SM of a B20
 constexpr int kMaxEc = 64;
 
 struct TcArgs {
+  const float* W_r;        // [D][E] fp32
   const float* bias;       // [E] or nullptr
   float* logits_out;       // [N][E] or nullptr
   int32_t* idx;            // [N][k]
@@ -61,7 +62,7 @@ struct TcArgs {
   int mode;                // MOE_ROUTE_*
   int64_t N;
   int64_t tiles;
-  int E, k, renorm;
+  int D, E, k, renorm;
   int Ep;                  // E rounded up to 8 (TMEM load granularity)
   int NB;                  // MMA N: 3 * Ep rounded up to 16
   int zstride;             // floats per row of the partial-logit buffer (Ep + 4)
@@ -71,11 +72,19 @@ struct TcArgs {
   uint64_t timeout_ns;
 };
 
+// Three bf16 terms of w (w = t0 + t1 + t2 to 24 significant bits): t0 = bf16(w), and the
+// remainders w - t0 and (w - t0) - t1 are exact in fp32.
+__device__ __forceinline__ void split3(float w, float& t0, float& t1, float& t2) {
+  t0 = __bfloat162float(__float2bfloat16_rn(w));
+  const float r1 = w - t0;
+  t1 = __bfloat162float(__float2bfloat16_rn(r1));
+  t2 = r1 - t1;  // rounded to bf16 when packed
+}
+
 // EB: the experts the epilogue holds in registers per token (8, 16, 32 or 64; >= E).
 template <int EB>
 __global__ void __launch_bounds__(kThreads, 1)
-    route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                    const TcArgs a) {
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -102,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 3);  // the X copy (with its bytes) and the two B-writer warps
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -114,7 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     fence_barrier_init();
     prefetch_tensormap(&tmX);
-    prefetch_tensormap(&tmW);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -125,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // every CTA's barriers exist before any remote arrival
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
-  const uint32_t tx_bytes = static_cast<uint32_t>(kABytes + a.NB * BK * 2);
+  const uint32_t tx_bytes = static_cast<uint32_t>(kABytes);
 
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------------ TMA producer
@@ -142,7 +150,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* dst = smem + stage * a.stage_bytes;
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
           tma_load_2d(dst, &tmX, &full[stage], kb * BK, static_cast<int>(tile * kRows));
-          tma_load_2d(dst + a.b_off, &tmW, &full[stage], kb * BK, 0);
           if (++stage == a.stages) {
             stage = 0;
             phase ^= 1u;
@@ -197,6 +204,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(drain);  // flips once every MMA issued above has completed
       if (!mbar_wait(drain, 0, a.timeout_ns)) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
+    }
+  } else if (warp >= 6) {  // ------------------------------------------ B operand writers
+    // Item (c, e): 8 consecutive k of expert e's W_r column (a 16-byte chunk c of the
+    // 128-byte K-major rows), split into its three bf16 terms, stored in rows e, Ep + e and
+    // 2 Ep + e at the 128-byte-swizzled position of chunk c (chunk c ^ (row & 7)). Lanes take
+    // consecutive e, so the fp32 reads are coalesced and each 8-lane phase of the 16-byte
+    // stores hits 8 distinct chunks.
+    const int ct = threadIdx.x - (kThreads - kConvThreads);
+    const int E = a.E;
+    const int items = 8 * E;
+    // Padding rows (e in [E, Ep) of each term, and rows past 3 Ep) stay zero: written once.
+    const int pad_rows = a.NB - 3 * E;
+    for (int s = 0; s < a.stages; ++s) {
+      uint8_t* b = smem + s * a.stage_bytes + a.b_off;
+      for (int i = ct; i < pad_rows * 8; i += kConvThreads) {
+        const int pr = i >> 3, c = i & 7;
+        int n;  // the pr-th padding row
+        if (pr < 3 * (a.Ep - E)) n = (pr / (a.Ep - E)) * a.Ep + E + pr % (a.Ep - E);
+        else n = 3 * a.Ep + (pr - 3 * (a.Ep - E));
+        *reinterpret_cast<uint4*>(b + n * 128 + ((c ^ (n & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t tile = first_tile; ok && tile < a.tiles; tile += a.num_clusters) {
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, a.timeout_ns)) {
+          if (lane == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
+          ok = false;
+          break;
+        }
+        uint8_t* b = smem + stage * a.stage_bytes + a.b_off;
+        for (int i = ct; i < items; i += kConvThreads) {
+          const int c = i / E, e = i - c * E;
+          const int d0 = kb * BK + c * 8;
+          float t0[8], t1[8], t2[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float w = d0 + j < a.D ? __ldg(a.W_r + static_cast<int64_t>(d0 + j) * E + e) : 0.f;
+            split3(w, t0[j], t1[j], t2[j]);
+          }
+          const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
+                                      pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
+          const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
+                                      pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
+          const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
+                                      pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
+          const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
+          *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
+          *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
+          *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
+        }
+        fence_proxy_async_smem();  // generic-proxy stores before the MMA (async proxy) reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
     }
   } else {  // ------------------------------------------------------------------- epilogue
     // Thread row = q*32 + lane reads TMEM lane `row` (tile row = token). With S = 1 it owns
@@ -348,47 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
 }
 
-// Wt[i * Ep + e][d] = term i of W_r[d][e] (zero for e >= E and for rows >= 3 * Ep).
-// One thread per (row group, 8 consecutive d): rows e, Ep + e and 2 Ep + e for e < Ep, or one
-// padding row past 3 Ep; each row written as one 16-byte store (D % 8 == 0).
-constexpr int kSplitThreads = 256;
-
-__global__ void __launch_bounds__(kSplitThreads)
-    split_wr_kernel(const float* __restrict__ W_r, __nv_bfloat16* __restrict__ Wt, int D, int E,
-                    int Ep, int NB) {
-  const int chunks = D / 8;
-  const int groups = Ep + (NB - 3 * Ep);  // experts, then padding rows
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * kSplitThreads + threadIdx.x;
-  if (i >= static_cast<int64_t>(groups) * chunks) return;
-  const int grp = static_cast<int>(i / chunks);
-  const int d0 = static_cast<int>(i - static_cast<int64_t>(grp) * chunks) * 8;
-  if (grp >= Ep) {  // padding row 3 Ep + (grp - Ep)
-    *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(3 * Ep + grp - Ep) * D + d0) =
-        make_uint4(0u, 0u, 0u, 0u);
-    return;
-  }
-  const int e = grp;
-  float t0[8], t1[8], t2[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float w = e < E ? __ldg(W_r + static_cast<int64_t>(d0 + j) * E + e) : 0.f;
-    t0[j] = __bfloat162float(__float2bfloat16_rn(w));
-    const float r1 = w - t0[j];  // exact: t0 holds w's leading 8 significant bits
-    t1[j] = __bfloat162float(__float2bfloat16_rn(r1));
-    t2[j] = r1 - t1[j];          // exact for the same reason; rounded to bf16 below
-  }
-  uint4 v0, v1, v2;
-  v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]), pack_bf16x2(t0[4], t0[5]),
-                  pack_bf16x2(t0[6], t0[7]));
-  v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]), pack_bf16x2(t1[4], t1[5]),
-                  pack_bf16x2(t1[6], t1[7]));
-  v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]), pack_bf16x2(t2[4], t2[5]),
-                  pack_bf16x2(t2[6], t2[7]));
-  *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(e) * D + d0) = v0;
-  *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(Ep + e) * D + d0) = v1;
-  *reinterpret_cast<uint4*>(Wt + static_cast<int64_t>(2 * Ep + e) * D + d0) = v2;
-}
-
 struct TcShape {
   int Ep, NB, zstride, num_kb, S, num_clusters, stages;
   int64_t tiles;
@@ -438,34 +465,22 @@ bool route_tc_supported(const moe_problem& p) {
   return p.dtype == MOE_DTYPE_BF16 && p.E <= kMaxEc;
 }
 
-size_t route_tc_wt_bytes(const moe_problem& p) {
-  if (!route_tc_supported(p)) return 0;
-  const TcShape s = tc_shape(p.N, static_cast<int>(p.D), p.E);
-  return static_cast<size_t>(s.NB) * static_cast<size_t>(p.D) * 2;
-}
-
 cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
-                            const float* bias, const float* noise, __nv_bfloat16* wt,
-                            float* logits_out, int32_t* idx, float* gate, float* colsum_partial,
-                            float* zl_partial, int* grid_out, int* err, uint64_t timeout_ns,
-                            cudaStream_t stream) {
+                            const float* bias, const float* noise, float* logits_out,
+                            int32_t* idx, float* gate, float* colsum_partial, float* zl_partial,
+                            int* grid_out, int* err, uint64_t timeout_ns, cudaStream_t stream) {
   const TcShape s = tc_shape(p.N, static_cast<int>(p.D), p.E);
   *grid_out = 0;
   if (p.N == 0) return cudaSuccess;
   if (s.stages < 2) return cudaErrorInvalidConfiguration;
   const int D = static_cast<int>(p.D);
-  const int64_t split_threads = static_cast<int64_t>(s.Ep + (s.NB - 3 * s.Ep)) * (D / 8);
-  split_wr_kernel<<<static_cast<unsigned>((split_threads + kSplitThreads - 1) / kSplitThreads),
-                    kSplitThreads, 0, stream>>>(W_r, wt, D, p.E, s.Ep, s.NB);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  CUtensorMap tX, tW;
+  CUtensorMap tX;
   if (!make_tensor_map_2d_bf16(&tX, X, static_cast<uint64_t>(D), static_cast<uint64_t>(p.N), 64,
-                               kRows) ||
-      !make_tensor_map_2d_bf16(&tW, wt, static_cast<uint64_t>(D), static_cast<uint64_t>(s.NB), 64,
-                               static_cast<uint32_t>(s.NB)))
+                               kRows))
     return cudaErrorInvalidValue;
+  cudaError_t e = cudaSuccess;
   TcArgs a;
+  a.W_r = W_r;
   a.bias = bias;
   a.logits_out = logits_out;
   a.idx = idx;
@@ -476,6 +491,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   a.mode = p.routing_mode;
   a.N = p.N;
   a.tiles = s.tiles;
+  a.D = D;
   a.E = p.E;
   a.k = p.k;
   a.renorm = p.renormalize;
@@ -493,7 +509,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   a.bar_off = s.bar_off;
   a.err = err;
   a.timeout_ns = timeout_ns;
-  void (*kern)(const CUtensorMap, const CUtensorMap, const TcArgs) =
+  void (*kern)(const CUtensorMap, const TcArgs) =
       s.Ep <= 8 ? route_tc_kernel<8>
                 : (s.Ep <= 16 ? route_tc_kernel<16> : (s.Ep <= 32 ? route_tc_kernel<32> : route_tc_kernel<64>));
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -511,7 +527,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tX, tW, a);
+  e = cudaLaunchKernelEx(&cfg, kern, tX, a);
   if (e != cudaSuccess) return e;
   *grid_out = s.num_clusters * s.S;
   return cudaGetLastError();
