@@ -428,6 +428,12 @@ def run_gpu(args, cfg, world, rank, device):
     sampler.stop()
     if abi.device_error(ws) != 0:
         raise RuntimeError("device error during the timed steps")
+    clocks = sampler.summary(t_wall0, t_wall1)
+    clocks["timed_region_s"] = t_wall1 - t_wall0
+    # The tensor-core denominator: the sustained cuBLAS figure for kernels timed inside a long
+    # run (a timed region of a second or more, or the power cap active), the burst figure for
+    # a short one; the other is reported beside it.
+    sustained = clocks["timed_region_s"] >= 1.0 or "sw_power_cap" in clocks.get("reasons", [])
 
     per = {n: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, n in enumerate(names)}
     total_ms = sum(ev[0].elapsed_time(ev[5]) for ev in evs)
@@ -444,7 +450,9 @@ def run_gpu(args, cfg, world, rank, device):
     bytes_gather = (tokens_with_kept + kept) * D * es
     bytes_combine = kept * D * es + N * D * es + N * k * 13
     hbm = peaks["hbm_gbs"]
-    tc = peaks["bf16_tflops"]
+    tc_burst = peaks["bf16_tflops"]
+    tc = peaks["bf16_tflops_sustained"] if sustained else tc_burst
+    tc_kind = "bf16 sustained" if sustained else "bf16 burst"
     kern = {
         "route": {"ms": mean["route"], "GB/s": bytes_route / mean["route"] / 1e6},
         "dispatch": {"ms": mean["dispatch"], "gather_GB/s_lower_bound":
@@ -458,6 +466,7 @@ def run_gpu(args, cfg, world, rank, device):
         kern[n]["frac_8TBs"] = kern[n]["GB/s"] / DATASHEET_HBM_GBS
     for n in ("up", "down"):
         kern[n]["frac_bf16_peak"] = kern[n]["TFLOP/s"] / tc
+        kern[n]["frac_bf16_burst"] = kern[n]["TFLOP/s"] / tc_burst
         kern[n]["frac_bf16_datasheet"] = kern[n]["TFLOP/s"] / DATASHEET_BF16_TFLOPS
     ffn_ms = mean["up"] + mean["down"]
     gemm_tflops = 6.0 * kept * D * F / ffn_ms / 1e9
@@ -477,7 +486,8 @@ def run_gpu(args, cfg, world, rank, device):
         roof = {"kernel": up_kernel + " (expert up-projection + gating)",
                 "bound": "tensor", "achieved": kern["up"]["TFLOP/s"], "peak": tc,
                 "unit": "TFLOP/s", "frac": kern["up"]["TFLOP/s"] / tc,
-                "peak_source": psrc + ", bf16 burst", "flops_per_launch": flops_up}
+                "peak_source": f"{psrc}, {tc_kind}", "frac_burst": kern["up"]["TFLOP/s"] / tc_burst,
+                "flops_per_launch": flops_up}
     else:
         gbs = bytes_up / mean["up"] / 1e6
         roof = {"kernel": up_kernel
@@ -603,9 +613,8 @@ def run_gpu(args, cfg, world, rank, device):
                 "single_call_value": e2e_single,
                 "single_call_api": None if w8 else "moe_forward_host, one call per step"},
         "gpu_launches": sum(launches.values()) * args.steps,
-        "clocks": sampler.summary(t_wall0, t_wall1),
+        "clocks": clocks,
     }
-    line["clocks"]["timed_region_s"] = t_wall1 - t_wall0
     mhz = line["clocks"].get("sm_mhz")
     if roof["bound"] == "tensor" and mhz:
         # Tensor throughput scales with the SM clock: the achieved rate against the datasheet
