@@ -421,6 +421,14 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
   return v;
 }
 
+// 16 bytes into the shared memory of a CTA of this cluster (address from mapa_shared); a later
+// release.cluster arrival of the same thread orders it before the receiver's acquire.
+__device__ __forceinline__ void st_dsmem_f4(uint32_t cluster_addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 // Orders this thread's earlier shared-memory accesses before its later ones as seen by the
 // other CTAs of the cluster (used before another lane signals a peer).
 __device__ __forceinline__ void fence_cluster() {

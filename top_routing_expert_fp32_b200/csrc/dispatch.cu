@@ -301,14 +301,18 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------ fused dispatch
 //
 // Count, slot assignment and gather in one cooperative launch (every block resident at
-// once). Phase 1: blocks b < nchunks count chunk b per expert (as count_kernel). Grid
-// barrier. Phase 2: the same blocks assign their chunks' positions, drop flags and row map
-// (as assign_kernel; block 0 also writes load and offsets). Grid barrier. Phase 3: every
-// block copies rows X_perm[row] = X[row_token[row]] for row < offsets[E], one warp per row
-// at a time, 16-byte words with four loads in flight per lane. Data another block wrote in an
-// earlier phase is read at L2 (ld.global.cg). The barrier counters live in the workspace
-// header (zero at rest); the last block to finish returns them to zero, also after a barrier
-// timed out. Bit-exact with the three-kernel path.
+// once). Phase 1: blocks b < nchunks count chunk b (kDispatchChunk records) per expert (as
+// count_kernel). Grid barrier. Phase 2: block b takes the b-th of G equal slices of the
+// records; an expert's records before the slice are the counts of the earlier chunks plus a
+// recount of the slice's own chunk up to the slice start; inside the slice, warps rank equal
+// experts with __match_any_sync and a per-expert scan over the warps orders them (the stable
+// counting-sort rank, as assign_kernel). The block writes its records' positions, drop flags
+// and row map (block 0 also load and offsets) and copies the X rows of its kept records to
+// X_perm straight away (one warp per row, 16-byte words, four loads in flight per lane): no
+// second barrier, and every block has copy work. Counts another block wrote are read at L2
+// (ld.global.cg). The barrier counters live in the workspace header (zero at rest); the last
+// block to finish returns them to zero, also after the barrier timed out. Bit-exact with the
+// three-kernel path.
 
 constexpr int kFusedThreads = 512;
 
@@ -364,6 +368,8 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
   __shared__ int s_tot[kMaxE];
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_wpre[kFusedThreads / 32][kMaxE];
+  __shared__ int s_row[kFusedThreads];      // X_perm row of each record of the tile (-1: none)
+  __shared__ int32_t s_tok[kFusedThreads];  // and its token
   const int E = a.E;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -391,20 +397,35 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
   }
   ok = grid_barrier(a.bar, G, a.timeout_ns, a.err);
 
-  // Phase 2: positions in record order (stable counting-sort rank), drop flags, row map.
-  for (int c = blockIdx.x; ok && c < a.nchunks; c += G) {
+  // Phase 2: this block's slice [s0, s1) of the records.
+  const int64_t slice = (a.R + G - 1) / G;
+  const int64_t s0 = std::min<int64_t>(a.R, static_cast<int64_t>(blockIdx.x) * slice);
+  const int64_t s1 = std::min<int64_t>(a.R, s0 + slice);
+  if (ok && s0 < s1) {
+    const int c0 = static_cast<int>(s0 / kDispatchChunk);
+    for (int e = threadIdx.x; e < E; e += kFusedThreads) hist[e] = 0;
+    __syncthreads();
+    // Recount the records of chunk c0 before s0.
+    for (int64_t r = static_cast<int64_t>(c0) * kDispatchChunk + threadIdx.x; r < s0;
+         r += kFusedThreads) {
+      int64_t t, j;
+      record_at(r, a.N, a.k, a.token_major, t, j);
+      const int e = a.idx[t * a.k + j];
+      if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    }
     if (threadIdx.x < E) {
       const int e = threadIdx.x;
       int base = 0, total = 0;
       for (int cc = 0; cc < a.nchunks; ++cc) {
         const int v = __ldcg(a.counts + static_cast<int64_t>(cc) * E + e);
-        if (cc < c) base += v;
+        if (cc < c0) base += v;
         total += v;
       }
       s_base[e] = base;
       s_tot[e] = total;
     }
     __syncthreads();
+    if (threadIdx.x < E) s_base[threadIdx.x] += hist[threadIdx.x];
     if (threadIdx.x == 0) {
       int run = 0;
       for (int e = 0; e < E; ++e) {
@@ -413,7 +434,7 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
         run += static_cast<int>(tot < a.C ? tot : a.C);
       }
       s_off[E] = run;
-      if (c == 0) {
+      if (blockIdx.x == 0) {
         for (int e = 0; e < E; ++e) {
           a.load[e] = s_tot[e];
           a.offsets[e] = s_off[e];
@@ -422,15 +443,14 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
       }
     }
     __syncthreads();
-    int running = 0;  // thread e < E: records of expert e in earlier tiles of this chunk
-    const int64_t r0 = static_cast<int64_t>(c) * kDispatchChunk;
-    const int64_t r1 = std::min<int64_t>(r0 + kDispatchChunk, a.R);
+    int running = 0;  // thread e < E: records of expert e in earlier tiles of this slice
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int64_t tile = r0; tile < r1; tile += kFusedThreads) {
+    const uint32_t words = a.row_words;
+    for (int64_t tile = s0; tile < s1; tile += kFusedThreads) {
       for (int i = threadIdx.x; i < kWarps * kMaxE; i += kFusedThreads) (&s_wpre[0][0])[i] = 0;
       __syncthreads();
       const int64_t r = tile + threadIdx.x;
-      const bool valid = r < r1;
+      const bool valid = r < s1;
       int64_t j = 0, t = 0;
       int e = -1;
       if (valid) {
@@ -453,6 +473,7 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
         running = run;
       }
       __syncthreads();
+      int my_row = -1;
       if (valid) {
         const int64_t rec = t * a.k + j;
         if (e >= 0) {
@@ -460,38 +481,40 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
           const bool drop = p >= a.C;
           a.pos[rec] = p;
           a.dropped[rec] = drop ? 1 : 0;
-          if (!drop) a.row_token[s_off[e] + p] = static_cast<int32_t>(t);
+          if (!drop) {
+            my_row = s_off[e] + p;
+            a.row_token[my_row] = static_cast<int32_t>(t);
+          }
         } else {
           a.pos[rec] = -1;
           a.dropped[rec] = 1;
         }
       }
-      __syncthreads();
-    }
-  }
-
-  // Phase 3: the permutation, one warp per row.
-  if (a.X != nullptr) {
-    ok = grid_barrier(a.bar, 2 * G, a.timeout_ns, a.err) && ok;
-    if (ok) {
-      const int64_t rows = __ldcg(a.offsets + E);
-      const int64_t W = static_cast<int64_t>(G) * kWarps;
-      const uint32_t words = a.row_words;
-      for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + warp; row < rows; row += W) {
-        const int64_t tok = __ldcg(a.row_token + row);
-        const uint4* src = reinterpret_cast<const uint4*>(a.X) + tok * words;
-        uint4* dst = reinterpret_cast<uint4*>(a.X_perm) + row * words;
-        uint32_t w = lane;
-        for (; w + 96 < words; w += 128) {
-          const uint4 v0 = __ldg(src + w), v1 = __ldg(src + w + 32), v2 = __ldg(src + w + 64),
-                      v3 = __ldg(src + w + 96);
-          dst[w] = v0;
-          dst[w + 32] = v1;
-          dst[w + 64] = v2;
-          dst[w + 96] = v3;
+      if (a.X != nullptr) {
+        // Copy the kept rows of this tile, spread over all warps of the block.
+        s_row[threadIdx.x] = my_row;
+        s_tok[threadIdx.x] = static_cast<int32_t>(t);
+        __syncthreads();
+        const int n_here = static_cast<int>(std::min<int64_t>(kFusedThreads, s1 - tile));
+        for (int i = warp; i < n_here; i += kWarps) {
+          const int row = s_row[i];
+          if (row < 0) continue;
+          const int64_t tok = s_tok[i];
+          const uint4* src = reinterpret_cast<const uint4*>(a.X) + tok * words;
+          uint4* dst = reinterpret_cast<uint4*>(a.X_perm) + static_cast<int64_t>(row) * words;
+          uint32_t w = lane;
+          for (; w + 96 < words; w += 128) {
+            const uint4 v0 = __ldg(src + w), v1 = __ldg(src + w + 32),
+                        v2 = __ldg(src + w + 64), v3 = __ldg(src + w + 96);
+            dst[w] = v0;
+            dst[w + 32] = v1;
+            dst[w + 64] = v2;
+            dst[w + 96] = v3;
+          }
+          for (; w < words; w += 32) dst[w] = __ldg(src + w);
         }
-        for (; w < words; w += 32) dst[w] = __ldg(src + w);
       }
+      __syncthreads();
     }
   }
 
@@ -621,12 +644,15 @@ cudaError_t launch_dispatch_fused(const moe_problem& p, int64_t capacity, const 
   a.token_major = p.capacity_order == MOE_ORDER_TOKEN_MAJOR;
   a.row_words = static_cast<uint32_t>(static_cast<int64_t>(p.D) * elem / 16);
   a.timeout_ns = timeout_ns;
-  // Enough warps for the gather (one row each in flight), at least one block per chunk.
-  const int64_t want_rows = X != nullptr ? R : 0;
-  const int64_t want = std::max<int64_t>(
-      nchunks, (want_rows + kFusedThreads / 32 - 1) / (kFusedThreads / 32));
-  // More chunks than resident blocks: blocks loop over chunks (still one launch).
-  const int grid = static_cast<int>(std::min<int64_t>(want, max_blocks));
+  // With rows to copy, every resident block takes a slice (the copy is spread over the whole
+  // device); without, one block per 512 records. At least one block per chunk.
+  const int64_t want = X != nullptr ? max_blocks
+                                    : std::max<int64_t>(nchunks, (R + kFusedThreads - 1) /
+                                                                     kFusedThreads);
+  // At most two blocks per SM (room for a kernel of another stream beside it); with more
+  // chunks than blocks, blocks loop over chunks (still one launch).
+  const int grid = static_cast<int>(
+      std::min<int64_t>(want, std::min<int64_t>(max_blocks, 2 * static_cast<int64_t>(num_sms()))));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(std::max(grid, 1)));
   cfg.blockDim = dim3(kFusedThreads);

@@ -15,14 +15,17 @@
 // Kernel (one launch per call): route_tc_kernel, clusters of S CTAs (S = 1, 2, 4 or 8),
 // persistent over 128-token tiles; CTA r of a cluster accumulates the r-th slice of D
 // (split-K), so that a batch of few tiles still spreads over the SMs. Warp 0 issues the TMA
-// loads of X, warps 6-7 write the B operand of each k-block straight from the fp32 W_r (the
-// three bf16 terms of its 64 x E slice, in the 128-byte-swizzled K-major layout the MMA
-// reads; row i * Ep + e holds term i of expert e, padding rows are zero), warp 1 issues the
-// tcgen05.mma, warps 2-5 are the epilogue: each CTA puts its partial logits in its own shared
-// memory, the cluster synchronises through mbarriers, and CTA r adds the S partials of tokens
-// [r*128/S, (r+1)*128/S) of the tile in slice order (distributed shared memory loads), adds
-// the bias and takes the routing decision. No global round trip, no atomics; the result does
-// not depend on timing.
+// loads of X and a bulk copy of the k-block's fp32 W_r slice (64 x E, contiguous) into the
+// stage; warps 6-9 turn that slice into the B operand (the three bf16 terms, in the
+// 128-byte-swizzled K-major layout the MMA reads; row i * Ep + e holds term i of expert e,
+// padding rows are zero) from shared memory, so no global latency sits between the
+// k-blocks; warp 1 issues the
+// tcgen05.mma, warps 2-5 are the epilogue: CTA r owns tokens [r*128/S, (r+1)*128/S) of the
+// tile; every epilogue thread stores its row's partial logits into the owner's shared memory
+// (a slot per source CTA, remote stores) and arrives there (release.cluster), and the owner
+// adds the S slots of its rows in slice order from its own shared memory, adds the bias and
+// takes the routing decision. No global round trip, no remote loads, no atomics; the result
+// does not depend on timing.
 // Every barrier wait is bounded in time; on a timeout the CTA records MOE_DEVERR_WAIT_TIMEOUT,
 // unwinds, drains its MMAs and frees its tensor memory.
 #include <algorithm>
@@ -38,9 +41,10 @@ namespace {
 constexpr int kRows = 128;        // tokens per tile = accumulator lanes
 constexpr int BK = 64;            // k-block: one 128-byte swizzle row of bf16
 constexpr int UK = 16;            // K of one tcgen05.mma kind::f16
-constexpr int kThreads = 256;
-constexpr int kEpiThreads = 128;  // warps 2-5
-constexpr int kConvThreads = 64;  // warps 6-7: the B operand from W_r
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 128;   // warps 2-5
+constexpr int kConvThreads = 128;  // warps 6-9: the B operand from the staged W_r slice
+constexpr int kConvWarps = kConvThreads / 32;
 constexpr int kABytes = kRows * BK * 2;  // 16 KB
 constexpr int kMaxStages = 8;
 constexpr int kMaxCluster = 8;
@@ -67,7 +71,7 @@ struct TcArgs {
   int NB;                  // MMA N: 3 * Ep rounded up to 16
   int zstride;             // floats per row of the partial-logit buffer (Ep + 4)
   int num_kb, S, num_clusters, stages;
-  uint32_t stage_bytes, b_off, zbuf_off, sz_off, bar_off;
+  uint32_t stage_bytes, b_off, w_off, zbuf_off, sz_off, bar_off;
   int* err;
   uint64_t timeout_ns;
 };
@@ -94,10 +98,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* zready = tempty + 2;  // all S partials of the current tile are in place
-  uint64_t* zfree = zready + 1;   // every CTA has finished reading this CTA's partials
+  uint64_t* zready = tempty + 2;  // the S partials of this CTA's rows have been stored here
+  uint64_t* zfree = zready + 1;   // the owners have read the partials this CTA stored
   uint64_t* drain = zfree + 1;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* wfull = drain + 1;    // [kMaxStages] the k-block's fp32 W_r slice has landed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(wfull + kMaxStages);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -111,15 +116,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
-      mbar_init(&full[s], 3);  // the X copy (with its bytes) and the two B-writer warps
+      mbar_init(&full[s], 1 + kConvWarps);  // the X copy (with its bytes), the B writers
       mbar_init(&empty[s], 1);
+      mbar_init(&wfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
     }
-    mbar_init(zready, 4 * S);  // one arrival per epilogue warp of every CTA of the cluster
-    mbar_init(zfree, 4 * S);
+    // zready: one arrival per pushed row (T owned rows x S source CTAs = 128); zfree: one per
+    // owned row read, from the owner threads of the S CTAs (S x T = 128).
+    mbar_init(zready, kRows);
+    mbar_init(zfree, kRows);
     mbar_init(drain, 1);
     fence_barrier_init();
     prefetch_tensormap(&tmX);
@@ -150,6 +158,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* dst = smem + stage * a.stage_bytes;
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
           tma_load_2d(dst, &tmX, &full[stage], kb * BK, static_cast<int>(tile * kRows));
+          // W_r rows [kb*64, kb*64 + rows) are one contiguous run of rows * E floats (a
+          // multiple of 32 bytes, since D % 8 == 0); the B writers convert it.
+          const int wrows = min(BK, a.D - kb * BK);
+          const uint32_t wbytes = static_cast<uint32_t>(wrows * a.E * 4);
+          mbar_arrive_expect_tx(&wfull[stage], wbytes);
+          bulk_g2s(dst + a.w_off, a.W_r + static_cast<int64_t>(kb) * BK * a.E, wbytes,
+                   &wfull[stage]);
           if (++stage == a.stages) {
             stage = 0;
             phase ^= 1u;
@@ -231,31 +246,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t tile = first_tile; ok && tile < a.tiles; tile += a.num_clusters) {
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, a.timeout_ns)) {
+        // The slice lands after the producer has seen this stage free (empty), so waiting for
+        // it also orders these stores after the MMAs that read the stage's previous B.
+        if (!mbar_wait(&wfull[stage], phase, a.timeout_ns)) {
           if (lane == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
           ok = false;
           break;
         }
         uint8_t* b = smem + stage * a.stage_bytes + a.b_off;
-        for (int i = ct; i < items; i += kConvThreads) {
-          const int c = i / E, e = i - c * E;
-          const int d0 = kb * BK + c * 8;
-          float t0[8], t1[8], t2[8];
+        const float* wf = reinterpret_cast<const float*>(smem + stage * a.stage_bytes + a.w_off);
+        const int wrows = min(BK, a.D - kb * BK);
+        // kBatch items per thread at a time, all their loads first: independent chains for
+        // the scheduler (E = 64 gives each thread 4 items per k-block).
+        constexpr int kBatch = 4;
+        for (int i0 = ct; i0 < items; i0 += kBatch * kConvThreads) {
+          float w[kBatch][8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float w = d0 + j < a.D ? __ldg(a.W_r + static_cast<int64_t>(d0 + j) * E + e) : 0.f;
-            split3(w, t0[j], t1[j], t2[j]);
+          for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kConvThreads;
+            const int c = i / E, e = i - c * E;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int d = c * 8 + j;
+              w[u][j] = (i < items && d < wrows) ? wf[d * E + e] : 0.f;
+            }
           }
-          const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
-                                      pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
-          const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
-                                      pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
-          const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
-                                      pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
-          const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
-          *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
-          *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
-          *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kConvThreads;
+            if (i >= items) break;
+            const int c = i / E, e = i - c * E;
+            float t0[8], t1[8], t2[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) split3(w[u][j], t0[j], t1[j], t2[j]);
+            const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
+                                        pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
+            const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
+                                        pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
+            const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
+                                        pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
+            const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
+            *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
+            *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
+            *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
+          }
         }
         fence_proxy_async_smem();  // generic-proxy stores before the MMA (async proxy) reads
         __syncwarp();
@@ -277,7 +311,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int share0 = static_cast<int>(rank) * T;
     const bool owner = row >= share0 && row < share0 + T;
     const int E = a.E;
-    const uint32_t zrow_s = smem_u32(zbuf) + static_cast<uint32_t>(row * a.zstride) * 4u;
     float colsum_acc = 0.f;
     float zl_acc = 0.f;
     int it = 0;
@@ -285,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = it & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
       bool ok = mbar_wait(&tfull[acc], acc_phase, a.timeout_ns);
-      // The previous tile's partials must have been read by every CTA before they are
+      // The owners must have read this CTA's pushes of the previous tile before they are
       // overwritten.
       if (S > 1 && ok && it > 0)
         ok = mbar_wait_cluster(zfree, static_cast<uint32_t>(it - 1) & 1u, a.timeout_ns);
@@ -320,56 +353,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);  // the MMA warp may reuse this accumulator
       if (S > 1) {
-        // 2. Publish this CTA's partials, then add the S partials of the owned rows in slice
-        //    order (distributed shared memory).
+        // 2. Push this row's partial to its owner q (slot [rank][row - q T] of q's receive
+        //    buffer), arrive on q's zready; then each owner adds the S slots of its rows in
+        //    slice order, locally.
+        const int q = row / T;
+        const uint32_t dst = mapa_shared(
+            smem_u32(zbuf) + static_cast<uint32_t>(((static_cast<int>(rank) * T + row - q * T) *
+                                                    a.zstride) * 4),
+            static_cast<uint32_t>(q));
 #pragma unroll
         for (int c = 0; c < EB; c += 4)
-          if (c < a.Ep)
-            reinterpret_cast<float4*>(zbuf + row * a.zstride)[c / 4] =
-                make_float4(z[c], z[c + 1], z[c + 2], z[c + 3]);
-        fence_cluster();  // this lane's partials before lane 0's release to the peers
-        __syncwarp();
-        if (lane == 0)
-          for (int r = 0; r < S; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(zready), r));
+          if (c < a.Ep) st_dsmem_f4(dst + c * 4u, make_float4(z[c], z[c + 1], z[c + 2], z[c + 3]));
+        mbar_arrive_cluster(mapa_shared(smem_u32(zready), static_cast<uint32_t>(q)));
         ok = mbar_wait_cluster(zready, static_cast<uint32_t>(it) & 1u, a.timeout_ns);
         if (named_bar_any(1, kEpiThreads, !ok)) {
           if (et == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
           break;
         }
         if (owner) {
-          float v[EB];
+          const float* slot = zbuf + (row - share0) * a.zstride;  // slice r: + r T zstride
 #pragma unroll
           for (int c = 0; c < EB; c += 4) {
             if (c < a.Ep) {
-              float4 acc4 = rank == 0 ? make_float4(z[c], z[c + 1], z[c + 2], z[c + 3])
-                                      : ld_dsmem_f4(mapa_shared(zrow_s + c * 4u, 0));
+              float4 acc4 = *reinterpret_cast<const float4*>(slot + c);
 #pragma unroll
               for (int r = 1; r < kMaxCluster; ++r) {
                 if (r < S) {
-                  const float4 w = r == static_cast<int>(rank)
-                                       ? make_float4(z[c], z[c + 1], z[c + 2], z[c + 3])
-                                       : ld_dsmem_f4(mapa_shared(zrow_s + c * 4u, r));
+                  const float4 w = *reinterpret_cast<const float4*>(slot + r * T * a.zstride + c);
                   acc4.x += w.x;
                   acc4.y += w.y;
                   acc4.z += w.z;
                   acc4.w += w.w;
                 }
               }
-              v[c] = acc4.x;
-              v[c + 1] = acc4.y;
-              v[c + 2] = acc4.z;
-              v[c + 3] = acc4.w;
+              z[c] = acc4.x;
+              z[c + 1] = acc4.y;
+              z[c + 2] = acc4.z;
+              z[c + 3] = acc4.w;
             } else {
-              v[c] = v[c + 1] = v[c + 2] = v[c + 3] = 0.f;
+              z[c] = z[c + 1] = z[c + 2] = z[c + 3] = 0.f;
             }
           }
-#pragma unroll
-          for (int e = 0; e < EB; ++e) z[e] = v[e];
+          // Another tile follows: tell every source CTA its slot of this row has been read.
+          if (tile + a.num_clusters < a.tiles)
+            for (int r = 0; r < S; ++r)
+              mbar_arrive_cluster(mapa_shared(smem_u32(zfree), static_cast<uint32_t>(r)));
         }
-        fence_cluster();  // this lane's reads of the peers' partials before the release below
-        __syncwarp();
-        if (lane == 0)  // done reading every CTA's partials of this tile
-          for (int r = 0; r < S; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(zfree), r));
       }
       // 3. Bias and the routing decision for the owned tokens.
       const int64_t t = tile * kRows + row;
@@ -381,12 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < EB; ++e)
             if (e < E) a.logits_out[t * E + e] = z[e];
+        // The decision runs from the token's row of shared memory (loops over E, not unrolled
+        // per expert and per choice: compact code, and the same arithmetic as the SIMT
+        // routers); with the balance statistic the row is left holding the probabilities.
         float* zt = s_z + (row - share0) * (E + 1);  // column E: (log Z)^2 of the token
+#pragma unroll
+        for (int e = 0; e < EB; ++e)
+          if (e < E) zt[e] = z[e];
         float lse = 0.f;
-        select_token_regs<EB>(z, E, a.k, a.renorm, a.mode,
-                              a.noise != nullptr ? a.noise + t * E : nullptr, a.idx + t * a.k,
-                              a.gate + t * a.k, a.colsum_partial != nullptr ? zt : nullptr,
-                              a.zl_partial != nullptr ? &lse : nullptr);
+        select_token(zt, E, a.k, a.renorm, a.mode, a.noise != nullptr ? a.noise + t * E : nullptr,
+                     a.idx + t * a.k, a.gate + t * a.k, a.colsum_partial != nullptr,
+                     a.zl_partial != nullptr ? &lse : nullptr);
         zt[E] = lse * lse;
       }
       if (a.colsum_partial != nullptr || a.zl_partial != nullptr) {  // sums in token order
@@ -416,10 +450,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
 }
 
+constexpr uint32_t kBarBytes = 512;  // mbarriers and the TMEM address
+
 struct TcShape {
   int Ep, NB, zstride, num_kb, S, num_clusters, stages;
   int64_t tiles;
-  uint32_t stage_bytes, b_off, zbuf_off, sz_off, bar_off, smem_bytes;
+  uint32_t stage_bytes, b_off, w_off, zbuf_off, sz_off, bar_off, smem_bytes;
 };
 
 TcShape tc_shape(int64_t N, int D, int E) {
@@ -443,19 +479,23 @@ TcShape tc_shape(int64_t N, int D, int E) {
   }
   s.num_clusters = static_cast<int>(
       std::max<int64_t>(1, std::min<int64_t>(s.tiles, kUnitTarget / s.S)));
-  // Shared memory: [stages][A 16 KB | B] [partials 128 x zstride] [summed logits] [barriers]
+  // Shared memory: [stages][A 16 KB | B (bf16 terms) | W (fp32 slice, 64 x E)]
+  // [partials 128 x zstride] [summed logits] [barriers]; A and B 1024-byte aligned.
+  const uint32_t b_bytes = static_cast<uint32_t>((s.NB * BK * 2 + 1023) / 1024 * 1024);
+  const uint32_t w_bytes = static_cast<uint32_t>((BK * E * 4 + 1023) / 1024 * 1024);
   s.b_off = kABytes;
-  s.stage_bytes = static_cast<uint32_t>(kABytes + (s.NB * BK * 2 + 1023) / 1024 * 1024);
+  s.w_off = kABytes + b_bytes;
+  s.stage_bytes = kABytes + b_bytes + w_bytes;
   // Partials are exchanged only between the CTAs of a cluster (S > 1).
   const uint32_t zbuf_bytes = s.S > 1 ? static_cast<uint32_t>(kRows * s.zstride * 4) : 0u;
   const uint32_t sz_bytes = static_cast<uint32_t>(((kRows / s.S) * (E + 1) * 4 + 15) / 16 * 16);
-  const uint32_t fixed = 1024 /*align*/ + 256 /*barriers*/ + zbuf_bytes + sz_bytes;
+  const uint32_t fixed = 1024 /*align*/ + kBarBytes + zbuf_bytes + sz_bytes;
   s.stages = static_cast<int>(
       std::min<uint32_t>(kMaxStages, (kSmemLimit - fixed) / s.stage_bytes));
   s.zbuf_off = static_cast<uint32_t>(s.stages) * s.stage_bytes;
   s.sz_off = s.zbuf_off + zbuf_bytes;
   s.bar_off = s.sz_off + sz_bytes;
-  s.smem_bytes = s.bar_off + 256 + 1024;
+  s.smem_bytes = s.bar_off + kBarBytes + 1024;
   return s;
 }
 
@@ -504,6 +544,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   a.stages = s.stages;
   a.stage_bytes = s.stage_bytes;
   a.b_off = s.b_off;
+  a.w_off = s.w_off;
   a.zbuf_off = s.zbuf_off;
   a.sz_off = s.sz_off;
   a.bar_off = s.bar_off;

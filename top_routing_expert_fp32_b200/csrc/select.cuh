@@ -74,83 +74,4 @@ __device__ __forceinline__ void select_token(float* z, int E, int k, int renorm,
     for (int e = 0; e < E; ++e) z[e] = expf(z[e] - zmax) / s_all;
 }
 
-// The same decision with the logits in registers (EB >= E, entries past E ignored): every
-// loop is unrolled, so nothing waits on shared memory. Sums run in the same order as
-// select_token, so both give the same bits for the same logits. probs (shared memory,
-// optional) receives the softmax the gates come from.
-template <int EB>
-__device__ __forceinline__ void select_token_regs(float (&z)[EB], int E, int k, int renorm,
-                                                  int mode, const float* noise, int32_t* idx,
-                                                  float* gate, float* probs, float* lse) {
-  if (lse != nullptr) {
-    float m = z[0];
-#pragma unroll
-    for (int e = 1; e < EB; ++e)
-      if (e < E) m = z[e] > m ? z[e] : m;
-    float s = 0.f;
-#pragma unroll
-    for (int e = 0; e < EB; ++e)
-      if (e < E) s += expf(z[e] - m);
-    *lse = m + logf(s);
-  }
-  float n[EB];
-#pragma unroll
-  for (int e = 0; e < EB; ++e) n[e] = (mode != MOE_ROUTE_TOPK && e < E) ? noise[e] : 0.f;
-  if (mode == MOE_ROUTE_NOISY_TOPK) {
-#pragma unroll
-    for (int e = 0; e < EB; ++e) z[e] = z[e] + n[e];
-  }
-  float zmax = z[0];
-#pragma unroll
-  for (int e = 1; e < EB; ++e)
-    if (e < E) zmax = z[e] > zmax ? z[e] : zmax;
-  uint64_t chosen = 0;
-  int sel[8];
-  float selz[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    sel[j] = 0;
-    selz[j] = 0.f;
-    if (j < k) {
-      const bool perturbed = mode == MOE_ROUTE_GSHARD_RANDOM && j > 0;
-      int best = -1;
-      float vb = 0.f;
-#pragma unroll
-      for (int e = 0; e < EB; ++e) {
-        const float v = perturbed ? z[e] + n[e] : z[e];
-        const bool take = e < E && !((chosen >> e) & 1ull) && (best < 0 || v > vb);
-        best = take ? e : best;  // strict: equal keeps the lower index
-        vb = take ? v : vb;
-      }
-      chosen |= 1ull << best;
-      sel[j] = best;
-      float zs = 0.f;  // the gate uses the (unperturbed, or mode-1 perturbed) z of the choice
-#pragma unroll
-      for (int e = 0; e < EB; ++e) zs = e == best ? z[e] : zs;
-      selz[j] = zs;
-    }
-  }
-  float s_all = 0.f;
-#pragma unroll
-  for (int e = 0; e < EB; ++e)
-    if (e < E) s_all += expf(z[e] - zmax);
-  float s_sel = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < k) s_sel += expf(selz[j] - zmax);
-  const float denom = renorm ? s_sel : s_all;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j < k) {
-      idx[j] = sel[j];
-      gate[j] = expf(selz[j] - zmax) / denom;
-    }
-  }
-  if (probs != nullptr) {
-#pragma unroll
-    for (int e = 0; e < EB; ++e)
-      if (e < E) probs[e] = expf(z[e] - zmax) / s_all;
-  }
-}
-
 }  // namespace moe
