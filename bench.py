@@ -373,27 +373,27 @@ def run_gpu(args, cfg, world, rank, device):
     launches = {"route": 1, "dispatch": 1, "up": 1, "down": 1, "combine": 1}
 
     def step(ev):
-        ev[0].record(stream)
+        ev[0].record()
         abi.route(p, inp.X, inp.W_r, inp.bias, logits, idx, gate, None, ws)
-        ev[1].record(stream)
+        ev[1].record()
         abi.dispatch(p, inp.X, idx, load, offsets, pos, dropped, row_token, X_perm, ws)
-        ev[2].record(stream)
+        ev[2].record()
         if packed:
             abi.expert_up_w8p(p, X_perm, offsets, wq.W1q, wq.S1, wq.W2q, wq.S2, H, ws)
         elif w8:
             abi.expert_up_w8(p, X_perm, offsets, wq.W1q, wq.S1, wq.W2q, wq.S2, H, ws)
         else:
             abi.expert_up(p, X_perm, offsets, inp.W1, inp.W2, H, ws)
-        ev[3].record(stream)
+        ev[3].record()
         if packed:
             abi.expert_down_w8p(p, H, offsets, wq.W3q, wq.S3, Y, ws)
         elif w8:
             abi.expert_down_w8(p, H, offsets, wq.W3q, wq.S3, Y, ws)
         else:
             abi.expert_down(p, H, offsets, inp.W3, Y, ws)
-        ev[4].record(stream)
+        ev[4].record()
         abi.combine(p, Y, idx, gate, offsets, pos, dropped, out)
-        ev[5].record(stream)
+        ev[5].record()
 
     def new_events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
@@ -412,20 +412,51 @@ def run_gpu(args, cfg, world, rank, device):
         want = max(20, min(20000, math.ceil(TIMED_REGION_TARGET_S / max(t_step, 1e-6))))
         args.steps = int(reduce_max(float(want), device))
 
+    # With --graph the step (its five stages and the events between them) is captured once
+    # into a CUDA graph and each timed step is one replay; the stage times are read after each
+    # replay (a host wait between steps, outside the events).
+    graph, graph_note = None, None
+    if args.graph:
+        try:
+            # external: recorded as event nodes of the graph, readable after each replay
+            gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+            graph = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize(device)
+            with torch.cuda.graph(graph):
+                step(gev)
+            for _ in range(2):
+                graph.replay()
+                flush_l2()
+            torch.cuda.synchronize(device)
+            if abi.device_error(ws) != 0:
+                raise RuntimeError("device error in the captured step")
+        except Exception as ex:  # capture unsupported here: time the steps as launched
+            graph, graph_note = None, f"capture failed: {ex}"[:200]
+            torch.cuda.synchronize(device)
+
     sampler = ClockSampler(device.index).start()
     barrier(device)
     torch.cuda.synchronize(device)
     t_wall0 = time.time()
     evs = []
-    for _ in range(args.steps):
-        ev = new_events()
-        step(ev)
-        evs.append(ev)
-        flush_l2()   # outside the step's events
+    if graph is not None:
+        for _ in range(args.steps):
+            graph.replay()
+            gev[5].synchronize()
+            evs.append([gev[i].elapsed_time(gev[i + 1]) for i in range(5)])
+            flush_l2()   # outside the step's events
+    else:
+        for _ in range(args.steps):
+            ev = new_events()
+            step(ev)
+            evs.append(ev)
+            flush_l2()   # outside the step's events
     torch.cuda.synchronize(device)
     barrier(device)
     t_wall1 = time.time()
     sampler.stop()
+    if graph is None:  # stage times from the events of each step
+        evs = [[ev[i].elapsed_time(ev[i + 1]) for i in range(5)] for ev in evs]
     if abi.device_error(ws) != 0:
         raise RuntimeError("device error during the timed steps")
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -435,8 +466,8 @@ def run_gpu(args, cfg, world, rank, device):
     # a short one; the other is reported beside it.
     sustained = clocks["timed_region_s"] >= 1.0 or "sw_power_cap" in clocks.get("reasons", [])
 
-    per = {n: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, n in enumerate(names)}
-    total_ms = sum(ev[0].elapsed_time(ev[5]) for ev in evs)
+    per = {n: [ev[i] for ev in evs] for i, n in enumerate(names)}
+    total_ms = sum(sum(ev) for ev in evs)
     max_total = reduce_max(total_ms, device)
     agg = aggregate(N, world, max_total, args.steps)
     mean = {n: sum(v) / len(v) for n, v in per.items()}
@@ -597,6 +628,8 @@ def run_gpu(args, cfg, world, rank, device):
                    else dtype_name(cfg),
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "flushed between steps (512 MiB write + read-back, outside the step events)",
+                   "launch": ("CUDA graph of the step, one replay per step" if graph is not None
+                              else "stream launches" + (f" ({graph_note})" if graph_note else "")),
                    "kept_records": kept,
                    "diagnostics": diagnostics,
                    "grouped_gemm_TFLOP/s": gemm_tflops,
@@ -816,6 +849,8 @@ def main():
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
                     help="replicas: one independent layer per GPU; ep: experts split over the "
                          "GPUs, rows exchanged by all-to-all (bf16 weights)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the step into a CUDA graph and time its replays")
     ap.add_argument("--all-workloads", action="store_true",
                     help="one line per workload (1 GPU), each with diagnostics, near-tie flips "
                          "against the oracle's routing and the oracle's CPU throughput")

@@ -256,10 +256,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* b = smem + stage * a.stage_bytes + a.b_off;
         const float* wf = reinterpret_cast<const float*>(smem + stage * a.stage_bytes + a.w_off);
         const int wrows = min(BK, a.D - kb * BK);
-        // kBatch items per thread at a time, all their loads first: independent chains for
-        // the scheduler (E = 64 gives each thread 4 items per k-block).
+        // Item (c, e) -> its three 16-byte chunks of B.
+        auto convert_store = [&](int i, const float (&wv)[8]) {
+          const int c = i / E, e = i - c * E;
+          float t0[8], t1[8], t2[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) split3(wv[j], t0[j], t1[j], t2[j]);
+          const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
+                                      pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
+          const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
+                                      pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
+          const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
+                                      pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
+          const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
+          *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
+          *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
+          *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
+        };
+        if (items <= kConvThreads) {  // E <= 16: at most one item per thread
+          if (ct < items) {
+            const int c = ct / E, e = ct - c * E;
+            float wv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int d = c * 8 + j;
+              wv[j] = d < wrows ? wf[d * E + e] : 0.f;
+            }
+            convert_store(ct, wv);
+          }
+        }
+        // Larger E: kBatch items per thread at a time, all their loads first (independent
+        // chains for the scheduler; E = 64 gives each thread 4 items per k-block).
         constexpr int kBatch = 4;
-        for (int i0 = ct; i0 < items; i0 += kBatch * kConvThreads) {
+        for (int i0 = items <= kConvThreads ? items : ct; i0 < items;
+             i0 += kBatch * kConvThreads) {
           float w[kBatch][8];
 #pragma unroll
           for (int u = 0; u < kBatch; ++u) {
@@ -275,20 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < kBatch; ++u) {
             const int i = i0 + u * kConvThreads;
             if (i >= items) break;
-            const int c = i / E, e = i - c * E;
-            float t0[8], t1[8], t2[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) split3(w[u][j], t0[j], t1[j], t2[j]);
-            const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
-                                        pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
-            const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
-                                        pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
-            const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
-                                        pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
-            const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
-            *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
-            *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
-            *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
+            convert_store(i, w[u]);
           }
         }
         fence_proxy_async_smem();  // generic-proxy stores before the MMA (async proxy) reads
