@@ -644,11 +644,12 @@ cudaError_t launch_dispatch_fused(const moe_problem& p, int64_t capacity, const 
   a.token_major = p.capacity_order == MOE_ORDER_TOKEN_MAJOR;
   a.row_words = static_cast<uint32_t>(static_cast<int64_t>(p.D) * elem / 16);
   a.timeout_ns = timeout_ns;
-  // With rows to copy, every resident block takes a slice (the copy is spread over the whole
-  // device); without, one block per 512 records. At least one block per chunk.
-  const int64_t want = X != nullptr ? max_blocks
-                                    : std::max<int64_t>(nchunks, (R + kFusedThreads - 1) /
-                                                                     kFusedThreads);
+  // With rows to copy, a block per 96 KB of rows up to every resident block (the copy spread
+  // over the device; small batches keep the grid barrier small); without, one block per 512
+  // records. At least one block per chunk.
+  const int64_t copy_bytes = R * static_cast<int64_t>(p.D) * elem;
+  const int64_t want = std::max<int64_t>(
+      nchunks, X != nullptr ? (copy_bytes + 98303) / 98304 : (R + kFusedThreads - 1) / kFusedThreads);
   // At most two blocks per SM (room for a kernel of another stream beside it); with more
   // chunks than blocks, blocks loop over chunks (still one launch).
   const int grid = static_cast<int>(
