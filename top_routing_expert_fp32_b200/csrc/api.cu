@@ -26,6 +26,24 @@ int num_sms() {
   return cache[dev];
 }
 
+// Off by default: measured on decode- and mixtral-shaped layers, launching each kernel as a
+// programmatic dependent of the previous one was slower (decode back-to-back 476 -> 505 us)
+// or no faster. MOE_PDL=1 turns it on.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* env = std::getenv("MOE_PDL");
+    return env != nullptr && std::strcmp(env, "1") == 0;
+  }();
+  return on;
+}
+
+int pdl_attr(cudaLaunchAttribute* attr) {
+  if (!pdl_enabled()) return 0;
+  attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr->val.programmaticStreamSerializationAllowed = 1;
+  return 1;
+}
+
 }  // namespace moe
 
 namespace {

@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t t = static_cast<int64_t>(blockIdx.x) * (kWarps / wpt) + warp / wpt;
   const int64_t first = 32 * (warp % wpt) + lane;  // this lane's first chunk
   const int64_t step = 32 * wpt;
+  pdl_wait();  // Y and the routing come from the previous kernels
+  pdl_trigger();
   if (t >= N) return;  // uniform over the warp
   int64_t my_row = -1;
   float my_g = 0.f;
@@ -168,15 +170,23 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
   const uint4* y = static_cast<const uint4*>(Y);
   uint4* o = static_cast<uint4*>(out);
   const bool rk = p.drop_policy == MOE_DROP_RENORM_KEPT && dropped != nullptr;
-#define MOE_COMBINE(T, KM)                                                                      \
-  do {                                                                                          \
-    if (wpt == 1)                                                                               \
-      combine_kernel<T, KM, 1><<<grid, kThreads, 0, stream>>>(y, idx, gate, offsets, pos,       \
-                                                              dropped, o, p.N, p.k, p.E, chunks, \
-                                                              rk, err);                         \
-    else                                                                                        \
-      combine_kernel<T, KM, kWarps><<<grid, kThreads, 0, stream>>>(                             \
-          y, idx, gate, offsets, pos, dropped, o, p.N, p.k, p.E, chunks, rk, err);              \
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_attr(&attr[0]);
+  cudaError_t e = cudaSuccess;
+#define MOE_COMBINE(T, KM)                                                                     \
+  do {                                                                                         \
+    if (wpt == 1)                                                                              \
+      e = cudaLaunchKernelEx(&cfg, combine_kernel<T, KM, 1>, y, idx, gate, offsets, pos,       \
+                             dropped, o, p.N, p.k, p.E, chunks, rk, err);                      \
+    else                                                                                       \
+      e = cudaLaunchKernelEx(&cfg, combine_kernel<T, KM, kWarps>, y, idx, gate, offsets, pos,  \
+                             dropped, o, p.N, p.k, p.E, chunks, rk, err);                      \
   } while (0)
   if (p.dtype == MOE_DTYPE_BF16) {
     if (p.k <= 1) MOE_COMBINE(__nv_bfloat16, 1);
@@ -190,7 +200,7 @@ cudaError_t launch_combine(const moe_problem& p, const void* Y, const int32_t* i
     else MOE_COMBINE(float, 8);
   }
 #undef MOE_COMBINE
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace moe

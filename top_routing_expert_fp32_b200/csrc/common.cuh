@@ -39,6 +39,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Programmatic dependent launch: the layer's kernels may be launched while the previous kernel
+// of the stream is still running. pdl_wait() blocks until every grid this one depends on has
+// completed and its memory writes are visible (a no-op for an ordinary launch); nothing before
+// it may read or write global memory the previous kernels touch. pdl_trigger() lets the next
+// kernel of the stream be scheduled once every block of this grid has issued it (that kernel
+// still waits for this grid's completion in its own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

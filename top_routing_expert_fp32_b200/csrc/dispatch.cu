@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(kFusedThreads) dispatch_fused_kernel(FusedArgs
   constexpr int kWarps = kFusedThreads / 32;
   const int G = static_cast<int>(gridDim.x);
   bool ok = true;
+  pdl_wait();  // idx (and X) come from the previous kernels
+  pdl_trigger();
 
   // Phase 1: per-chunk histograms.
   for (int c = blockIdx.x; c < a.nchunks; c += G) {
@@ -659,12 +661,17 @@ cudaError_t launch_dispatch_fused(const moe_problem& p, int64_t capacity, const 
   cfg.blockDim = dim3(kFusedThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1 + pdl_attr(&attr[1]);
   cudaError_t e = cudaLaunchKernelEx(&cfg, dispatch_fused_kernel, a);
+  if (e != cudaSuccess && cfg.numAttrs > 1) {  // no dependent launch with a cooperative one here
+    (void)cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dispatch_fused_kernel, a);
+  }
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -145,6 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool mma_cta = rank == 0;
   const int cta_unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  pdl_wait();  // offsets, the A rows and the tile counter come from the previous kernels
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -576,8 +578,16 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   if (e != cudaSuccess) return e;
   if (!PAIR) {
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_upper)));
-    kern<<<grid, kThreads, S::kSmemBytes, stream>>>(a, b0, b1, gp);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_attr(&attr[0]);
+    e = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, gp);
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   const int clusters = static_cast<int>(
       std::max<int64_t>(1, std::min<int64_t>(max_pair_clusters(kern, S::kSmemBytes), tiles_upper)));
@@ -586,13 +596,13 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = S::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1 + pdl_attr(&attr[1]);
   e = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, gp);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -143,6 +143,15 @@ cudaError_t launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_
 
 int num_sms();
 
+// Whether the layer's kernels are launched as programmatic dependents of the previous kernel
+// in the stream (cudaLaunchAttributeProgrammaticStreamSerialization; each kernel waits in
+// pdl_wait() before touching global memory). Off unless MOE_PDL=1 (read once per process).
+bool pdl_enabled();
+
+// Fills attr with the programmatic-dependent-launch attribute when enabled; returns the
+// number of attributes written (0 or 1).
+int pdl_attr(cudaLaunchAttribute* attr);
+
 // Message returned by moe_last_error() on the calling thread.
 void set_last_error(const std::string& msg);
 

@@ -142,6 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
   const uint32_t tx_bytes = static_cast<uint32_t>(kABytes);
+  pdl_wait();  // X, W_r and the outputs belong to the previous kernels until here
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------------ TMA producer
@@ -578,13 +580,13 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = s.smem_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(s.S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1 + pdl_attr(&attr[1]);
   e = cudaLaunchKernelEx(&cfg, kern, tX, a);
   if (e != cudaSuccess) return e;
   *grid_out = s.num_clusters * s.S;
