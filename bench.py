@@ -526,9 +526,9 @@ def run_gpu(args, cfg, world, rank, device):
                 "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                 "frac": gbs / hbm, "peak_source": psrc, "bytes_per_launch": bytes_up}
     roof["min_us"] = {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6}
-    roof["denominator"] = ("peak = the measured " + ("cuBLAS bf16 GEMM burst" if
+    roof["denominator"] = ("peak = the " + (f"cuBLAS {tc_kind} GEMM figure" if
                            roof["bound"] == "tensor" else "HBM copy bandwidth") +
-                           "; frac_datasheet uses the B200 datasheet figure")
+                           f" ({psrc}); frac_datasheet uses the B200 datasheet figure")
     roof["peak_datasheet"] = (DATASHEET_BF16_TFLOPS if roof["bound"] == "tensor"
                               else DATASHEET_HBM_GBS)
     roof["frac_datasheet"] = roof["achieved"] / roof["peak_datasheet"]
