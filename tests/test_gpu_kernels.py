@@ -290,6 +290,13 @@ def test_gather_exact(abi, oracle_lib, N, D, E, k, cf, dtype):
 
 # ------------------------------------------------------------------ grouped expert FFN
 
+def _tile_env(monkeypatch, tile_rows):
+    # "128": one CTA per 128-row tile; "256": CTA pairs (tcgen05 cta_group::2) sharing a
+    # 256-row tile; "256w": CTA pairs with two MMAs per k-step into one 512-column accumulator.
+    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows.rstrip("w"))
+    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if tile_rows.endswith("w") else "0")
+
+
 def _ffn_case(abi, oracle_lib, counts, D, F, act, dtype=configs.DTYPE_BF16, seed=0):
     E = len(counts)
     R = int(sum(counts))
@@ -329,10 +336,9 @@ def _ffn_case(abi, oracle_lib, counts, D, F, act, dtype=configs.DTYPE_BF16, seed
     ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
     ([700, 0, 257, 1100], 512, 768, configs.ACT_GELU_ERF),
 ])
-@pytest.mark.parametrize("tile_rows", ["128", "256"])
+@pytest.mark.parametrize("tile_rows", ["128", "256", "256w"])
 def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, monkeypatch, counts, D, F, act, tile_rows):
-    # 128: one CTA per tile; 256: CTA pairs (tcgen05 cta_group::2) sharing one tile.
-    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
+    _tile_env(monkeypatch, tile_rows)
     _ffn_case(abi, oracle_lib, counts, D, F, act)
 
 
@@ -341,10 +347,11 @@ def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, monkeypatch, counts, D, F, act
     ([700, 0, 257, 1100], 512, 768),
     ([3, 0, 200, 1, 64, 65, 0, 128, 7], 128, 1280),
 ])
-@pytest.mark.parametrize("tile_rows,ngroup", [("128", "2"), ("128", "4"), ("256", "3")])
+@pytest.mark.parametrize("tile_rows,ngroup", [("128", "2"), ("128", "4"), ("256", "3"),
+                                              ("256w", "2")])
 def test_expert_ffn_tile_groups(abi, oracle_lib, monkeypatch, counts, D, F, tile_rows, ngroup):
     # Tiles visited in groups of column blocks (a shorter last group included).
-    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
+    _tile_env(monkeypatch, tile_rows)
     monkeypatch.setenv("MOE_GEMM_NGROUP", ngroup)
     _ffn_case(abi, oracle_lib, counts, D, F, configs.ACT_SILU, seed=3)
 
@@ -354,7 +361,7 @@ def test_expert_ffn_tile_groups(abi, oracle_lib, monkeypatch, counts, D, F, tile
     ([129, 127, 128, 0, 5, 256, 1, 64], 256, 384),
     ([2000, 1500, 0, 2600], 256, 2048),               # many tiles per CTA
 ])
-@pytest.mark.parametrize("tile_rows", ["128", "256"])
+@pytest.mark.parametrize("tile_rows", ["128", "256", "256w"])
 @pytest.mark.parametrize("order", ["dynamic", "static"])
 def test_expert_ffn_tile_counter_returns_to_zero(abi, oracle_lib, monkeypatch, counts, D, F,
                                                  tile_rows, order):
@@ -362,7 +369,7 @@ def test_expert_ffn_tile_counter_returns_to_zero(abi, oracle_lib, monkeypatch, c
     # every launch returns it to zero, so back-to-back launches on one workspace give the same
     # bits and see every tile. The static round-robin order (MOE_GEMM_SCHED=static) gives the
     # same results.
-    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows)
+    _tile_env(monkeypatch, tile_rows)
     monkeypatch.setenv("MOE_GEMM_SCHED", order)
     E = len(counts)
     R = int(sum(counts))

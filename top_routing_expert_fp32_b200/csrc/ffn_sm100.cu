@@ -5,7 +5,7 @@
 // ch.12, 12.1 (f_e(x) = [SiLU(x W1_e) (.) (x W2_e)] W3_e); Grok-1 book ch.5, 5.3.5 (GeGLU
 // variant, x W_value times GELU(x W_gate)) and 5.3.2 (weights stacked [E, D, F] / [E, F, D]).
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   warp 0 lane 0 : TMA producer. Per k-block of 64: one 128x64 A box (X_perm or H rows,
 //                   K-major, 128-byte swizzle) and four 64x64 B boxes from the 3-D weight
 //                   tensor [E][K][N] (N contiguous = MN-major B, 128-byte swizzle). GEMM1 takes
@@ -13,10 +13,13 @@
 //                   N=256 MMA produces both up-projections side by side.
 //   warp 1        : allocates 512 TMEM columns (two 128x256 fp32 accumulators); lane 0 issues
 //                   tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32) and commits to barriers.
-//   warps 2..5    : epilogue. tcgen05.ld of the accumulator rows (one row per thread), act in
+//   warps 2..9    : epilogue, two warps per TMEM lane quarter taking alternate 32-column
+//                   chunks. tcgen05.ld of the accumulator rows (one row per thread), act in
 //                   fp32, bf16 rounding, masked 16-byte stores (rows past the expert's segment
 //                   are never written). The accumulator is double buffered, so the epilogue
 //                   of tile i overlaps the main loop of tile i+1.
+// CTA pairs (cta_group::2, M=256) split A by rows and B by columns between the two CTAs; wide
+// pairs issue two N=256 MMAs per k-step into one 512-column accumulator (not double-buffered).
 // Tiles: per expert ceil(M_e/128) row blocks x ceil(N/NT) column blocks. The column blocks
 // are cut into groups of G; tiles run group by group, inside a group expert by expert, then
 // column block, with row blocks innermost (consecutive CTAs share a weight column block
@@ -55,17 +58,24 @@ constexpr int kABytes = kRows * BK * 2;            // 16 KB
 constexpr int kBoxBytes = 64 * BK * 2;             // 8 KB: 64 columns x 64 k-rows
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;      // producer warp, MMA warp, epilogue
 constexpr int kMaxE = 64;
 constexpr int kRing = 4;                           // tile ids in flight between the roles
 
 // Per-variant shape: a single CTA computes 128-row tiles with the whole B; a CTA pair
-// computes 256-row tiles, each CTA holding its 128 A rows and half of the B columns.
-template <bool PAIR>
+// computes 256-row tiles, each CTA holding its 128 A rows and half of the B columns. A wide
+// pair issues two N=256 MMAs per k-step into one 512-column accumulator (all of TMEM, so the
+// accumulator is not double-buffered): each CTA then moves 48 KB per k-block for twice the
+// FLOPs of the 32 KB of a plain pair, 25 % fewer bytes from L2 per FLOP.
+template <bool PAIR, bool WIDE>
 struct Shape {
+  static_assert(PAIR || !WIDE, "wide tiles are CTA pairs");
   static constexpr int kTileRows = PAIR ? 256 : 128;
-  static constexpr int kBBoxes = PAIR ? 2 : 4;                       // 64-col B boxes per CTA
-  static constexpr int kStages = PAIR ? 7 : 4;  // fills the 227 KB of shared memory
+  static constexpr int kMmas = WIDE ? 2 : 1;                         // N=256 MMAs per k-step
+  static constexpr int kAccBufs = WIDE ? 1 : 2;                      // accumulators in TMEM
+  static constexpr int kBBoxes = PAIR ? 2 * kMmas : 4;               // 64-col B boxes per CTA
+  static constexpr int kStages = PAIR ? (WIDE ? 4 : 7) : 4;  // fills the 227 KB of shared memory
   static constexpr int kBBytes = kBBoxes * kBoxBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTxBytes = PAIR ? 2 * kStageBytes : kStageBytes;  // per stage, both CTAs
@@ -113,12 +123,12 @@ __device__ __forceinline__ void sched_finish(int* sched, int ctas) {
   }
 }
 
-template <bool DUAL, int ACT, bool PAIR>
+template <bool DUAL, int ACT, bool PAIR, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_sm100(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
-  using S = Shape<PAIR>;
+  using S = Shape<PAIR, WIDE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -136,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_mstart = const_cast<int*>(s_ring) + kRing;    // [E+1] first row block of expert e
   int* s_seg = s_mstart + (kMaxE + 1);                 // [E+1]
 
-  constexpr int NT = DUAL ? 128 : 256;  // output columns per tile
+  constexpr int NT = (DUAL ? 128 : 256) * S::kMmas;  // output columns per tile
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_blocks = (p.n_out + NT - 1) / NT;
@@ -177,13 +187,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
+      mbar_init(&tempty[a], (PAIR ? 2 : 1) * kEpiWarps);  // per epilogue warp (of both CTAs)
     }
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&ring_full[r], 1);
-      // consumers of a tile id: the MMA issuer and 4 epilogue warps, plus (pairs) the second
-      // CTA's producer and its 4 epilogue warps
-      mbar_init(&ring_empty[r], PAIR ? 10 : 5);
+      // consumers of a tile id: the MMA issuer and the epilogue warps, plus (pairs) the
+      // second CTA's producer and its epilogue warps
+      mbar_init(&ring_empty[r], PAIR ? 2 * (1 + kEpiWarps) : 1 + kEpiWarps);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -303,14 +313,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (mma_cta) mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
             tma_load_2d_pair_hint(a_dst, &tmA, bar, k0, row0, pol_a);
-            if (DUAL) {  // CTA 0 holds the W1 columns, CTA 1 the W2 columns
-              const CUtensorMap* m = rank == 0 ? &tmB0 : &tmB1;
-              tma_load_3d_pair_hint(b_dst, m, bar, n0, k0, e, pol_b);
-              tma_load_3d_pair_hint(b_dst + kBoxBytes, m, bar, n0 + 64, k0, e, pol_b);
-            } else {     // CTA r holds columns [n0 + 128r, n0 + 128r + 128)
-              const int nc = n0 + static_cast<int>(rank) * 128;
-              tma_load_3d_pair_hint(b_dst, &tmB0, bar, nc, k0, e, pol_b);
-              tma_load_3d_pair_hint(b_dst + kBoxBytes, &tmB0, bar, nc + 64, k0, e, pol_b);
+            // MMA h of the k-step reads boxes 2h, 2h+1 of each CTA.
+#pragma unroll
+            for (int h = 0; h < S::kMmas; ++h) {
+              uint8_t* bh = b_dst + 2 * h * kBoxBytes;
+              if (DUAL) {  // CTA 0 holds W1 columns [n0 + 128h, +128), CTA 1 the same of W2
+                const CUtensorMap* m = rank == 0 ? &tmB0 : &tmB1;
+                tma_load_3d_pair_hint(bh, m, bar, n0 + 128 * h, k0, e, pol_b);
+                tma_load_3d_pair_hint(bh + kBoxBytes, m, bar, n0 + 128 * h + 64, k0, e, pol_b);
+              } else {     // CTA r holds columns [n0 + 256h + 128r, +128)
+                const int nc = n0 + 256 * h + static_cast<int>(rank) * 128;
+                tma_load_3d_pair_hint(bh, &tmB0, bar, nc, k0, e, pol_b);
+                tma_load_3d_pair_hint(bh + kBoxBytes, &tmB0, bar, nc + 64, k0, e, pol_b);
+              }
             }
           } else {
             mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
@@ -348,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ring_release();
         ring_advance();
         if (tile >= total_tiles) break;
-        const int acc = it & 1;
-        const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
+        const int acc = it % S::kAccBufs;
+        const uint32_t acc_phase = static_cast<uint32_t>(it / S::kAccBufs) & 1u;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
           record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
           ok = false;
@@ -377,10 +392,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // A: K-major SW128, advance 16 elements = 32 bytes inside the swizzle row.
             const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
             // B: MN-major SW128, 64-column blocks kBoxBytes apart (LBO), 8-row k groups
-            // 1024 bytes apart (SBO); advance 16 k-rows = 2048 bytes.
-            const uint64_t bd = smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
-            if (PAIR) umma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-            else umma_bf16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            // 1024 bytes apart (SBO); advance 16 k-rows = 2048 bytes. MMA h (wide tiles)
+            // reads boxes 2h, 2h+1 into accumulator columns [256h, 256h + 256).
+#pragma unroll
+            for (int h = 0; h < S::kMmas; ++h) {
+              const uint64_t bd =
+                  smem_desc_sw128(b_addr + 2 * h * kBoxBytes + kk * 2048, kBoxBytes, 1024);
+              const uint32_t dh = d_tmem + static_cast<uint32_t>(256 * h);
+              if (PAIR) umma_bf16_ss_pair(dh, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              else umma_bf16_ss(dh, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           // frees the smem stage (of both CTAs) once these MMAs have read it
           if (PAIR) umma_commit_pair(&empty[stage], 0x3);
@@ -402,6 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {  // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // this warp may access TMEM lanes [32q, 32q+32)
+    // The two warps of a lane quarter take alternate 32-column chunks of the accumulator.
+    const int c_first = (warp - 2) / 4;
     const uint32_t tempty_mma0 = PAIR ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
     for (int it = 0;; ++it) {
       int tile = 0;
@@ -414,8 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ring_release();
       ring_advance();
       if (tile >= total_tiles) break;
-      const int acc = it & 1;
-      const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
+      const int acc = it % S::kAccBufs;
+      const uint32_t acc_phase = static_cast<uint32_t>(it / S::kAccBufs) & 1u;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, p.timeout_ns);
       if (__any_sync(0xffffffffu, !ok)) {
         if (lane == 0) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
@@ -436,13 +459,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       __nv_bfloat16* orow = p.out + grow * p.n_out + n0;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
+      // The accumulator is handed back to the MMA issuer as soon as this warp's last
+      // tcgen05.ld has completed; the last chunk's activation and stores follow.
+      auto release_acc = [&]() {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_cluster(tempty_mma0 + static_cast<uint32_t>(acc * 8));
+          else mbar_arrive(&tempty[acc]);
+        }
+      };
       if (DUAL) {
+        // Output columns [32c, 32c + 32) of the tile: x W1 in accumulator columns
+        // 256h + 32(c mod 4) and x W2 128 further, h = c / 4 (wide tiles have two halves).
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = c_first; c < 4 * S::kMmas; c += 2) {
           uint32_t ra[32], rb[32];
-          tmem_ld_32cols(t_row + c * 32, ra);        // x W1 (activated branch)
-          tmem_ld_32cols(t_row + 128 + c * 32, rb);  // x W2 (linear branch)
+          const uint32_t col = static_cast<uint32_t>(256 * (c >> 2) + 32 * (c & 3));
+          tmem_ld_32cols(t_row + col, ra);        // x W1 (activated branch)
+          tmem_ld_32cols(t_row + col + 128, rb);  // x W2 (linear branch)
           tmem_ld_wait();
+          if (c + 2 >= 4 * S::kMmas) release_acc();
           if (valid) {
             uint32_t w[16];
 #pragma unroll
@@ -459,12 +496,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           }
         }
-      } else {
+      } else {  // accumulator column j is output column n0 + j
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = c_first; c < 8 * S::kMmas; c += 2) {
           uint32_t ra[32];
           tmem_ld_32cols(t_row + c * 32, ra);
           tmem_ld_wait();
+          if (c + 2 >= 8 * S::kMmas) release_acc();
           if (valid) {
             uint32_t w[16];
 #pragma unroll
@@ -477,12 +515,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           }
         }
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) {  // this warp is done with the accumulator
-        if (PAIR) mbar_arrive_cluster(tempty_mma0 + static_cast<uint32_t>(acc * 8));
-        else mbar_arrive(&tempty[acc]);
       }
     }
   }
@@ -569,11 +601,11 @@ int max_pair_clusters(Kern kern, int smem) {
   return n;
 }
 
-template <bool DUAL, int ACT, bool PAIR>
+template <bool DUAL, int ACT, bool PAIR, bool WIDE>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const GemmParams& gp, int64_t tiles_upper, cudaStream_t stream) {
-  using S = Shape<PAIR>;
-  auto kern = grouped_gemm_sm100<DUAL, ACT, PAIR>;
+  using S = Shape<PAIR, WIDE>;
+  auto kern = grouped_gemm_sm100<DUAL, ACT, PAIR, WIDE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (!PAIR) {
@@ -661,21 +693,37 @@ void l2_priorities(int* a, int* b) {
   }
 }
 
+// CTA-pair tiles twice as wide (two MMAs into one 512-column accumulator, not double-buffered):
+// 25 % fewer bytes from L2 per FLOP against an epilogue that no longer overlaps the next
+// tile's main loop. Measured faster for both projections on the mixtral and grok1 shapes.
+// MOE_GEMM_WIDE=0|1 overrides (testing and tuning).
+bool use_wide() {
+  if (const char* env = std::getenv("MOE_GEMM_WIDE")) {
+    if (std::strcmp(env, "1") == 0) return true;
+    if (std::strcmp(env, "0") == 0) return false;
+  }
+  return true;
+}
+
 template <bool DUAL, int ACT>
 cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUtensorMap& b0,
                          const CUtensorMap& b1, GemmParams gp, int n_tile,
                          cudaStream_t stream) {
   const int64_t R = p.N * p.k;
+  const bool pairs = use_pairs(p);
+  const bool wide = pairs && use_wide();
+  if (wide) n_tile *= 2;
   const int64_t n_blocks = (gp.n_out + n_tile - 1) / n_tile;
-  gp.n_group = column_group(use_pairs(p), n_blocks);
+  gp.n_group = column_group(pairs, n_blocks);
   gp.static_order = static_order();
   l2_priorities(&gp.l2_a, &gp.l2_b);
-  if (use_pairs(p)) {
+  if (pairs) {
     const int64_t tiles = ((R + 255) / 256 + p.E) * n_blocks;
-    return launch_gemm<DUAL, ACT, true>(a, b0, b1, gp, tiles, stream);
+    if (wide) return launch_gemm<DUAL, ACT, true, true>(a, b0, b1, gp, tiles, stream);
+    return launch_gemm<DUAL, ACT, true, false>(a, b0, b1, gp, tiles, stream);
   }
   const int64_t tiles = ((R + 127) / 128 + p.E) * n_blocks;
-  return launch_gemm<DUAL, ACT, false>(a, b0, b1, gp, tiles, stream);
+  return launch_gemm<DUAL, ACT, false, false>(a, b0, b1, gp, tiles, stream);
 }
 
 }  // namespace
