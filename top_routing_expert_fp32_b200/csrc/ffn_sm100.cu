@@ -62,6 +62,7 @@ constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;      // producer warp, MMA warp, epilogue
 constexpr int kMaxE = 64;
 constexpr int kRing = 4;                           // tile ids in flight between the roles
+constexpr int kStoreStage = 32 * 64;               // per epilogue warp: 32 rows x 32 bf16
 
 // Per-variant shape: a single CTA computes 128-row tiles with the whole B; a CTA pair
 // computes 256-row tiles, each CTA holding its 128 A rows and half of the B columns. A wide
@@ -75,11 +76,13 @@ struct Shape {
   static constexpr int kMmas = WIDE ? 2 : 1;                         // N=256 MMAs per k-step
   static constexpr int kAccBufs = WIDE ? 1 : 2;                      // accumulators in TMEM
   static constexpr int kBBoxes = PAIR ? 2 * kMmas : 4;               // 64-col B boxes per CTA
-  static constexpr int kStages = PAIR ? (WIDE ? 4 : 7) : 4;  // fills the 227 KB of shared memory
+  static constexpr int kStages = PAIR ? (WIDE ? 4 : 6) : 4;  // fills the 227 KB of shared memory
   static constexpr int kBBytes = kBBoxes * kBoxBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTxBytes = PAIR ? 2 * kStageBytes : kStageBytes;  // per stage, both CTAs
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kStoreStage +
+                                    1024 /*align*/ + 1024 /*barriers*/;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   // Instruction descriptor, kind::f16: D fp32, A bf16, B bf16, A K-major, B MN-major,
   // N = 256, M = tile rows.
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
@@ -134,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + S::kStages * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::kStages * S::kBBytes);
+  uint8_t* sT = sB + S::kStages * S::kBBytes;  // [kEpiWarps][32 rows][64 B] store staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(sT + kEpiWarps * kStoreStage);
   uint64_t* empty = full + S::kStages;
   uint64_t* tfull = empty + S::kStages;
   uint64_t* tempty = tfull + 2;
@@ -450,13 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode(tile, e, m_blk, n_blk);
       const int first_row = m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
       const int rows = min(kRows, s_seg[e + 1] - s_seg[e] - first_row);
-      // Row held by this thread's TMEM lane (M = 64 tiles use lanes 0-15 of each quarter).
+      // Row held by TMEM lane 32q + l (M = 64 tiles use lanes 0-15 of each quarter).
       const bool half = !PAIR && rows <= 64;
-      const int r = half ? (lane < 16 ? 16 * q + lane : kRows) : q * 32 + lane;
-      const bool valid = r < rows;
-      const int64_t grow = static_cast<int64_t>(s_seg[e]) + first_row + r;
+      auto tile_row = [&](int l) { return half ? (l < 16 ? 16 * q + l : kRows) : q * 32 + l; };
+      const int64_t row0 = static_cast<int64_t>(s_seg[e]) + first_row;
       const int n0 = n_blk * NT;
-      __nv_bfloat16* orow = p.out + grow * p.n_out + n0;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       // The accumulator is handed back to the MMA issuer as soon as this warp's last
@@ -469,6 +471,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           else mbar_arrive(&tempty[acc]);
         }
       };
+      // Output columns [n0 + 32c, +32) of the warp's 32 rows: each lane holds its row's 64 bytes.
+      // They pass through the warp's 2 KB of shared memory so that each global store
+      // instruction writes 8 whole 64-byte row segments (4 lanes per row) instead of 32
+      // scattered 16-byte pieces. Segment v of row l sits in slot v ^ ((l >> 1) & 3), which
+      // keeps both the row-wise writes and the segment-wise reads free of bank conflicts.
+      uint8_t* stage = sT + (warp - 2) * kStoreStage;
+      auto store_chunk = [&](const uint32_t (&w)[16], int c) {
+        uint4* mine = reinterpret_cast<uint4*>(stage + lane * 64);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          mine[v ^ ((lane >> 1) & 3)] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        __syncwarp();
+        const int sg = lane & 3;
+        const int col = n0 + c * 32 + sg * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int l = 8 * i + (lane >> 2);
+          const uint4 val = reinterpret_cast<const uint4*>(stage + l * 64)[sg ^ ((l >> 1) & 3)];
+          const int r = tile_row(l);
+          if (r < rows && col < p.n_out)
+            *reinterpret_cast<uint4*>(p.out + (row0 + r) * p.n_out + col) = val;
+        }
+        __syncwarp();  // the next chunk overwrites the staging rows
+      };
       if (DUAL) {
         // Output columns [32c, 32c + 32) of the tile: x W1 in accumulator columns
         // 256h + 32(c mod 4) and x W2 128 further, h = c / 4 (wide tiles have two halves).
@@ -480,21 +506,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32cols(t_row + col + 128, rb);  // x W2 (linear branch)
           tmem_ld_wait();
           if (c + 2 >= 4 * S::kMmas) release_acc();
-          if (valid) {
-            uint32_t w[16];
+          uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = activation<ACT>(__uint_as_float(ra[2 * i])) * __uint_as_float(rb[2 * i]);
-              const float h1 =
-                  activation<ACT>(__uint_as_float(ra[2 * i + 1])) * __uint_as_float(rb[2 * i + 1]);
-              w[i] = pack_bf16x2(h0, h1);
-            }
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (n0 + c * 32 + v * 8 < p.n_out)
-                reinterpret_cast<uint4*>(orow + c * 32)[v] =
-                    make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          for (int i = 0; i < 16; ++i) {
+            const float h0 = activation<ACT>(__uint_as_float(ra[2 * i])) * __uint_as_float(rb[2 * i]);
+            const float h1 =
+                activation<ACT>(__uint_as_float(ra[2 * i + 1])) * __uint_as_float(rb[2 * i + 1]);
+            w[i] = pack_bf16x2(h0, h1);
           }
+          store_chunk(w, c);
         }
       } else {  // accumulator column j is output column n0 + j
 #pragma unroll 1
@@ -503,17 +523,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32cols(t_row + c * 32, ra);
           tmem_ld_wait();
           if (c + 2 >= 8 * S::kMmas) release_acc();
-          if (valid) {
-            uint32_t w[16];
+          uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w[i] = pack_bf16x2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (n0 + c * 32 + v * 8 < p.n_out)
-                reinterpret_cast<uint4*>(orow + c * 32)[v] =
-                    make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
+          store_chunk(w, c);
         }
       }
     }
