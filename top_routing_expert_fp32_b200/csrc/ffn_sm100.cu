@@ -495,39 +495,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();  // the next chunk overwrites the staging rows
       };
+      // The TMEM loads are software-pipelined: the next piece's tcgen05.ld is issued before
+      // this piece's math, so its latency hides behind the math (tcgen05.wait::ld waits for
+      // every load the thread has in flight, hence the two statically indexed buffers).
       if (DUAL) {
         // Output columns [32c, 32c + 32) of the tile: x W1 in accumulator columns
-        // 256h + 32(c mod 4) and x W2 128 further, h = c / 4 (wide tiles have two halves).
-#pragma unroll 1
-        for (int c = c_first; c < 4 * S::kMmas; c += 2) {
-          uint32_t ra[32], rb[32];
-          const uint32_t col = static_cast<uint32_t>(256 * (c >> 2) + 32 * (c & 3));
-          tmem_ld_32cols(t_row + col, ra);        // x W1 (activated branch)
-          tmem_ld_32cols(t_row + col + 128, rb);  // x W2 (linear branch)
-          tmem_ld_wait();
-          if (c + 2 >= 4 * S::kMmas) release_acc();
-          uint32_t w[16];
+        // 256h + 32(c mod 4) and x W2 128 further, h = c / 4 (wide tiles have two halves);
+        // each chunk is read as two 16-column pieces.
+        const int n_c = (4 * S::kMmas - c_first + 1) / 2;  // this warp's chunks
+        auto piece_col = [&](int cc, int half) {
+          const int c = c_first + 2 * cc;
+          return static_cast<uint32_t>(256 * (c >> 2) + 32 * (c & 3) + 16 * half);
+        };
+        auto act_pack = [&](const uint32_t (&ra)[16], const uint32_t (&rb)[16], uint32_t* w) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             const float h0 = activation<ACT>(__uint_as_float(ra[2 * i])) * __uint_as_float(rb[2 * i]);
             const float h1 =
                 activation<ACT>(__uint_as_float(ra[2 * i + 1])) * __uint_as_float(rb[2 * i + 1]);
             w[i] = pack_bf16x2(h0, h1);
           }
-          store_chunk(w, c);
+        };
+        uint32_t ra0[16], rb0[16], ra1[16], rb1[16];
+        tmem_ld_16cols(t_row + piece_col(0, 0), ra0);        // x W1 (activated branch)
+        tmem_ld_16cols(t_row + piece_col(0, 0) + 128, rb0);  // x W2 (linear branch)
+#pragma unroll 1
+        for (int cc = 0; cc < n_c; ++cc) {
+          uint32_t w[16];
+          tmem_ld_wait();
+          tmem_ld_16cols(t_row + piece_col(cc, 1), ra1);
+          tmem_ld_16cols(t_row + piece_col(cc, 1) + 128, rb1);
+          act_pack(ra0, rb0, w);
+          tmem_ld_wait();
+          if (cc + 1 < n_c) {
+            tmem_ld_16cols(t_row + piece_col(cc + 1, 0), ra0);
+            tmem_ld_16cols(t_row + piece_col(cc + 1, 0) + 128, rb0);
+          } else {
+            release_acc();
+          }
+          act_pack(ra1, rb1, w + 8);
+          store_chunk(w, c_first + 2 * cc);
         }
       } else {  // accumulator column j is output column n0 + j
-#pragma unroll 1
-        for (int c = c_first; c < 8 * S::kMmas; c += 2) {
-          uint32_t ra[32];
-          tmem_ld_32cols(t_row + c * 32, ra);
-          tmem_ld_wait();
-          if (c + 2 >= 8 * S::kMmas) release_acc();
-          uint32_t w[16];
+        const int n_c = (8 * S::kMmas - c_first + 1) / 2;  // this warp's chunks (even)
+        auto pack = [&](const uint32_t (&ra)[32], uint32_t (&w)[16]) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
-          store_chunk(w, c);
+        };
+        uint32_t ra0[32], ra1[32];
+        tmem_ld_32cols(t_row + c_first * 32, ra0);
+#pragma unroll 1
+        for (int cc = 0; cc < n_c; cc += 2) {
+          uint32_t w[16];
+          tmem_ld_wait();
+          tmem_ld_32cols(t_row + (c_first + 2 * (cc + 1)) * 32, ra1);
+          pack(ra0, w);
+          store_chunk(w, c_first + 2 * cc);
+          tmem_ld_wait();
+          if (cc + 2 < n_c) tmem_ld_32cols(t_row + (c_first + 2 * (cc + 2)) * 32, ra0);
+          else release_acc();
+          pack(ra1, w);
+          store_chunk(w, c_first + 2 * (cc + 1));
         }
       }
     }
