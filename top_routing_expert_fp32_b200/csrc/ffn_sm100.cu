@@ -443,7 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tile >= total_tiles) break;
       const int acc = it % S::kAccBufs;
       const uint32_t acc_phase = static_cast<uint32_t>(it / S::kAccBufs) & 1u;
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, p.timeout_ns);
+      // The accumulator is ready only after the tile's whole main loop: suspend rather than
+      // spin while the MMAs run (eight warps polling would take issue slots and power).
+      const bool ok = mbar_wait_suspend(&tfull[acc], acc_phase, p.timeout_ns);
       if (__any_sync(0xffffffffu, !ok)) {
         if (lane == 0) record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
         break;
