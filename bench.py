@@ -46,13 +46,34 @@ TIMED_REGION_TARGET_S = 1.5
 # ------------------------------------------------------------------ small host helpers
 
 def load_peaks():
+    """The roofline denominators: MEASURED_PEAKS.json's figures, each missing one taken from
+    the fallback table. Returns (peaks, source): "measured", "fallback", or "measured
+    (fallback: <keys>)" when the file lacks some of them."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+        if not isinstance(d, dict):
+            raise ValueError("not an object")
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+    peaks, missing = {}, []
+    for k, v in FALLBACK_PEAKS.items():
+        try:
+            peaks[k] = float(d[k])
+        except (KeyError, TypeError, ValueError):
+            peaks[k] = v
+            missing.append(k)
+    if len(missing) == len(FALLBACK_PEAKS):
+        return peaks, "fallback"
+    return peaks, "measured" if not missing else f"measured (fallback: {', '.join(missing)})"
+
+
+def peak_key_source(peak_src: str, key: str) -> str:
+    """Where one denominator came from, given load_peaks()'s source string."""
+    if peak_src == "fallback" or (peak_src.startswith("measured (fallback:") and key in peak_src):
+        return "fallback"
+    return "measured (MEASURED_PEAKS.json)"
 
 
 def workload_desc(cfg, w8: bool = False, packed: bool = False) -> str:
@@ -512,7 +533,9 @@ def run_gpu(args, cfg, world, rank, device):
     t_tensor = flops_up / (tc * 1e12) if cfg.dtype == configs.DTYPE_BF16 else 0.0
     t_hbm = bytes_up / (hbm * 1e9)
     dom = "up"
-    psrc = (f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback")
+    psrc = peak_key_source(peak_src, "bf16_tflops_sustained" if sustained else "bf16_tflops")
+    if t_tensor < t_hbm:
+        psrc = peak_key_source(peak_src, "hbm_gbs")
     if t_tensor >= t_hbm:
         roof = {"kernel": up_kernel + " (expert up-projection + gating)",
                 "bound": "tensor", "achieved": kern["up"]["TFLOP/s"], "peak": tc,
@@ -732,7 +755,8 @@ def run_gpu_ep(args, cfg, world, rank, device):
             "achieved": (flops / step_s / 1e12) if t_tc >= t_link else off_rank / step_s / 1e9,
             "peak": tc if t_tc >= t_link else 770.0,
             "unit": "TFLOP/s" if t_tc >= t_link else "GB/s",
-            "peak_source": (f"{peak_src} (MEASURED_PEAKS.json), bf16 burst" if t_tc >= t_link
+            "peak_source": (peak_key_source(peak_src, "bf16_tflops") + ", bf16 burst"
+                            if t_tc >= t_link
                             else "measured 8-GPU peer copy per direction (pool figure)"),
             "traffic": None}
     roof["frac"] = roof["achieved"] / roof["peak"]

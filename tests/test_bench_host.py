@@ -20,6 +20,16 @@ def test_peaks_measured_or_fallback(tmp_path, monkeypatch):
     assert src == "measured" and peaks["hbm_gbs"] == 6508.8 and peaks["bf16_tflops"] == 1624.0
     (tmp_path / "MEASURED_PEAKS.json").write_text("{not json")
     assert bench.load_peaks()[1] == "fallback"
+    # a file without the sustained figure: the measured ones kept, the missing one named
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6400.0,
+                                                              "bf16_tflops": 1600.0}))
+    peaks, src = bench.load_peaks()
+    assert peaks["hbm_gbs"] == 6400.0 and peaks["bf16_tflops"] == 1600.0
+    assert peaks["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert src == "measured (fallback: bf16_tflops_sustained)"
+    assert bench.peak_key_source(src, "bf16_tflops_sustained") == "fallback"
+    assert bench.peak_key_source(src, "hbm_gbs").startswith("measured")
+    assert bench.peak_key_source("fallback", "hbm_gbs") == "fallback"
 
 
 def test_traffic_used_only_while_the_kernel_sources_are_unchanged(tmp_path, monkeypatch):
