@@ -40,6 +40,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 DATASHEET_BF16_TFLOPS = 2250.0
 DATASHEET_HBM_GBS = 8000.0
 DATASHEET_SM_MHZ = 1965.0
+DATASHEET_SMS = 148
 TIMED_REGION_TARGET_S = 1.5
 
 
@@ -516,6 +517,15 @@ def run_gpu(args, cfg, world, rank, device):
     for n in ("route", "combine"):
         kern[n]["frac_hbm"] = kern[n]["GB/s"] / hbm
         kern[n]["frac_8TBs"] = kern[n]["GB/s"] / DATASHEET_HBM_GBS
+    # The router's other ceiling: the 2 N D E multiply-adds of fp32 logits on the fp32 FMA
+    # units (148 SMs x 128 lanes x 2 FLOP per clock at the datasheet clock). At E = 64 it is
+    # longer than the HBM time, so no fp32 SIMT router reaches the HBM target there; this
+    # router runs the contraction on the tensor cores (three bf16 terms of W_r).
+    ffma_floor_s = 2.0 * N * D * E / (DATASHEET_SMS * 128 * 2 * DATASHEET_SM_MHZ * 1e6)
+    kern["route"]["fp32_ffma_floor_us"] = ffma_floor_s * 1e6
+    kern["route"]["hbm_floor_us"] = bytes_route / (hbm * 1e9) * 1e6
+    kern["route"]["time_over_larger_floor"] = (max(ffma_floor_s, bytes_route / (hbm * 1e9))
+                                               / (mean["route"] / 1e3))
     for n in ("up", "down"):
         kern[n]["frac_bf16_peak"] = kern[n]["TFLOP/s"] / tc
         kern[n]["frac_bf16_burst"] = kern[n]["TFLOP/s"] / tc_burst
