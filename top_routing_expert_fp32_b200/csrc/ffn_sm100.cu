@@ -380,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tile >= total_tiles) break;
         const int acc = it % S::kAccBufs;
         const uint32_t acc_phase = static_cast<uint32_t>(it / S::kAccBufs) & 1u;
+        // Wide tiles: tempty[0] / tempty[1] free the lower / upper 256 accumulator columns.
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
           record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
           ok = false;
@@ -393,24 +394,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           decode(tile, e, m_blk, n_blk);
           if (s_seg[e + 1] - s_seg[e] - m_blk * kRows <= 64) idesc = S::kIdesc64;
         }
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
-            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * S::kBBytes);
+        // The MMAs of k-block kb (MMA h writes accumulator columns [256h, 256h + 256)).
+        auto issue = [&](int kb, int st, int h_lo, int h_hi) {
+          const uint32_t a_addr = smem_u32(sA + st * kABytes);
+          const uint32_t b_addr = smem_u32(sB + st * S::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
             // A: K-major SW128, advance 16 elements = 32 bytes inside the swizzle row.
             const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
             // B: MN-major SW128, 64-column blocks kBoxBytes apart (LBO), 8-row k groups
             // 1024 bytes apart (SBO); advance 16 k-rows = 2048 bytes. MMA h (wide tiles)
-            // reads boxes 2h, 2h+1 into accumulator columns [256h, 256h + 256).
-#pragma unroll
-            for (int h = 0; h < S::kMmas; ++h) {
+            // reads boxes 2h, 2h+1.
+            for (int h = h_lo; h < h_hi; ++h) {
               const uint64_t bd =
                   smem_desc_sw128(b_addr + 2 * h * kBoxBytes + kk * 2048, kBoxBytes, 1024);
               const uint32_t dh = d_tmem + static_cast<uint32_t>(256 * h);
@@ -418,9 +413,56 @@ __global__ void __launch_bounds__(kThreads, 1)
               else umma_bf16_ss(dh, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
           }
-          // frees the smem stage (of both CTAs) once these MMAs have read it
-          if (PAIR) umma_commit_pair(&empty[stage], 0x3);
-          else umma_commit(&empty[stage]);
+        };
+        auto free_stage = [&](int st) {  // once these MMAs have read it (both CTAs)
+          if (PAIR) umma_commit_pair(&empty[st], 0x3);
+          else umma_commit(&empty[st]);
+        };
+        int kb = 0;
+        if (WIDE) {
+          // The epilogue hands back the lower half of the accumulator before the upper one.
+          // Meanwhile the lower-half MMAs of the first k-blocks already in the ring run; their
+          // stages are freed once the upper-half MMAs have read them too.
+          const int pre = min(num_kb, S::kStages);
+          int st = stage;
+          uint32_t ph = phase;
+          for (int j = 0; j < pre; ++j) {
+            if (!mbar_wait(&full[st], ph, p.timeout_ns)) {
+              record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            issue(j, st, 0, 1);
+            if (++st == S::kStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+          }
+          if (ok && !mbar_wait(&tempty[1], acc_phase ^ 1u, p.timeout_ns)) {
+            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+            ok = false;
+          }
+          if (!ok) break;
+          tc_fence_after_sync();
+          for (; kb < pre; ++kb) {
+            issue(kb, stage, 1, 2);
+            free_stage(stage);
+            if (++stage == S::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        for (; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
+            record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          issue(kb, stage, 0, S::kMmas);
+          free_stage(stage);
           if (++stage == S::kStages) {
             stage = 0;
             phase ^= 1u;
@@ -475,13 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       // The accumulator is handed back to the MMA issuer as soon as this warp's last
-      // tcgen05.ld has completed; the last chunk's activation and stores follow.
-      auto release_acc = [&]() {
+      // tcgen05.ld from it has completed; the last chunk's activation and stores follow. Wide
+      // tiles hand back their lower 256 columns (barrier tempty[0]) once the warp's loads from
+      // them are done, and the upper ones (tempty[1]) after its last load.
+      auto release_acc = [&](int part) {
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) {
-          if (PAIR) mbar_arrive_cluster(tempty_mma0 + static_cast<uint32_t>(acc * 8));
-          else mbar_arrive(&tempty[acc]);
+          if (PAIR) mbar_arrive_cluster(tempty_mma0 + static_cast<uint32_t>((acc + part) * 8));
+          else mbar_arrive(&tempty[acc + part]);
         }
       };
       // Output columns [n0 + 32c, +32) of the warp's 32 rows: each lane holds its row's 64 bytes.
@@ -540,11 +584,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_16cols(t_row + piece_col(cc, 1) + 128, rb1);
           act_pack(ra0, rb0, w);
           tmem_ld_wait();
+          if (WIDE && 2 * (cc + 1) == n_c) release_acc(0);  // the last chunk of the lower half
           if (cc + 1 < n_c) {
             tmem_ld_16cols(t_row + piece_col(cc + 1, 0), ra0);
             tmem_ld_16cols(t_row + piece_col(cc + 1, 0) + 128, rb0);
           } else {
-            release_acc();
+            release_acc(WIDE ? 1 : 0);
           }
           act_pack(ra1, rb1, w + 8);
           store_chunk(w, c_first + 2 * cc);
@@ -566,8 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pack(ra0, w);
           store_chunk(w, c_first + 2 * cc);
           tmem_ld_wait();
+          if (WIDE && 2 * (cc + 2) == n_c) release_acc(0);  // the last chunk of the lower half
           if (cc + 2 < n_c) tmem_ld_32cols(t_row + (c_first + 2 * (cc + 2)) * 32, ra0);
-          else release_acc();
+          else release_acc(WIDE ? 1 : 0);
           pack(ra1, w);
           store_chunk(w, c_first + 2 * (cc + 1));
         }
