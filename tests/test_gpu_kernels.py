@@ -409,6 +409,77 @@ def test_expert_ffn_f32(abi, oracle_lib):
     assert err.max() <= 1e-5
 
 
+def _act64(x, act):
+    """The activations in float64 (LLMs-from-scratch 12.1; Grok-1 book 5.3.5)."""
+    if act == configs.ACT_SILU:
+        return x / (1.0 + np.exp(-x))
+    if act == configs.ACT_GELU_ERF:
+        return x * 0.5 * np.array([math.erfc(-v / math.sqrt(2.0)) for v in x])
+    u = math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)
+    return x / (1.0 + np.exp(-2.0 * u))      # = x (1 + tanh u) / 2, which cancels in float64 too
+
+
+def _bf16_grid(limit):
+    # every finite bf16 value with 2^-20 <= |v| <= limit, and zero
+    bits = np.arange(0, 1 << 16, dtype=np.uint32)
+    bits = bits[(bits & 0x7F80) != 0x7F80]          # no inf / NaN patterns
+    v = (bits << 16).view(np.float32).astype(np.float64)
+    v = v[(np.abs(v) <= limit) & ((np.abs(v) >= 2.0 ** -20) | (v == 0))]
+    return np.unique(v)
+
+
+@pytest.mark.parametrize("dtype", [configs.DTYPE_F32, configs.DTYPE_BF16])
+@pytest.mark.parametrize("act", [configs.ACT_SILU, configs.ACT_GELU_ERF, configs.ACT_GELU_TANH])
+def test_activation_values_through_the_up_projection(abi, dtype, act):
+    # H = act(x W1) (.) (x W2) with x_r = e_r, W1[r, f] = the value to test and W2 = 1: every
+    # pre-activation reaches the epilogue exactly (one exact product, the rest zeros), so H is
+    # the kernel's activation of a chosen value, checked against float64 over [-14, 14] on
+    # every value of magnitude >= 1e-30: relative error within 1e-6 (4 + x^2) (the activations'
+    # relative condition number grows like x^2 in the negative tail, so each fp32 rounding
+    # inside, of x^2 or of the tanh argument, costs up to about x^2 2^-24 there), plus half a
+    # bf16 ulp on the bf16 tensor-core path. The negative tails included: there the forms
+    # 1 + erf(x / sqrt 2) and 1 + tanh(u) cancel to zero in fp32.
+    D = 64
+    if dtype == configs.DTYPE_F32:
+        vals = np.unique(np.concatenate([np.linspace(-14.0, 14.0, 64 * 4096 - 200),
+                                         -np.logspace(-20, 1, 100), np.logspace(-20, 1, 100)])
+                         .astype(np.float32)).astype(np.float64)
+    else:
+        vals = _bf16_grid(14.0)
+    F = -(-len(vals) // (D * 64)) * 64
+    grid = np.zeros(D * F)
+    grid[:len(vals)] = vals
+    grid = grid.reshape(D, F)
+    cfg = _cfg(D, D, F, 1, 1, dtype=dtype, act=act)
+    tdt = inputs.torch_dtype(dtype)
+    Xp = torch.eye(D, dtype=torch.float32, device="cuda").to(tdt)
+    W1 = torch.tensor(grid, dtype=torch.float32, device="cuda").to(tdt).reshape(1, D, F)
+    W2 = torch.ones((1, D, F), dtype=tdt, device="cuda")
+    assert np.array_equal(W1.float().cpu().numpy().reshape(D, F), grid)   # exactly representable
+    offsets = torch.tensor([0, D], dtype=torch.int32, device="cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    H = torch.full((D, F), float("nan"), dtype=tdt, device="cuda")
+    abi.expert_up(p, Xp, offsets, W1, W2, H, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    x = grid.ravel()
+    got = H.double().cpu().numpy().ravel()
+    ref = _act64(x, act)
+    assert np.isfinite(got).all()
+    sel = np.abs(ref) >= 1e-30
+    rel = 1e-6 * (4.0 + x * x)
+    if dtype == configs.DTYPE_F32:
+        bound = rel * np.abs(ref)
+    else:
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-300))) - 7)
+        bound = 0.5 * ulp + rel * np.abs(ref)
+    bad = sel & (np.abs(got - ref) > bound)
+    assert not bad.any(), (f"{bad.sum()} values off, first x={x[bad][:5]} "
+                           f"got={got[bad][:5]} ref={ref[bad][:5]}")
+    assert (np.abs(got[~sel] - ref[~sel]) <= 1e-6 * np.maximum(1.0, np.abs(x[~sel]))).all()
+
+
 def test_expert_ffn_empty(abi, oracle_lib):
     _ffn_case(abi, oracle_lib, [0, 0, 0], 64, 128, configs.ACT_SILU)
 

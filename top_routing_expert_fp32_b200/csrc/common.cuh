@@ -354,6 +354,42 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 // ------------------------------------------------------------------ activations
 
+// Exact (erf) GELU, x * Phi(x) with Phi(x) = erfc(-x / sqrt 2) / 2 (Grok-1 book 5.3.5).
+// The upper tail q = erfc(|x| / sqrt 2) / 2 is evaluated directly and Phi = q for x < 0,
+// 1 - q otherwise, so the negative tail keeps its relative accuracy (the form
+// 0.5 x (1 + erf(x / sqrt 2)) cancels there: zero below x = -5.7 in fp32). With
+// t = 1 / (1 + |x| / (2 sqrt 2)), erfc(z) = t exp(-z^2 + p(t)) (the form of Press et al.,
+// Numerical Recipes 6.2, "erfcc"), here in base 2 with the halving folded into P:
+//   q = t * 2^(P(t) - x^2 log2(e) / 2),   P = log2(e) p - 1, a degree-9 polynomial in t.
+// P's coefficients are a least-squares Chebyshev fit made by gelu_coeffs.py in this
+// directory. Relative error of the result against float64: 5e-7 for |x| < 1, 1.5e-6 for
+// -5 < x < -1, 7.6e-6 in the far negative tail (the rounding of x^2 log2(e) / 2). One
+// approximate reciprocal and one approximate exponential (both MUFU), 9 FMAs for P: about
+// half the issue cycles of the erff form.
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+__device__ __forceinline__ float ex2_approx(float v) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+__device__ __forceinline__ float gelu_erf(float x) {
+  constexpr float kP[10] = {-2.82574821f,  1.44272923f,  0.539700627f, 0.139630064f,
+                            -0.268756866f, 0.402321607f, -1.63775313f, 2.14747453f,
+                            -1.18611491f,  0.246517316f};  // P(t) = sum kP[i] t^i
+  const float t = rcp_approx(fmaf(fabsf(x), 0.353553390593273762f, 1.0f));
+  float P = kP[9];
+#pragma unroll
+  for (int i = 8; i >= 0; --i) P = fmaf(P, t, kP[i]);
+  const float q = t * ex2_approx(fmaf(x * x, -0.721347520444481703f, P));
+  return x * (x < 0.0f ? q : 1.0f - q);
+}
+
 // act(a) applied to the first up-projection (LLMs-from-scratch 12.1; Grok-1 book 5.3.5).
 template <int ACT>
 __device__ __forceinline__ float activation(float a) {
@@ -362,10 +398,12 @@ __device__ __forceinline__ float activation(float a) {
     // the largest cost of the GEMM epilogue. For a -> -inf it gives -0, as a / inf does.
     return __fdividef(a, 1.0f + expf(-a));
   } else if constexpr (ACT == MOE_ACT_GELU_ERF) {
-    return 0.5f * a * (1.0f + erff(a * 0.70710678118654752440f));
+    return gelu_erf(a);
   } else {
+    // 0.5 a (1 + tanh u) = a / (1 + exp(-2u)): the same value without the cancellation of
+    // 1 + tanh u in the negative tail, and without tanhf.
     const float u = 0.79788456080286535588f * (a + 0.044715f * a * a * a);
-    return 0.5f * a * (1.0f + tanhf(u));
+    return __fdividef(a, 1.0f + expf(-2.0f * u));
   }
 }
 
