@@ -292,9 +292,13 @@ def test_gather_exact(abi, oracle_lib, N, D, E, k, cf, dtype):
 
 def _tile_env(monkeypatch, tile_rows):
     # "128": one CTA per 128-row tile; "256": CTA pairs (tcgen05 cta_group::2) sharing a
-    # 256-row tile; "256w": CTA pairs with two MMAs per k-step into one 512-column accumulator.
-    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows.rstrip("w"))
-    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if tile_rows.endswith("w") else "0")
+    # 256-row tile; "256w": CTA pairs with two MMAs per k-step into one 512-column accumulator,
+    # the tiles of a short last round split into half tiles (one MMA each; with fewer tiles
+    # than half the pairs, as in most cases here, every tile); "256wf": the same with whole
+    # tiles only.
+    monkeypatch.setenv("MOE_GEMM_TILE_ROWS", tile_rows[:3])
+    monkeypatch.setenv("MOE_GEMM_WIDE", "1" if "w" in tile_rows else "0")
+    monkeypatch.setenv("MOE_GEMM_HALVES", "0" if tile_rows.endswith("wf") else "1")
 
 
 def _ffn_case(abi, oracle_lib, counts, D, F, act, dtype=configs.DTYPE_BF16, seed=0):
@@ -336,7 +340,7 @@ def _ffn_case(abi, oracle_lib, counts, D, F, act, dtype=configs.DTYPE_BF16, seed
     ([16, 17, 15, 16, 16, 16, 16, 16], 4096, 1024, configs.ACT_SILU),
     ([700, 0, 257, 1100], 512, 768, configs.ACT_GELU_ERF),
 ])
-@pytest.mark.parametrize("tile_rows", ["128", "256", "256w"])
+@pytest.mark.parametrize("tile_rows", ["128", "256", "256w", "256wf"])
 def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, monkeypatch, counts, D, F, act, tile_rows):
     _tile_env(monkeypatch, tile_rows)
     _ffn_case(abi, oracle_lib, counts, D, F, act)
@@ -348,7 +352,7 @@ def test_expert_ffn_bf16_tcgen05(abi, oracle_lib, monkeypatch, counts, D, F, act
     ([3, 0, 200, 1, 64, 65, 0, 128, 7], 128, 1280),
 ])
 @pytest.mark.parametrize("tile_rows,ngroup", [("128", "2"), ("128", "4"), ("256", "3"),
-                                              ("256w", "2")])
+                                              ("256w", "2"), ("256wf", "2")])
 def test_expert_ffn_tile_groups(abi, oracle_lib, monkeypatch, counts, D, F, tile_rows, ngroup):
     # Tiles visited in groups of column blocks (a shorter last group included).
     _tile_env(monkeypatch, tile_rows)
@@ -361,7 +365,7 @@ def test_expert_ffn_tile_groups(abi, oracle_lib, monkeypatch, counts, D, F, tile
     ([129, 127, 128, 0, 5, 256, 1, 64], 256, 384),
     ([2000, 1500, 0, 2600], 256, 2048),               # many tiles per CTA
 ])
-@pytest.mark.parametrize("tile_rows", ["128", "256", "256w"])
+@pytest.mark.parametrize("tile_rows", ["128", "256", "256w", "256wf"])
 @pytest.mark.parametrize("order", ["dynamic", "static"])
 def test_expert_ffn_tile_counter_returns_to_zero(abi, oracle_lib, monkeypatch, counts, D, F,
                                                  tile_rows, order):
@@ -400,6 +404,53 @@ def test_expert_ffn_tile_counter_returns_to_zero(abi, oracle_lib, monkeypatch, c
     ref = oracle_lib.expert_ffn(sel.astype(np.int32), rec_e, np_host(Xp), np_host(W1),
                                 np_host(W2), np_host(W3), oracle.BF16, configs.ACT_SILU)
     err = normwise_rel_err(to_f64(outs[0][1][sel]), ref)
+    assert err.max() <= TOL_BF16, f"max normwise rel err {err.max():.3g}"
+
+
+@pytest.mark.parametrize("halves", ["0", "1", "all"])
+@pytest.mark.parametrize("counts,D,F", [
+    # up: 25 row blocks x 7 column blocks = 175 tiles; down: 25 x 3 = 75. On 74 pairs both
+    # leave a last round of 27 and 1 tiles, which the default splits (whole and half tiles in
+    # one launch).
+    ([2000, 1500, 0, 2600], 1536, 1792),
+    ([300, 0, 513, 40, 1], 1024, 1280),
+])
+def test_expert_ffn_half_tiles(abi, oracle_lib, monkeypatch, halves, counts, D, F):
+    # Wide tiles split into two half-width tiles (one N=256 MMA, half the output columns):
+    # never, for a short last round (default), or all of them. Same bits in every mode (the
+    # MMAs of an output column are the same), and the oracle on sampled rows.
+    _tile_env(monkeypatch, "256w")
+    monkeypatch.setenv("MOE_GEMM_HALVES", halves)
+    E = len(counts)
+    R = int(sum(counts))
+    cfg = _cfg(R, D, F, E, 1, act=configs.ACT_GELU_ERF)
+    Xp = inputs.randn((R, D), 1.0, torch.bfloat16, "cuda", 11, 1)
+    W1 = inputs.randn((E, D, F), 1 / math.sqrt(D), torch.bfloat16, "cuda", 11, 3)
+    W2 = inputs.randn((E, D, F), 1 / math.sqrt(D), torch.bfloat16, "cuda", 11, 4)
+    W3 = inputs.randn((E, F, D), 1 / math.sqrt(F), torch.bfloat16, "cuda", 11, 5)
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32,
+                           device="cuda")
+    p = abi.problem(cfg)
+    ws = abi.workspace(p)
+    H = torch.full((R, F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Y = torch.full((R, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    abi.expert_ffn(p, Xp, offsets, W1, W2, W3, H, Y, ws)
+    torch.cuda.synchronize()
+    assert abi.device_error(ws) == 0
+    assert not torch.isnan(H.float()).any() and not torch.isnan(Y.float()).any()
+    monkeypatch.setenv("MOE_GEMM_HALVES", "0")
+    H0 = torch.empty_like(H)
+    Y0 = torch.empty_like(Y)
+    abi.expert_ffn(p, Xp, offsets, W1, W2, W3, H0, Y0, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(H.view(torch.int16), H0.view(torch.int16))
+    assert torch.equal(Y.view(torch.int16), Y0.view(torch.int16))
+    sel = np.unique(np.concatenate([np.arange(0, R, max(1, R // 40)), np.cumsum(counts) - 1,
+                                    [R - 1]]))
+    rec_e = np.repeat(np.arange(E, dtype=np.int32), counts)[sel]
+    ref = oracle_lib.expert_ffn(sel.astype(np.int32), rec_e, np_host(Xp), np_host(W1),
+                                np_host(W2), np_host(W3), oracle.BF16, configs.ACT_GELU_ERF)
+    err = normwise_rel_err(to_f64(Y[sel]), ref)
     assert err.max() <= TOL_BF16, f"max normwise rel err {err.max():.3g}"
 
 

@@ -109,6 +109,7 @@ struct GemmParams {
   int* err;
   int* sched;              // [2]: next tile to hand out, CTAs (or pairs) finished; zero at rest
   int static_order;        // 1: CTA (pair) u takes tiles u, u + units, ... (no counter)
+  int halves;              // wide tiles split in two: 0 never, 1 a short last round, 2 all
   uint64_t timeout_ns;
 };
 
@@ -179,9 +180,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_tiles = m_total * n_blocks;
   const int group = min(max(p.n_group, 1), n_blocks);
   const int group_tiles = m_total * group;
-  // More CTAs (pairs) than tiles: the surplus ones take no tile; they only count themselves
+  // Wide tiles of a last round that would keep at most half of the pairs busy are split
+  // into two half tiles (one N=256 MMA each, NT/2 output columns), so that the round takes
+  // half a tile's time: ids [0, first_half) are whole tiles in the order below, id
+  // first_half + 2j + h is half h of tile first_half + j.
+  int split = 0;
+  if (WIDE) {
+    if (p.halves == 2) {
+      split = total_tiles;
+    } else if (p.halves == 1) {
+      const int r = total_tiles % units;
+      if (2 * r <= units) split = r;
+    }
+  }
+  const int first_half = total_tiles - split;
+  const int work = total_tiles + split;  // tile ids handed out
+  // More CTAs (pairs) than tile ids: the surplus ones take none; they only count themselves
   // finished. Uniform over the block and over the pair.
-  if (cta_unit >= total_tiles) {
+  if (cta_unit >= work) {
     if (threadIdx.x == 0 && mma_cta) sched_finish(p.sched, units);
     return;
   }
@@ -237,6 +253,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     m_blk = local - n_in * m_tiles;
     n_blk = c * group + n_in;
   };
+  // Tile id -> its tile and the first output column; *mmas = N=256 MMAs per k-step.
+  auto decode_id = [&](int id, int& e, int& m_blk, int& n0, int& mmas) {
+    int base = id, h = -1;
+    if (WIDE && id >= first_half) {
+      base = first_half + ((id - first_half) >> 1);
+      h = (id - first_half) & 1;
+    }
+    int n_blk;
+    decode(base, e, m_blk, n_blk);
+    n0 = n_blk * NT + (h > 0 ? NT / 2 : 0);
+    mmas = h >= 0 ? 1 : S::kMmas;
+  };
 
   // Next tile id from the ring (consumers). The second CTA of a pair receives the ids from
   // the first CTA (remote store + release.cluster arrival), so it waits with cluster scope
@@ -290,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&ring_full[r_slot]);
           if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&ring_full[r_slot]), 1));
           ring_advance();
-          if (tile >= total_tiles) break;
+          if (tile >= work) break;
           if (p.static_order) next = tile + units;
         } else {
           if (!ring_take(tile)) {
@@ -299,12 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ring_release();
           ring_advance();
-          if (tile >= total_tiles) break;
+          if (tile >= work) break;
         }
-        int e, m_blk, n_blk;
-        decode(tile, e, m_blk, n_blk);
+        int e, m_blk, n0, mmas;
+        decode_id(tile, e, m_blk, n0, mmas);
         const int row0 = s_seg[e] + m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
-        const int n0 = n_blk * NT;
         // The next tile id is taken when this tile's loads start (its latency hides behind
         // them), except during a CTA's first tile: then it is taken a few k-blocks before the
         // tile's last loads. Taking it at the start of the first tile let the CTAs that
@@ -326,11 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (PAIR) {
             // Both CTAs' bytes are counted on the MMA CTA's barrier.
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-            if (mma_cta) mbar_arrive_expect_tx(&full[stage], S::kTxBytes);
+            if (mma_cta)
+              mbar_arrive_expect_tx(&full[stage],
+                                    mmas == S::kMmas ? S::kTxBytes
+                                                     : 2 * (kABytes + 2 * mmas * kBoxBytes));
             tma_load_2d_pair_hint(a_dst, &tmA, bar, k0, row0, pol_a);
             // MMA h of the k-step reads boxes 2h, 2h+1 of each CTA.
-#pragma unroll
-            for (int h = 0; h < S::kMmas; ++h) {
+            for (int h = 0; h < mmas; ++h) {
               uint8_t* bh = b_dst + 2 * h * kBoxBytes;
               if (DUAL) {  // CTA 0 holds W1 columns [n0 + 128h, +128), CTA 1 the same of W2
                 const CUtensorMap* m = rank == 0 ? &tmB0 : &tmB1;
@@ -377,10 +406,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ring_release();
         ring_advance();
-        if (tile >= total_tiles) break;
+        if (tile >= work) break;
+        const int mmas = WIDE && tile >= first_half ? 1 : S::kMmas;  // a half tile: one MMA
         const int acc = it % S::kAccBufs;
         const uint32_t acc_phase = static_cast<uint32_t>(it / S::kAccBufs) & 1u;
-        // Wide tiles: tempty[0] / tempty[1] free the lower / upper 256 accumulator columns.
+        // Wide tiles: tempty[0] / tempty[1] free the lower / upper 256 accumulator columns
+        // (both are waited for on every tile, half tiles included, so that no epilogue warp
+        // can arrive for a tile before every warp has arrived for the one before).
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
           record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
           ok = false;
@@ -446,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after_sync();
           for (; kb < pre; ++kb) {
-            issue(kb, stage, 1, 2);
+            issue(kb, stage, 1, mmas);
             free_stage(stage);
             if (++stage == S::kStages) {
               stage = 0;
@@ -461,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after_sync();
-          issue(kb, stage, 0, S::kMmas);
+          issue(kb, stage, 0, mmas);
           free_stage(stage);
           if (++stage == S::kStages) {
             stage = 0;
@@ -493,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) ring_release();
       ring_advance();
-      if (tile >= total_tiles) break;
+      if (tile >= work) break;
       const int acc = it % S::kAccBufs;
       const uint32_t acc_phase = static_cast<uint32_t>(it / S::kAccBufs) & 1u;
       // The accumulator is ready only after the tile's whole main loop: suspend rather than
@@ -505,15 +537,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       tc_fence_after_sync();
-      int e, m_blk, n_blk;
-      decode(tile, e, m_blk, n_blk);
+      int e, m_blk, n0, mmas;
+      decode_id(tile, e, m_blk, n0, mmas);
       const int first_row = m_blk * S::kTileRows + static_cast<int>(rank) * kRows;
       const int rows = min(kRows, s_seg[e + 1] - s_seg[e] - first_row);
       // Row held by TMEM lane 32q + l (M = 64 tiles use lanes 0-15 of each quarter).
       const bool half = !PAIR && rows <= 64;
       auto tile_row = [&](int l) { return half ? (l < 16 ? 16 * q + l : kRows) : q * 32 + l; };
       const int64_t row0 = static_cast<int64_t>(s_seg[e]) + first_row;
-      const int n0 = n_blk * NT;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       // The accumulator is handed back to the MMA issuer as soon as this warp's last
@@ -527,6 +558,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (PAIR) mbar_arrive_cluster(tempty_mma0 + static_cast<uint32_t>((acc + part) * 8));
           else mbar_arrive(&tempty[acc + part]);
         }
+      };
+      // After the warp's last load: the whole accumulator (wide tiles: the upper half, and the
+      // lower half too for a half tile, which has not released it yet).
+      auto release_all = [&]() {
+        if (WIDE && mmas == 1) release_acc(0);
+        release_acc(WIDE ? 1 : 0);
       };
       // Output columns [n0 + 32c, +32) of the warp's 32 rows: each lane holds its row's 64 bytes.
       // They pass through the warp's 2 KB of shared memory so that each global store
@@ -559,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Output columns [32c, 32c + 32) of the tile: x W1 in accumulator columns
         // 256h + 32(c mod 4) and x W2 128 further, h = c / 4 (wide tiles have two halves);
         // each chunk is read as two 16-column pieces.
-        const int n_c = (4 * S::kMmas - c_first + 1) / 2;  // this warp's chunks
+        const int n_c = (4 * mmas - c_first + 1) / 2;  // this warp's chunks
         auto piece_col = [&](int cc, int half) {
           const int c = c_first + 2 * cc;
           return static_cast<uint32_t>(256 * (c >> 2) + 32 * (c & 3) + 16 * half);
@@ -584,18 +621,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_16cols(t_row + piece_col(cc, 1) + 128, rb1);
           act_pack(ra0, rb0, w);
           tmem_ld_wait();
-          if (WIDE && 2 * (cc + 1) == n_c) release_acc(0);  // the last chunk of the lower half
+          if (mmas == 2 && 2 * (cc + 1) == n_c) release_acc(0);  // the lower half is read
           if (cc + 1 < n_c) {
             tmem_ld_16cols(t_row + piece_col(cc + 1, 0), ra0);
             tmem_ld_16cols(t_row + piece_col(cc + 1, 0) + 128, rb0);
           } else {
-            release_acc(WIDE ? 1 : 0);
+            release_all();
           }
           act_pack(ra1, rb1, w + 8);
           store_chunk(w, c_first + 2 * cc);
         }
       } else {  // accumulator column j is output column n0 + j
-        const int n_c = (8 * S::kMmas - c_first + 1) / 2;  // this warp's chunks (even)
+        const int n_c = (8 * mmas - c_first + 1) / 2;  // this warp's chunks (even)
         auto pack = [&](const uint32_t (&ra)[32], uint32_t (&w)[16]) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -611,9 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pack(ra0, w);
           store_chunk(w, c_first + 2 * cc);
           tmem_ld_wait();
-          if (WIDE && 2 * (cc + 2) == n_c) release_acc(0);  // the last chunk of the lower half
+          if (mmas == 2 && 2 * (cc + 2) == n_c) release_acc(0);  // the lower half is read
           if (cc + 2 < n_c) tmem_ld_32cols(t_row + (c_first + 2 * (cc + 2)) * 32, ra0);
-          else release_acc(WIDE ? 1 : 0);
+          else release_all();
           pack(ra1, w);
           store_chunk(w, c_first + 2 * (cc + 1));
         }
@@ -780,6 +817,17 @@ int static_order() {
   return env != nullptr && std::strcmp(env, "static") == 0 ? 1 : 0;
 }
 
+// Half tiles (wide tiles only): the tiles of a last round that would keep at most half of the
+// pairs busy run as two half-width tiles each (default, 1); MOE_GEMM_HALVES=0 never splits,
+// MOE_GEMM_HALVES=all splits every tile (testing).
+int halves_mode() {
+  if (const char* env = std::getenv("MOE_GEMM_HALVES")) {
+    if (std::strcmp(env, "0") == 0) return 0;
+    if (std::strcmp(env, "all") == 0) return 2;
+  }
+  return 1;
+}
+
 // L2 priorities of the GEMM operands: an expert's A rows are read again by every column block
 // of that expert, its weights by the few row blocks running at the same time. Default: A rows
 // evict_last, weights evict_normal. MOE_GEMM_L2=<a>,<b> (each -1, 0 or 1) overrides.
@@ -818,10 +866,14 @@ cudaError_t launch_shape(const moe_problem& p, const CUtensorMap& a, const CUten
   const int64_t n_blocks = (gp.n_out + n_tile - 1) / n_tile;
   gp.n_group = column_group(pairs, n_blocks);
   gp.static_order = static_order();
+  gp.halves = wide ? halves_mode() : 0;
   l2_priorities(&gp.l2_a, &gp.l2_b);
   if (pairs) {
     const int64_t tiles = ((R + 255) / 256 + p.E) * n_blocks;
-    if (wide) return launch_gemm<DUAL, ACT, true, true>(a, b0, b1, gp, tiles, stream);
+    // half tiles: up to twice as many ids as tiles
+    if (wide)
+      return launch_gemm<DUAL, ACT, true, true>(a, b0, b1, gp, gp.halves ? 2 * tiles : tiles,
+                                                stream);
     return launch_gemm<DUAL, ACT, true, false>(a, b0, b1, gp, tiles, stream);
   }
   const int64_t tiles = ((R + 127) / 128 + p.E) * n_blocks;
