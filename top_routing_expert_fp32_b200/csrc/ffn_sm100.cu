@@ -195,9 +195,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int first_half = total_tiles - split;
   const int work = total_tiles + split;  // tile ids handed out
-  // More CTAs (pairs) than tile ids: the surplus ones take none; they only count themselves
+  // Single CTAs: only ceil(work / rounds) of them take tiles, rounds = ceil(work / units), so
+  // that every active CTA gets `rounds` tiles or one fewer and no last round runs on a few
+  // CTAs while the rest wait. Streaming (HBM-bound) tiles then share the bandwidth evenly to
+  // the end; compute-bound tiles take the same number of rounds either way.
+  const int rounds = (work + units - 1) / units;
+  const int active = PAIR ? units : (rounds > 0 ? (work + rounds - 1) / rounds : 0);
+  // CTAs (pairs) beyond the active ones take no tile id; they only count themselves
   // finished. Uniform over the block and over the pair.
-  if (cta_unit >= work) {
+  if (cta_unit >= active || cta_unit >= work) {
     if (threadIdx.x == 0 && mma_cta) sched_finish(p.sched, units);
     return;
   }
@@ -319,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&ring_full[r_slot]), 1));
           ring_advance();
           if (tile >= work) break;
-          if (p.static_order) next = tile + units;
+          if (p.static_order) next = tile + active;
         } else {
           if (!ring_take(tile)) {
             record_error(p.err, MOE_DEVERR_WAIT_TIMEOUT);
