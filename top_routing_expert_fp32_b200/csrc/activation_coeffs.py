@@ -1,4 +1,7 @@
-"""Coefficients of the exact-GELU evaluation in common.cuh (``gelu_erf``).
+"""Constants of the activations in common.cuh: the exact-GELU polynomial (``gelu_erf``) and
+the reciprocal seed of SiLU (``silu``).
+
+Exact GELU.
 
 GELU(x) = x * Phi(x) with Phi(x) = erfc(-x / sqrt 2) / 2. The kernels evaluate the upper tail
 q(x) = erfc(|x| / sqrt 2) / 2 and take Phi = q for x < 0 and 1 - q otherwise, so the negative
@@ -16,8 +19,16 @@ the base change for the hardware exponential and the halving:
 
     q = t * 2^(P(t) - x^2 * log2(e) / 2),   P(t) = log2(e) * p(t) - 1.
 
-Run ``python gelu_coeffs.py`` to print the initializer and the error of the fp32 Horner
-evaluation of P against float64 (as a relative error of q).
+SiLU. a / (1 + e^-a) takes the reciprocal of y = 1 + e^-a on the FMA pipe: a first
+approximation float(K - bits(y)) from y's bit pattern (subtracting the bits from a constant
+negates the exponent and roughly inverts the mantissa), then three Newton steps
+r <- r + r (1 - y r). K is chosen here to minimise the seed's largest relative error over two
+binades (the error pattern repeats every two); the three steps then leave at most about one
+ulp.
+
+Run ``python activation_coeffs.py`` to print the constants, the error of the fp32 Horner
+evaluation of P against float64 (as a relative error of q), and the seed's and the refined
+reciprocal's errors.
 """
 import numpy as np
 import numpy.polynomial.chebyshev as cheb
@@ -60,9 +71,37 @@ def max_rel_error_of_q(coef):
     return float(np.max(np.abs(err)) * np.log(2.0))
 
 
+def seed_error(K, y):
+    bits = y.astype(np.float32).view(np.int32).astype(np.int64)
+    r0 = (np.int64(K) - bits).astype(np.int32).view(np.float32).astype(np.float64)
+    return float(np.max(np.abs(r0 * y.astype(np.float32).astype(np.float64) - 1.0)))
+
+
+def reciprocal_seed():
+    """K minimising max |float(K - bits(y)) * y - 1| over y in [1, 4), coarse then fine."""
+    y = np.linspace(1.0, 4.0, 200001)
+    best = min(range(0x7EF00000, 0x7EF80000, 0x400), key=lambda K: seed_error(K, y))
+    return min(range(best - 0x400, best + 0x400, 4), key=lambda K: seed_error(K, y))
+
+
+def newton_reciprocal_f32(K, y):
+    """The kernel's reciprocal of fp32 y in fp32: the seed and three Newton steps."""
+    y = y.astype(np.float32)
+    r = (np.int64(K) - y.view(np.int32).astype(np.int64)).astype(np.int32).view(np.float32)
+    for _ in range(3):
+        e = (np.float32(1.0) - y.astype(np.float64) * r.astype(np.float64)).astype(np.float32)
+        r = (r.astype(np.float64) + r.astype(np.float64) * e.astype(np.float64)).astype(np.float32)
+    return r
+
+
 if __name__ == "__main__":
     coef = fit()
     print(f"// degree {DEGREE}, max relative error of q from P in fp32: "
           f"{max_rel_error_of_q(coef):.2e}")
     print("constexpr float kGeluP[%d] = {" % (DEGREE + 1))
     print("    " + ", ".join(f"{float(a):.9g}f" for a in coef) + "};")
+    K = reciprocal_seed()
+    y = np.concatenate([np.linspace(1.0, 2.0 ** 20, 400001), np.logspace(0, 37.9, 20001)])
+    r = newton_reciprocal_f32(K, y).astype(np.float64)
+    print(f"// reciprocal seed K = {K:#x}: seed error {seed_error(K, np.linspace(1, 4, 200001)):.4f}, "
+          f"after three Newton steps {np.max(np.abs(r * y.astype(np.float32) - 1.0)):.2e}")

@@ -361,7 +361,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // t = 1 / (1 + |x| / (2 sqrt 2)), erfc(z) = t exp(-z^2 + p(t)) (the form of Press et al.,
 // Numerical Recipes 6.2, "erfcc"), here in base 2 with the halving folded into P:
 //   q = t * 2^(P(t) - x^2 log2(e) / 2),   P = log2(e) p - 1, a degree-9 polynomial in t.
-// P's coefficients are a least-squares Chebyshev fit made by gelu_coeffs.py in this
+// P's coefficients are a least-squares Chebyshev fit made by activation_coeffs.py in this
 // directory. Relative error of the result against float64: 5e-7 for |x| < 1, 1.5e-6 for
 // -5 < x < -1, 7.6e-6 in the far negative tail (the rounding of x^2 log2(e) / 2). One
 // approximate reciprocal and one approximate exponential (both MUFU), 9 FMAs for P: about
@@ -390,13 +390,28 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return x * (x < 0.0f ? q : 1.0f - q);
 }
 
+// SiLU a / (1 + e^-a) with one MUFU operation (the exponential): the reciprocal of
+// y = 1 + e^-a runs on the FMA pipe, from a first approximation float(K - bits(y)) (K fitted by
+// activation_coeffs.py in this directory: 5.1 % relative error at most) and three Newton steps
+// r <- r + r (1 - y r), which leave about one ulp. The exponent is clamped at 126 so that y
+// stays finite: for a < -87.3 the result is a 2^-126 (magnitude below 1e-36 for |a| < 100)
+// instead of the underflowing a e^a. Relative error against float64: below 4e-7 for
+// |a| <= 5, below 1e-6 for |a| <= 14 (the rounding of a log2(e) grows with |a|). The
+// exponential and division form used two MUFU operations, the issue limit of the GEMM
+// epilogue on the SiLU layers.
+__device__ __forceinline__ float silu(float a) {
+  const float y = 1.0f + ex2_approx(fminf(a * -1.44269504088896341f, 126.0f));
+  float r = __int_as_float(0x7EF311C4 - __float_as_int(y));
+#pragma unroll
+  for (int i = 0; i < 3; ++i) r = fmaf(r, fmaf(-y, r, 1.0f), r);
+  return a * r;
+}
+
 // act(a) applied to the first up-projection (LLMs-from-scratch 12.1; Grok-1 book 5.3.5).
 template <int ACT>
 __device__ __forceinline__ float activation(float a) {
   if constexpr (ACT == MOE_ACT_SILU) {
-    // The quotient with the approximate reciprocal (2 ulp): the IEEE division sequence was
-    // the largest cost of the GEMM epilogue. For a -> -inf it gives -0, as a / inf does.
-    return __fdividef(a, 1.0f + expf(-a));
+    return silu(a);
   } else if constexpr (ACT == MOE_ACT_GELU_ERF) {
     return gelu_erf(a);
   } else {
