@@ -19,7 +19,11 @@
 //                   are never written). The accumulator is double buffered, so the epilogue
 //                   of tile i overlaps the main loop of tile i+1.
 // CTA pairs (cta_group::2, M=256) split A by rows and B by columns between the two CTAs; wide
-// pairs issue two N=256 MMAs per k-step into one 512-column accumulator (not double-buffered).
+// pairs issue two N=256 MMAs per k-step into one 512-column accumulator (not double-buffered:
+// the epilogue hands the lower 256 columns back first, and the next tile's MMAs into them start
+// on the k-blocks already loaded). A last round of wide tiles that would keep at most half of
+// the pairs busy runs as half tiles (one MMA per k-step, half the output columns). Single-CTA
+// launches run only the CTAs that an even split of the rounds needs.
 // Tiles: per expert ceil(M_e/128) row blocks x ceil(N/NT) column blocks. The column blocks
 // are cut into groups of G; tiles run group by group, inside a group expert by expert, then
 // column block, with row blocks innermost (consecutive CTAs share a weight column block
