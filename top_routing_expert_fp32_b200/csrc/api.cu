@@ -90,8 +90,8 @@ size_t elem_size(const moe_problem& p) { return p.dtype == MOE_DTYPE_BF16 ? 2 : 
 
 // Device workspace regions (byte offsets from the workspace base).
 struct Layout {
-  size_t err, colsum_part, zl_part, counts, idx, gate, pos, dropped, load, offsets, row_token,
-      xperm, h, y;
+  size_t err, colsum_part, zl_part, route_op, counts, idx, gate, pos, dropped, load, offsets,
+      row_token, xperm, h, y;
   size_t total;       // moe_forward and every other entry point
   size_t xin, xout;   // moe_forward_host / moe_forward_host_many
   size_t xin2, xout2; // second buffers of moe_forward_host_many
@@ -111,6 +111,7 @@ Layout make_layout(const moe_problem& p) {
   L.err = take(256);
   L.colsum_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)) * p.E);
   L.zl_part = take(sizeof(float) * static_cast<size_t>(route_num_blocks(p.N, p.E)));
+  L.route_op = take(route_tc_operand_bytes(p));
   L.counts = take(sizeof(int32_t) * static_cast<size_t>(dispatch_num_chunks(R)) * p.E);
   L.idx = take(sizeof(int32_t) * R);
   L.gate = take(sizeof(float) * R);
@@ -350,7 +351,7 @@ moe_status route_impl(const moe_problem& p, const void* X, const float* W_r, con
   }
   MOE_CUDA(launch_route(p, X, W_r, bias, noise, logits, topk_idx, topk_gate,
                         at<float>(ws, L.colsum_part), prob_colsum, at<float>(ws, L.zl_part), z_loss,
-                        at<int>(ws, L.err), wait_timeout_ns(), s),
+                        at<void>(ws, L.route_op), at<int>(ws, L.err), wait_timeout_ns(), s),
            "route");
   return MOE_OK;
 }

@@ -31,20 +31,27 @@ int route_num_blocks(int64_t N, int E);
 // Router logits + softmax + top-k + gates. X == nullptr: `logits` is an input.
 // colsum_partial: [route_num_blocks][E] floats (or nullptr when prob_colsum is nullptr).
 // noise: [N][E] (p.routing_mode != TOPK). zl_partial: [route_num_blocks] floats, used when
-// z_loss (device scalar) is requested.
+// z_loss (device scalar) is requested. operand: route_tc_operand_bytes(p) bytes of workspace
+// (256-byte aligned) for the tensor-core router's bf16 operand, or nullptr when that is 0.
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          const float* noise, float* logits, int32_t* idx, float* gate,
                          float* colsum_partial, float* prob_colsum, float* zl_partial,
-                         float* z_loss, int* err, uint64_t timeout_ns, cudaStream_t stream);
+                         float* z_loss, void* operand, int* err, uint64_t timeout_ns,
+                         cudaStream_t stream);
 
 // Tensor-core router for bf16 X (logits from a three-term bf16 split of W_r, made in the same
 // kernel, then the routing decision). colsum_partial may be nullptr; *grid_out = blocks that
 // wrote a colsum partial row.
+// With more than 16 experts the three bf16 terms of W_r are written once per call by a small
+// kernel into `operand` ([3 Ep rounded up to 16][D] bf16, route_tc_operand_bytes(p) bytes) and
+// loaded by TMA; with fewer the router splits each W_r slice itself in shared memory.
 bool route_tc_supported(const moe_problem& p);
+size_t route_tc_operand_bytes(const moe_problem& p);
 cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
                             const float* bias, const float* noise, float* logits_out,
                             int32_t* idx, float* gate, float* colsum_partial, float* zl_partial,
-                            int* grid_out, int* err, uint64_t timeout_ns, cudaStream_t stream);
+                            void* operand, int* grid_out, int* err, uint64_t timeout_ns,
+                            cudaStream_t stream);
 
 // 2-D bf16 tensor map (cols contiguous, row stride cols * 2 bytes), box box_cols x box_rows,
 // 128-byte swizzle, out-of-range elements read as zero.

@@ -571,7 +571,8 @@ int route_num_blocks(int64_t N, int E) {
 cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, const float* bias,
                          const float* noise, float* logits, int32_t* idx, float* gate,
                          float* colsum_partial, float* prob_colsum, float* zl_partial,
-                         float* z_loss, int* err, uint64_t timeout_ns, cudaStream_t stream) {
+                         float* z_loss, void* operand, int* err, uint64_t timeout_ns,
+                         cudaStream_t stream) {
   if (p.N == 0) return cudaSuccess;
   RouteArgs a;
   a.noise = p.routing_mode != MOE_ROUTE_TOPK ? noise : nullptr;
@@ -596,7 +597,7 @@ cudaError_t launch_route(const moe_problem& p, const void* X, const float* W_r, 
   if (X != nullptr && route_tc_supported(p)) {
     // bf16 activations: one tensor-core kernel computes the logits and routes.
     e = launch_route_tc(p, X, W_r, bias, a.noise, a.logits_out, idx, gate, a.colsum_partial,
-                        a.zl_partial, &grid, err, timeout_ns, stream);
+                        a.zl_partial, operand, &grid, err, timeout_ns, stream);
   } else if (kind == Kind::kSelect) {
     grid = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>((p.N + kSelThreads - 1) / kSelThreads, kMaxBlocks)));

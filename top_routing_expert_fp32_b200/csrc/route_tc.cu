@@ -19,7 +19,9 @@
 // stage; warps 6-9 turn that slice into the B operand (the three bf16 terms, in the
 // 128-byte-swizzled K-major layout the MMA reads; row i * Ep + e holds term i of expert e,
 // padding rows are zero) from shared memory, so no global latency sits between the
-// k-blocks; warp 1 issues the
+// k-blocks; with more than 16 experts a small kernel writes the three terms once per call
+// instead ([3 Ep, rounded up to 16][D] bf16 in the workspace) and warp 0 loads each k-block's
+// B by TMA beside X, so the loop no longer waits on the conversion; warp 1 issues the
 // tcgen05.mma, warps 2-5 are the epilogue: CTA r owns tokens [r*128/S, (r+1)*128/S) of the
 // tile; every epilogue thread stores its row's partial logits into the owner's shared memory
 // (a slot per source CTA, remote stores) and arrives there (release.cluster), and the owner
@@ -71,6 +73,7 @@ struct TcArgs {
   int NB;                  // MMA N: 3 * Ep rounded up to 16
   int zstride;             // floats per row of the partial-logit buffer (Ep + 4)
   int num_kb, S, num_clusters, stages;
+  int prepared;            // 1: B comes by TMA from the operand written by route_operand_kernel
   uint32_t stage_bytes, b_off, w_off, zbuf_off, sz_off, bar_off;
   int* err;
   uint64_t timeout_ns;
@@ -85,10 +88,35 @@ __device__ __forceinline__ void split3(float w, float& t0, float& t1, float& t2)
   t2 = r1 - t1;  // rounded to bf16 when packed
 }
 
+// The router's B operand for all of D, once per call: row n = i Ep + e holds term i of expert
+// e's column of W_r (k contiguous, the K-major rows a 128-byte-swizzled TMA box of 64 k
+// delivers to shared memory as the MMA reads them); rows e >= E of each term and rows past
+// 3 Ep are zero. One thread per element, consecutive threads along k.
+__global__ void route_operand_kernel(const float* __restrict__ W_r, int D, int E, int Ep, int NB,
+                                     __nv_bfloat16* __restrict__ out) {
+  pdl_wait();  // W_r and the workspace belong to the previous kernels until here
+  pdl_trigger();
+  const int64_t total = static_cast<int64_t>(NB) * D;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i / D);
+    const int d = static_cast<int>(i - static_cast<int64_t>(n) * D);
+    const int term = n / Ep, e = n - term * Ep;
+    float v = 0.f;
+    if (term < 3 && e < E) {
+      float t0, t1, t2;
+      split3(__ldg(W_r + static_cast<int64_t>(d) * E + e), t0, t1, t2);
+      v = term == 0 ? t0 : (term == 1 ? t1 : t2);
+    }
+    out[i] = __float2bfloat16_rn(v);
+  }
+}
+
 // EB: the experts the epilogue holds in registers per token (8, 16, 32 or 64; >= E).
 template <int EB>
 __global__ void __launch_bounds__(kThreads, 1)
-    route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const TcArgs a) {
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                    const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -116,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
-      mbar_init(&full[s], 1 + kConvWarps);  // the X copy (with its bytes), the B writers
+      // the X copy (with its bytes) and the B writers, or the X and B copies
+      mbar_init(&full[s], a.prepared ? 1 : 1 + kConvWarps);
       mbar_init(&empty[s], 1);
       mbar_init(&wfull[s], 1);
     }
@@ -131,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     fence_barrier_init();
     prefetch_tensormap(&tmX);
+    if (a.prepared) prefetch_tensormap(&tmB);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -141,7 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // every CTA's barriers exist before any remote arrival
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
-  const uint32_t tx_bytes = static_cast<uint32_t>(kABytes);
+  // X box, plus the B box (NB rows of 128 bytes) when B comes by TMA
+  const uint32_t tx_bytes = static_cast<uint32_t>(kABytes + (a.prepared ? a.NB * 128 : 0));
   pdl_wait();  // X, W_r and the outputs belong to the previous kernels until here
   pdl_trigger();
 
@@ -160,13 +191,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* dst = smem + stage * a.stage_bytes;
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
           tma_load_2d(dst, &tmX, &full[stage], kb * BK, static_cast<int>(tile * kRows));
-          // W_r rows [kb*64, kb*64 + rows) are one contiguous run of rows * E floats (a
-          // multiple of 32 bytes, since D % 8 == 0); the B writers convert it.
-          const int wrows = min(BK, a.D - kb * BK);
-          const uint32_t wbytes = static_cast<uint32_t>(wrows * a.E * 4);
-          mbar_arrive_expect_tx(&wfull[stage], wbytes);
-          bulk_g2s(dst + a.w_off, a.W_r + static_cast<int64_t>(kb) * BK * a.E, wbytes,
-                   &wfull[stage]);
+          if (a.prepared) {
+            tma_load_2d(dst + a.b_off, &tmB, &full[stage], kb * BK, 0);
+          } else {
+            // W_r rows [kb*64, kb*64 + rows) are one contiguous run of rows * E floats (a
+            // multiple of 32 bytes, since D % 8 == 0); the B writers convert it.
+            const int wrows = min(BK, a.D - kb * BK);
+            const uint32_t wbytes = static_cast<uint32_t>(wrows * a.E * 4);
+            mbar_arrive_expect_tx(&wfull[stage], wbytes);
+            bulk_g2s(dst + a.w_off, a.W_r + static_cast<int64_t>(kb) * BK * a.E, wbytes,
+                     &wfull[stage]);
+          }
           if (++stage == a.stages) {
             stage = 0;
             phase ^= 1u;
@@ -223,99 +258,101 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(drain, 0, a.timeout_ns)) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
     }
   } else if (warp >= 6) {  // ------------------------------------------ B operand writers
-    // Item (c, e): 8 consecutive k of expert e's W_r column (a 16-byte chunk c of the
-    // 128-byte K-major rows), split into its three bf16 terms, stored in rows e, Ep + e and
-    // 2 Ep + e at the 128-byte-swizzled position of chunk c (chunk c ^ (row & 7)). Lanes take
-    // consecutive e, so the fp32 reads are coalesced and each 8-lane phase of the 16-byte
-    // stores hits 8 distinct chunks.
-    const int ct = threadIdx.x - (kThreads - kConvThreads);
-    const int E = a.E;
-    const int items = 8 * E;
-    // Padding rows (e in [E, Ep) of each term, and rows past 3 Ep) stay zero: written once.
-    const int pad_rows = a.NB - 3 * E;
-    for (int s = 0; s < a.stages; ++s) {
-      uint8_t* b = smem + s * a.stage_bytes + a.b_off;
-      for (int i = ct; i < pad_rows * 8; i += kConvThreads) {
-        const int pr = i >> 3, c = i & 7;
-        int n;  // the pr-th padding row
-        if (pr < 3 * (a.Ep - E)) n = (pr / (a.Ep - E)) * a.Ep + E + pr % (a.Ep - E);
-        else n = 3 * a.Ep + (pr - 3 * (a.Ep - E));
-        *reinterpret_cast<uint4*>(b + n * 128 + ((c ^ (n & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+    if (!a.prepared) {  // (with the prepared operand B comes by TMA: nothing to convert)
+      // Item (c, e): 8 consecutive k of expert e's W_r column (a 16-byte chunk c of the
+      // 128-byte K-major rows), split into its three bf16 terms, stored in rows e, Ep + e and
+      // 2 Ep + e at the 128-byte-swizzled position of chunk c (chunk c ^ (row & 7)). Lanes take
+      // consecutive e, so the fp32 reads are coalesced and each 8-lane phase of the 16-byte
+      // stores hits 8 distinct chunks.
+      const int ct = threadIdx.x - (kThreads - kConvThreads);
+      const int E = a.E;
+      const int items = 8 * E;
+      // Padding rows (e in [E, Ep) of each term, and rows past 3 Ep) stay zero: written once.
+      const int pad_rows = a.NB - 3 * E;
+      for (int s = 0; s < a.stages; ++s) {
+        uint8_t* b = smem + s * a.stage_bytes + a.b_off;
+        for (int i = ct; i < pad_rows * 8; i += kConvThreads) {
+          const int pr = i >> 3, c = i & 7;
+          int n;  // the pr-th padding row
+          if (pr < 3 * (a.Ep - E)) n = (pr / (a.Ep - E)) * a.Ep + E + pr % (a.Ep - E);
+          else n = 3 * a.Ep + (pr - 3 * (a.Ep - E));
+          *reinterpret_cast<uint4*>(b + n * 128 + ((c ^ (n & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
-    }
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int64_t tile = first_tile; ok && tile < a.tiles; tile += a.num_clusters) {
-      for (int kb = kb0; kb < kb1; ++kb) {
-        // The slice lands after the producer has seen this stage free (empty), so waiting for
-        // it also orders these stores after the MMAs that read the stage's previous B.
-        if (!mbar_wait(&wfull[stage], phase, a.timeout_ns)) {
-          if (lane == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
-          ok = false;
-          break;
-        }
-        uint8_t* b = smem + stage * a.stage_bytes + a.b_off;
-        const float* wf = reinterpret_cast<const float*>(smem + stage * a.stage_bytes + a.w_off);
-        const int wrows = min(BK, a.D - kb * BK);
-        // Item (c, e) -> its three 16-byte chunks of B.
-        auto convert_store = [&](int i, const float (&wv)[8]) {
-          const int c = i / E, e = i - c * E;
-          float t0[8], t1[8], t2[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) split3(wv[j], t0[j], t1[j], t2[j]);
-          const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
-                                      pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
-          const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
-                                      pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
-          const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
-                                      pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
-          const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
-          *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
-          *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
-          *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
-        };
-        if (items <= kConvThreads) {  // E <= 16: at most one item per thread
-          if (ct < items) {
-            const int c = ct / E, e = ct - c * E;
-            float wv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int d = c * 8 + j;
-              wv[j] = d < wrows ? wf[d * E + e] : 0.f;
-            }
-            convert_store(ct, wv);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t tile = first_tile; ok && tile < a.tiles; tile += a.num_clusters) {
+        for (int kb = kb0; kb < kb1; ++kb) {
+          // The slice lands after the producer has seen this stage free (empty), so waiting for
+          // it also orders these stores after the MMAs that read the stage's previous B.
+          if (!mbar_wait(&wfull[stage], phase, a.timeout_ns)) {
+            if (lane == 0) record_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
+            ok = false;
+            break;
           }
-        }
-        // Larger E: kBatch items per thread at a time, all their loads first (independent
-        // chains for the scheduler; E = 64 gives each thread 4 items per k-block).
-        constexpr int kBatch = 4;
-        for (int i0 = items <= kConvThreads ? items : ct; i0 < items;
-             i0 += kBatch * kConvThreads) {
-          float w[kBatch][8];
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u * kConvThreads;
+          uint8_t* b = smem + stage * a.stage_bytes + a.b_off;
+          const float* wf = reinterpret_cast<const float*>(smem + stage * a.stage_bytes + a.w_off);
+          const int wrows = min(BK, a.D - kb * BK);
+          // Item (c, e) -> its three 16-byte chunks of B.
+          auto convert_store = [&](int i, const float (&wv)[8]) {
             const int c = i / E, e = i - c * E;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int d = c * 8 + j;
-              w[u][j] = (i < items && d < wrows) ? wf[d * E + e] : 0.f;
+            float t0[8], t1[8], t2[8];
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) split3(wv[j], t0[j], t1[j], t2[j]);
+            const uint4 v0 = make_uint4(pack_bf16x2(t0[0], t0[1]), pack_bf16x2(t0[2], t0[3]),
+                                        pack_bf16x2(t0[4], t0[5]), pack_bf16x2(t0[6], t0[7]));
+            const uint4 v1 = make_uint4(pack_bf16x2(t1[0], t1[1]), pack_bf16x2(t1[2], t1[3]),
+                                        pack_bf16x2(t1[4], t1[5]), pack_bf16x2(t1[6], t1[7]));
+            const uint4 v2 = make_uint4(pack_bf16x2(t2[0], t2[1]), pack_bf16x2(t2[2], t2[3]),
+                                        pack_bf16x2(t2[4], t2[5]), pack_bf16x2(t2[6], t2[7]));
+            const int n0 = e, n1 = a.Ep + e, n2 = 2 * a.Ep + e;
+            *reinterpret_cast<uint4*>(b + n0 * 128 + ((c ^ (n0 & 7)) << 4)) = v0;
+            *reinterpret_cast<uint4*>(b + n1 * 128 + ((c ^ (n1 & 7)) << 4)) = v1;
+            *reinterpret_cast<uint4*>(b + n2 * 128 + ((c ^ (n2 & 7)) << 4)) = v2;
+          };
+          if (items <= kConvThreads) {  // E <= 16: at most one item per thread
+            if (ct < items) {
+              const int c = ct / E, e = ct - c * E;
+              float wv[8];
+  #pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int d = c * 8 + j;
+                wv[j] = d < wrows ? wf[d * E + e] : 0.f;
+              }
+              convert_store(ct, wv);
             }
           }
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u * kConvThreads;
-            if (i >= items) break;
-            convert_store(i, w[u]);
+          // Larger E: kBatch items per thread at a time, all their loads first (independent
+          // chains for the scheduler; E = 64 gives each thread 4 items per k-block).
+          constexpr int kBatch = 4;
+          for (int i0 = items <= kConvThreads ? items : ct; i0 < items;
+               i0 += kBatch * kConvThreads) {
+            float w[kBatch][8];
+  #pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int i = i0 + u * kConvThreads;
+              const int c = i / E, e = i - c * E;
+  #pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int d = c * 8 + j;
+                w[u][j] = (i < items && d < wrows) ? wf[d * E + e] : 0.f;
+              }
+            }
+  #pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int i = i0 + u * kConvThreads;
+              if (i >= items) break;
+              convert_store(i, w[u]);
+            }
           }
-        }
-        fence_proxy_async_smem();  // generic-proxy stores before the MMA (async proxy) reads
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == a.stages) {
-          stage = 0;
-          phase ^= 1u;
+          fence_proxy_async_smem();  // generic-proxy stores before the MMA (async proxy) reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[stage]);
+          if (++stage == a.stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
     }
@@ -477,6 +514,9 @@ struct TcShape {
   uint32_t stage_bytes, b_off, w_off, zbuf_off, sz_off, bar_off, smem_bytes;
 };
 
+// More than 16 experts: the B operand is written once per call and loaded by TMA.
+bool prepared_operand(int E) { return E > 16; }
+
 TcShape tc_shape(int64_t N, int D, int E) {
   TcShape s{};
   s.Ep = (E + 7) / 8 * 8;
@@ -498,10 +538,12 @@ TcShape tc_shape(int64_t N, int D, int E) {
   }
   s.num_clusters = static_cast<int>(
       std::max<int64_t>(1, std::min<int64_t>(s.tiles, kUnitTarget / s.S)));
-  // Shared memory: [stages][A 16 KB | B (bf16 terms) | W (fp32 slice, 64 x E)]
-  // [partials 128 x zstride] [summed logits] [barriers]; A and B 1024-byte aligned.
+  // Shared memory: [stages][A 16 KB | B (bf16 terms) | W (fp32 slice, 64 x E; not with the
+  // prepared operand)] [partials 128 x zstride] [summed logits] [barriers]; A and B
+  // 1024-byte aligned.
   const uint32_t b_bytes = static_cast<uint32_t>((s.NB * BK * 2 + 1023) / 1024 * 1024);
-  const uint32_t w_bytes = static_cast<uint32_t>((BK * E * 4 + 1023) / 1024 * 1024);
+  const uint32_t w_bytes =
+      prepared_operand(E) ? 0u : static_cast<uint32_t>((BK * E * 4 + 1023) / 1024 * 1024);
   s.b_off = kABytes;
   s.w_off = kABytes + b_bytes;
   s.stage_bytes = kABytes + b_bytes + w_bytes;
@@ -524,20 +566,48 @@ bool route_tc_supported(const moe_problem& p) {
   return p.dtype == MOE_DTYPE_BF16 && p.E <= kMaxEc;
 }
 
+size_t route_tc_operand_bytes(const moe_problem& p) {
+  if (!route_tc_supported(p) || !prepared_operand(p.E) || p.E < 1) return 0;
+  const TcShape s = tc_shape(1, static_cast<int>(p.D), p.E);
+  return static_cast<size_t>(s.NB) * static_cast<size_t>(p.D) * 2;
+}
+
 cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_r,
                             const float* bias, const float* noise, float* logits_out,
                             int32_t* idx, float* gate, float* colsum_partial, float* zl_partial,
-                            int* grid_out, int* err, uint64_t timeout_ns, cudaStream_t stream) {
+                            void* operand, int* grid_out, int* err, uint64_t timeout_ns,
+                            cudaStream_t stream) {
   const TcShape s = tc_shape(p.N, static_cast<int>(p.D), p.E);
   *grid_out = 0;
   if (p.N == 0) return cudaSuccess;
   if (s.stages < 2) return cudaErrorInvalidConfiguration;
   const int D = static_cast<int>(p.D);
-  CUtensorMap tX;
+  const bool prepared = prepared_operand(p.E);
+  if (prepared && operand == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap tX, tB;
   if (!make_tensor_map_2d_bf16(&tX, X, static_cast<uint64_t>(D), static_cast<uint64_t>(p.N), 64,
                                kRows))
     return cudaErrorInvalidValue;
+  tB = tX;  // unused unless prepared
   cudaError_t e = cudaSuccess;
+  if (prepared) {
+    // The B operand [NB][D] bf16, rows 128 bytes apart in each 64-k box (128-byte swizzle).
+    if (!make_tensor_map_2d_bf16(&tB, operand, static_cast<uint64_t>(D),
+                                 static_cast<uint64_t>(s.NB), 64, static_cast<uint32_t>(s.NB)))
+      return cudaErrorInvalidValue;
+    const int64_t total = static_cast<int64_t>(s.NB) * D;
+    const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * num_sms()));
+    cudaLaunchConfig_t ocfg = {};
+    ocfg.gridDim = dim3(static_cast<unsigned>(std::max(blocks, 1)));
+    ocfg.blockDim = dim3(256);
+    ocfg.stream = stream;
+    cudaLaunchAttribute oattr[1];
+    ocfg.attrs = oattr;
+    ocfg.numAttrs = pdl_attr(&oattr[0]);
+    e = cudaLaunchKernelEx(&ocfg, route_operand_kernel, W_r, D, p.E, s.Ep, s.NB,
+                           static_cast<__nv_bfloat16*>(operand));
+    if (e != cudaSuccess) return e;
+  }
   TcArgs a;
   a.W_r = W_r;
   a.bias = bias;
@@ -561,6 +631,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   a.S = s.S;
   a.num_clusters = s.num_clusters;
   a.stages = s.stages;
+  a.prepared = prepared ? 1 : 0;
   a.stage_bytes = s.stage_bytes;
   a.b_off = s.b_off;
   a.w_off = s.w_off;
@@ -569,7 +640,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   a.bar_off = s.bar_off;
   a.err = err;
   a.timeout_ns = timeout_ns;
-  void (*kern)(const CUtensorMap, const TcArgs) =
+  void (*kern)(const CUtensorMap, const CUtensorMap, const TcArgs) =
       s.Ep <= 8 ? route_tc_kernel<8>
                 : (s.Ep <= 16 ? route_tc_kernel<16> : (s.Ep <= 32 ? route_tc_kernel<32> : route_tc_kernel<64>));
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -587,7 +658,7 @@ cudaError_t launch_route_tc(const moe_problem& p, const void* X, const float* W_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1 + pdl_attr(&attr[1]);
-  e = cudaLaunchKernelEx(&cfg, kern, tX, a);
+  e = cudaLaunchKernelEx(&cfg, kern, tX, tB, a);
   if (e != cudaSuccess) return e;
   *grid_out = s.num_clusters * s.S;
   return cudaGetLastError();
