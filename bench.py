@@ -390,9 +390,12 @@ def run_gpu(args, cfg, world, rank, device):
     stream = torch.cuda.current_stream(device)
 
     names = ["route", "dispatch", "up", "down", "combine"]
-    # Kernels per step: one router (tensor-core for bf16 X, SIMT for fp32 X), one cooperative
-    # dispatch (count, slot assignment and gather), one launch each for up, down, combine.
-    launches = {"route": 1, "dispatch": 1, "up": 1, "down": 1, "combine": 1}
+    # Kernels per step: one router (tensor-core for bf16 X, SIMT for fp32 X; with bf16 X and
+    # more than 16 experts a small kernel writes the router's bf16 operand first), one
+    # cooperative dispatch (count, slot assignment and gather), one launch each for up, down,
+    # combine.
+    route_launches = 2 if (cfg.dtype == configs.DTYPE_BF16 and cfg.E > 16) else 1
+    launches = {"route": route_launches, "dispatch": 1, "up": 1, "down": 1, "combine": 1}
 
     def step(ev):
         ev[0].record()
@@ -793,7 +796,9 @@ def run_gpu_ep(args, cfg, world, rank, device):
         et += e0v.elapsed_time(e1v)
     e_max = reduce_max(et, device)
     barrier(device)
-    launches = 1 + 1 + 2 + 2 + 1  # route, dispatch, 2 reorders, up + down, combine
+    # route (plus the router operand with bf16 X and more than 16 experts), dispatch,
+    # 2 reorders, up + down, combine
+    launches = (2 if (cfg.dtype == configs.DTYPE_BF16 and cfg.E > 16) else 1) + 1 + 2 + 2 + 1
     return {
         "metric": METRIC, "value": agg["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": agg["ms_per_step"],
