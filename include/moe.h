@@ -136,8 +136,10 @@ typedef struct {
 moe_status moe_capacity(const moe_problem* p, int64_t* C);
 
 /* Host only. Bytes of workspace every entry point below accepts for problem p (one size for
- * all of them). The workspace holds the device error word, scratch counters and, for
- * moe_forward, the intermediate buffers (routing results, X_perm, H, Y). */
+ * all of them). The workspace holds the device error word, scratch counters, the router's
+ * bf16 operand (bf16 X with more than 16 experts: the three bf16 terms of W_r, written by each
+ * router call) and, for moe_forward, the intermediate buffers (routing results, X_perm, H,
+ * Y). */
 moe_status moe_workspace_size(const moe_problem* p, size_t* bytes);
 
 /* Router + softmax + top-k + gates (Grok-1 book 5.2, 5.2.3; walkthrough 1.1, 1.2;
