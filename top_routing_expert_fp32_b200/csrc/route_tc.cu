@@ -12,7 +12,7 @@
 // concatenated [w0 | w1 | w2] columns gives the three partial dot products; they are added
 // smallest first, z = (z2 + z1) + z0.
 //
-// Kernel (one launch per call): route_tc_kernel, clusters of S CTAs (S = 1, 2, 4 or 8),
+// Kernel (one launch per call; two with more than 16 experts): route_tc_kernel, clusters of S CTAs (S = 1, 2, 4 or 8),
 // persistent over 128-token tiles; CTA r of a cluster accumulates the r-th slice of D
 // (split-K), so that a batch of few tiles still spreads over the SMs. Warp 0 issues the TMA
 // loads of X and a bulk copy of the k-block's fp32 W_r slice (64 x E, contiguous) into the
