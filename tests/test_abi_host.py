@@ -100,6 +100,29 @@ def test_workspace_size_covers_intermediates(abi):
     assert abi.workspace_size(p0) >= 256
 
 
+def test_workspace_size_covers_the_router_operand(abi):
+    # bf16 X with more than 16 experts: the router writes the three bf16 terms of W_r, rows
+    # 3 Ep rounded up to 16 by D, into the workspace once per call; 16 experts or fewer (and
+    # fp32 X) need no such region.
+    from top_routing_expert_fp32_b200 import configs
+    cfg = configs.CONFIGS["capacity"]
+    D, E = cfg.D, cfg.E
+    nb = -(-3 * (-(-E // 8) * 8) // 16) * 16
+    with64 = abi.workspace_size(abi.problem(cfg))
+    def variant(name, E_, dtype):
+        return configs.MoEConfig(name, N=cfg.N, D=D, F=cfg.F, E=E_, k=cfg.k, dtype=dtype,
+                                 activation=cfg.activation, renormalize=cfg.renormalize,
+                                 capacity_factor=cfg.capacity_factor)
+    cfg16 = variant("e16", 16, configs.DTYPE_BF16)
+    cfg17 = variant("e17", 17, configs.DTYPE_BF16)
+    n16 = abi.workspace_size(abi.problem(cfg16))
+    n17 = abi.workspace_size(abi.problem(cfg17))
+    assert n17 - n16 >= (-(-3 * 24 // 16) * 16) * D * 2      # E = 17: Ep = 24, 80 rows
+    assert with64 >= nb * D * 2 + 2 * cfg.N * cfg.k * (2 * D + cfg.F)
+    n32 = abi.workspace_size(abi.problem(variant("f32", 64, configs.DTYPE_F32)))
+    assert n32 >= 4 * cfg.N * cfg.k * (2 * D + cfg.F)   # fp32 intermediates, no operand
+
+
 def _call_route(abi, p, ws=None, ws_bytes=0, X=None, W_r=None, logits=None, idx=8, gate=8):
     return abi.lib.moe_route(ctypes.byref(p), X, W_r, None, logits, idx, gate, None, ws,
                              ws_bytes, None)
